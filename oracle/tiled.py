@@ -1,0 +1,64 @@
+"""Tiled online-softmax attention in plain float64 Python, for tiny inputs.
+
+TEST INFRASTRUCTURE ONLY (see `oracle/attention.py`). It exists to check the pages'
+exactness claim: processing the keys tile by tile with a running maximum and a running
+normaliser gives the same result as the untiled definition (page "Kotaemon
+FlashAttention", algorithm bullets: Q split into row blocks, K_j/V_j blocks loaded per
+row block, running max and normaliser updated, result identical to the original).
+
+It follows the pages' outer/inner loop order (page "Flash Attention ... IO-aware exact"
+(fr), tiling pseudo-code: loop over row blocks Q_i, load K_j and V_j, form
+S_ij = Q_i K_j^T / sqrt(d), accumulate O_i, write O_i once at the end and return O and
+L). That listing is garbled: it has no loop over j, leaves Tr undefined and applies a
+local softmax to each tile with a plain ``+=``. The reading taken here, stated in the
+pages' own terms elsewhere (page "Flash Attention" (zh), online-softmax bullet), is the
+running-max rescale: for every tile,
+
+    m_new = max(m, rowmax(S_ij));  alpha = exp(m - m_new)
+    P_ij  = exp(S_ij - m_new);     l = alpha * l + rowsum(P_ij)
+    O_i   = alpha * O_i + P_ij V_j
+
+and after the last tile ``O_i / l`` and ``L_i = m + log(l)``. Tr = ceil(Nq/Br),
+Tc = ceil(Nk/Bc); masked scores are -inf.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .attention import _f64, visible_mask
+
+__all__ = ["tiled_attention_f64"]
+
+
+def tiled_attention_f64(Q, K, V, causal: bool, scale: float, Br: int, Bc: int):
+    """One head: Q [Nq,d], K and V [Nk,d]. Returns O [Nq,d] and L [Nq] (float64)."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    Nq, d = Q.shape
+    Nk = K.shape[0]
+    Tr = -(-Nq // Br)
+    Tc = -(-Nk // Bc)
+    O = np.zeros((Nq, d))
+    L = np.full(Nq, -np.inf)
+    for i in range(Tr):
+        r0, r1 = i * Br, min(Nq, (i + 1) * Br)
+        Qi = Q[r0:r1]
+        Oi = np.zeros((r1 - r0, d))
+        li = np.zeros(r1 - r0)
+        mi = np.full(r1 - r0, -np.inf)
+        for j in range(Tc):
+            c0, c1 = j * Bc, min(Nk, (j + 1) * Bc)
+            Kj, Vj = K[c0:c1], V[c0:c1]
+            Sij = scale * (Qi @ Kj.T)
+            vis = visible_mask(np.arange(r0, r1), Nq, Nk, causal)[:, c0:c1]
+            Sij = np.where(vis, Sij, -np.inf)
+            m_new = np.maximum(mi, Sij.max(axis=1))
+            ref = np.where(np.isfinite(m_new), m_new, 0.0)   # rows with nothing visible yet
+            alpha = np.where(np.isfinite(mi), np.exp(mi - ref), 0.0)
+            Pij = np.exp(Sij - ref[:, None])
+            li = alpha * li + Pij.sum(axis=1)
+            Oi = alpha[:, None] * Oi + Pij @ Vj
+            mi = m_new
+        seen = li > 0
+        O[r0:r1][seen] = Oi[seen] / li[seen, None]
+        L[r0:r1][seen] = mi[seen] + np.log(li[seen])
+    return O, L
