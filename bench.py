@@ -1,0 +1,369 @@
+"""Benchmark of the exact-attention hot path on B200.
+
+One step = one pass over the whole path on one batch of synthetic input:
+  * fa_fwd on the causal self-attention workload B=8 H=12 N=2048 d=64 fp16 (O and LSE),
+  * fa_decode on the GQA decode workload B=64 Hq=32 Hkv=8 d=128 bf16, kv_len ~ U[512,4096].
+`value` is the forward's throughput in TFLOP/s (algorithmic, causal-adjusted FLOPs:
+4*d per visible query-key pair); the decode's KV-read GB/s is reported beside it.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun (N > 1) each rank runs an independent replica (the path needs no
+collective); the barrier and the max-over-ranks time are the only communication.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, decode_kv_bytes, fwd_flops, make_decode_inputs, make_fwd_inputs  # noqa: E402
+
+METRIC = "attn fwd TFLOP/s & % BF16 TC peak; decode KV-read GB/s & % HBM peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------------------
+# Clock sampling during the timed region (NVML, read-only)
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = [("gpu_idle", 0x1), ("applications_clocks_setting", 0x2), ("sw_power_cap", 0x4),
+               ("hw_slowdown", 0x8), ("sync_boost", 0x10), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80)]
+
+    def __init__(self, cuda_index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = self._handle(cuda_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report the clocks as unavailable
+            self.nvml, self.error = None, f"{type(e).__name__}: {e}"
+
+    def _handle(self, idx):
+        import torch
+        pynvml = self.nvml
+        try:
+            uuid = str(torch.cuda.get_device_properties(idx).uuid)
+            for u in (uuid, "GPU-" + uuid):
+                try:
+                    return pynvml.nvmlDeviceGetHandleByUUID(u)
+                except Exception:
+                    pass
+        except Exception:
+            pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            try:
+                idx = int(vis.split(",")[idx])
+            except Exception:
+                pass
+        return pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        p = self.nvml
+        get_reasons = getattr(p, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(p, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self._stop.is_set():
+            try:
+                self.samples.append(p.nvmlDeviceGetClockInfo(self.handle, p.NVML_CLOCK_SM))
+                self.reasons |= int(get_reasons(self.handle))
+            except Exception as e:
+                self.error = str(e)
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "note": self.error or "no samples"}
+        names = [n for n, bit in self.REASONS if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------
+def oracle_cpu_baseline(w, budget_s: float):
+    """Time the float64 oracle as it stands on this host on a bounded sample of the forward
+    workload's heads (whole (batch, head) problems, in order, until `budget_s` elapses)."""
+    import numpy as np
+    from oracle import attention_rows_f64
+    q, k, v = make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed)
+    rows = np.arange(w.N)
+    heads, t0 = 0, time.perf_counter()
+    for b in range(w.B):
+        for h in range(w.Hq):
+            attention_rows_f64(q, k, v, w.causal, w.scale, b, h, rows)
+            heads += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        else:
+            continue
+        break
+    el = time.perf_counter() - t0
+    flops = fwd_flops(1, 1, w.N, w.N, w.d, w.causal) * heads
+    cores = len(os.sched_getaffinity(0))
+    return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{heads} of {w.B * w.Hq} (batch, head) problems of {w.describe()}, "
+                      f"float64 NumPy, {el:.1f} s"}
+
+
+def run_reference(args):
+    """Reference arm: the float64 CPU oracle as it stands, on rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    import numpy as np
+    from oracle import attention_rows_f64
+    q, k, v = make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed)
+    rows = np.arange(w.N)
+    per_step = max(1, args.ref_heads_per_step)
+    order = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+
+    def step(i):
+        for j in range(per_step):
+            b, h = order[(i * per_step + j) % len(order)]
+            attention_rows_f64(q, k, v, w.causal, w.scale, b, h, rows)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    el = time.perf_counter() - t0
+    flops = fwd_flops(1, 1, w.N, w.N, w.d, w.causal) * per_step * args.steps
+    val = flops / el / 1e12
+    cores = len(os.sched_getaffinity(0))
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.describe(), "parallelism": "single process, host cores",
+                       "sample_per_step": f"{per_step} (batch, head) problems of the workload"},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{per_step} (batch, head) problems per step"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import io_aware_exact_28_b200 as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    peaks, peak_src = load_peaks()
+    w = WORKLOADS[args.workload]
+    wd = WORKLOADS[args.decode_workload]
+
+    # Inputs (seeded, CPU-generated), resident on the device before timing.
+    q, k, v = (t.to(dev) for t in make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    kv_lens_cpu, dq, kc, vc = make_decode_inputs(wd.B, wd.Hq, wd.Hkv, wd.N, wd.d, wd.dtype,
+                                                 wd.kv_len_lo, wd.kv_len_hi, wd.seed)
+    kv_lens, dq, kc, vc = kv_lens_cpu.to(dev), dq.to(dev), kc.to(dev), vc.to(dev)
+    do = torch.empty_like(dq)
+    dlse = torch.empty((wd.B, wd.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.decode_workspace_bytes(wd.B, wd.Hq, wd.N, wd.d), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    fl = fwd_flops(w.B, w.Hq, w.N, w.N, w.d, w.causal)
+    fwd_bytes = 2 * (2 * q.numel() + 2 * k.numel()) + 4 * lse.numel()   # Q,K,V read, O write, LSE
+    kv_bytes = decode_kv_bytes(kv_lens_cpu, wd.Hkv, wd.d)
+    dec_bytes = kv_bytes + 2 * (dq.numel() + do.numel()) + 4 * dlse.numel()
+
+    def fwd_call():
+        fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+
+    def dec_call():
+        fa.decode(dq, kc, vc, kv_lens, scale=wd.scale, out=do, lse=dlse, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd_call()
+        dec_call()
+    torch.cuda.synchronize()
+    if fa.device_status() != fa.FA_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for i in range(K):
+        flush.zero_()                 # L2 flush between steps, outside the timed events
+        ev[i][0].record()
+        fwd_call()
+        ev[i][1].record()
+        ev[i][2].record()             # decode inputs (1 GiB+) exceed L2 by themselves
+        dec_call()
+        ev[i][3].record()
+    torch.cuda.synchronize()
+    sampler.stop()
+    if world > 1:
+        dist.barrier()
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    dec_ms = sum(e[2].elapsed_time(e[3]) for e in ev)
+    t = torch.tensor([fwd_ms, dec_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    fwd_ms, dec_ms = float(t[0]), float(t[1])
+    status = fa.device_status()
+
+    fwd_tflops = world * K * fl / (fwd_ms * 1e-3) / 1e12
+    dec_gbs = world * K * dec_bytes / (dec_ms * 1e-3) / 1e9
+    fwd_avg_s = fwd_ms / K * 1e-3
+    dec_avg_s = dec_ms / K * 1e-3
+    roof_fwd = {"kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": fl / fwd_avg_s / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": fl / fwd_avg_s / 1e12 / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": f"{peak_src} dense bf16 burst (fp16 dense rate is the same)",
+                "algorithmic_flops_per_launch": fl, "algorithmic_bytes_per_launch": fwd_bytes}
+    roof_dec = {"kernel": "fa_decode (split + combine)", "bound": "hbm",
+                "achieved": dec_bytes / dec_avg_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": dec_bytes / dec_avg_s / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peak_src} HBM copy bandwidth",
+                "algorithmic_bytes_per_launch": dec_bytes, "kv_bytes_per_launch": kv_bytes}
+    dominant = roof_fwd if fwd_ms >= dec_ms else roof_dec
+
+    # End to end through the public API: host (pinned) inputs in, host outputs back.
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        dq2, dk2, dv2 = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        E = max(3, min(K, 50))
+
+        def e2e_step():
+            dq2.copy_(hq, non_blocking=True)
+            dk2.copy_(hk, non_blocking=True)
+            dv2.copy_(hv, non_blocking=True)
+            fa.fwd(dq2, dk2, dv2, causal=w.causal, scale=w.scale, out=o, lse=lse)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(E):
+            e2e_step()
+        s1.record()
+        torch.cuda.synchronize()
+        tt = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * E * fl / (float(tt[0]) * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 2 * (q.numel() + k.numel() + v.numel()),
+               "d2h_bytes_per_step": 2 * o.numel() + 4 * lse.numel(), "steps": E,
+               "path": "fa.fwd (C ABI fa_fwd) with pinned host buffers, copies on the same stream"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_cpu_baseline(w, args.cpu_budget_s)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": fwd_tflops, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": (fwd_ms + dec_ms) / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.describe(), "decode_workload": wd.describe(),
+                       "l2": "flushed (256 MiB write) before each step; decode caches exceed L2",
+                       "parallelism": "replicas" if world > 1 else "single GPU",
+                       "value_is": "forward TFLOP/s, causal-adjusted algorithmic FLOPs"},
+            "fwd": {"tflops": fwd_tflops, "ms_per_launch": fwd_ms / K,
+                    "frac_of_measured_bf16_peak": roof_fwd["frac"],
+                    "frac_of_spec_2250_tflops": fl / fwd_avg_s / 1e12 / 2250.0},
+            "decode": {"value": dec_gbs, "unit": "GB/s", "ms_per_launch": dec_ms / K,
+                       "dtype": wd.dtype, "frac_of_measured_hbm": roof_dec["frac"],
+                       "frac_of_spec_8000_gbs": dec_bytes / dec_avg_s / 1e9 / 8000.0},
+            "roofline": dominant, "rooflines": [roof_fwd, roof_dec],
+            "e2e": e2e, "cpu_baseline": cpu,
+            "gpu_launches": K * 3,
+            "gpu_launches_note": "per step: 1 fa_fwd_kernel + fa_decode_split_kernel + fa_decode_combine_kernel",
+            "clocks": sampler.summary(),
+            "device_status": fa.status_string(status),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mha2k", choices=[k for k, v in WORKLOADS.items() if v.kind == "fwd"])
+    ap.add_argument("--decode-workload", default="decode")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--ref-heads-per-step", type=int, default=2)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

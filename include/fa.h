@@ -1,0 +1,156 @@
+/*
+ * fa.h — C ABI of the B200 exact-attention library (libfa_b200.so).
+ *
+ * The library computes exact scaled-dot-product attention
+ *     O = softmax(scale * Q K^T) V,    LSE_i = log(sum_j exp(scale * q_i . k_j))
+ * tile by tile with an online softmax, so the score matrix never reaches device memory.
+ * Sources: page "Kotaemon FlashAttention" (attention formula; algorithm bullets: Q row
+ * blocks, K_j/V_j blocks streamed through on-chip memory, running max and normaliser,
+ * result identical to the untiled formula); page "Flash Attention ... IO-aware exact"
+ * (fr), tiling pseudo-code (returns O and the per-row statistic L) and PyTorch section
+ * (is_causal); page "Flash Attention" (zh), online-softmax bullet and the O(N) memory
+ * claim.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library allocates
+ *    no device memory and keeps no per-call state; work is enqueued asynchronously on
+ *    `stream` (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *  - Tensors are contiguous, row-major, 16-bit (fp16 or bf16 per `dtype`); LSE is fp32.
+ *  - `scale` multiplies Q.K^T before the softmax (every workload passes 1/sqrt(d)).
+ *  - Grouped-query attention: query head h reads KV head h / (Hq / Hkv).
+ *  - Causal masking is bottom-right aligned: key j is visible to query i iff
+ *    j <= i + (Nk - Nq) (page "Flash Attention ... IO-aware exact" (fr), manual chunking
+ *    example). A row with no visible key gets O = 0 and LSE = -inf.
+ *  - Errors are returned as fa_status; nothing is thrown across the ABI. Host-side
+ *    argument checks run before any CUDA call, so FA_ERR_INVALID_ARG /
+ *    FA_ERR_UNSUPPORTED / FA_ERR_ALIGNMENT leave the stream untouched.
+ *  - Device-side waits are bounded. A wait that runs out sets a device status word that
+ *    fa_device_status() reads (FA_ERR_DEVICE_TIMEOUT); the kernel then returns early.
+ */
+#ifndef FA_B200_FA_H_
+#define FA_B200_FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,     /* null pointer, non-positive size, Hq % Hkv != 0, bad scale */
+  FA_ERR_UNSUPPORTED = 2,     /* d not in {64,128}, unknown dtype, device is not sm_100 */
+  FA_ERR_ALIGNMENT = 3,       /* a tensor pointer is not 16-byte aligned */
+  FA_ERR_CUDA = 4,            /* a CUDA runtime/driver call or a launch failed */
+  FA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait ran out (see fa_device_status) */
+  FA_ERR_WORKSPACE = 6        /* decode workspace missing or smaller than required */
+} fa_status;
+
+/*
+ * fa_fwd — prefill / forward attention, O and per-row LSE.
+ *
+ * Defined by: page "Kotaemon FlashAttention", attention formula and algorithm bullets;
+ * page "Flash Attention ... IO-aware exact" (fr), tiling pseudo-code (outputs O and L)
+ * and the PyTorch section (causal flag).
+ *
+ *   q    [B, Hq,  Nq, d]  fp16/bf16
+ *   k, v [B, Hkv, Nk, d]  fp16/bf16
+ *   o    [B, Hq,  Nq, d]  same dtype as q (written, rounded to nearest even)
+ *   lse  [B, Hq,  Nq]     fp32, natural log of the row normaliser of the scaled scores;
+ *                         may be NULL (then not written)
+ *   causal  0 or 1 (bottom-right aligned when Nq != Nk)
+ *   scale   finite, > 0
+ *
+ * Requirements: B, Hq, Hkv, Nq, Nk >= 1; Hq % Hkv == 0; d in {64, 128}; q, k, v, o
+ * 16-byte aligned, lse 4-byte aligned; sm_100 device; B*Hq and B*Hkv < 2^31.
+ * Returns FA_OK once the kernel is enqueued on `stream`.
+ */
+FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                 int causal, float scale, fa_dtype dtype, void* stream);
+
+/*
+ * fa_decode_workspace_bytes — bytes of scratch that fa_decode needs for these sizes.
+ *
+ * The split-KV decode writes, per (sequence, query head, KV split), a partial output
+ * row (d fp32) and its logsumexp (fp32), then merges them. max_kv_len is the cache
+ * capacity (its row stride), which bounds the number of splits. Returns 0 for invalid
+ * sizes.
+ */
+FA_API size_t fa_decode_workspace_bytes(int B, int Hq, int max_kv_len, int d);
+
+/*
+ * fa_decode — single-token decode over a grouped-query KV cache (split-KV).
+ *
+ * Defined by: the attention formula (page "Kotaemon FlashAttention") with one query row
+ * per sequence, non-causal over the cache's valid rows; KV-cache use and its per-token
+ * size with 8 KV heads of dimension 128 (page "Empreinte mémoire et calcul des couches
+ * Transformer", KV-cache paragraph). The merge of the per-split partial results uses the
+ * same rescaling identity as the online softmax (page "Kotaemon FlashAttention", running
+ * max and normaliser).
+ *
+ *   q         [B, Hq, d]               fp16/bf16
+ *   kcache,
+ *   vcache    [B, Hkv, max_kv_len, d]  fp16/bf16; rows >= kv_lens[b] are never read
+ *   kv_lens   [B] int32, device memory; values are clamped to [0, max_kv_len]
+ *   o         [B, Hq, d]               same dtype as q
+ *   lse       [B, Hq] fp32, may be NULL
+ *   workspace device scratch of at least fa_decode_workspace_bytes(B, Hq, max_kv_len, d)
+ *             bytes, 16-byte aligned, owned by the caller; contents need no initialisation
+ *             and are meaningless after the call. Two decodes that may run at the same
+ *             time need separate workspaces.
+ *
+ * A sequence with kv_lens[b] == 0 gets O = 0 and LSE = -inf.
+ * Requirements: as fa_fwd, plus workspace_bytes >= the required size
+ * (FA_ERR_WORKSPACE otherwise).
+ */
+FA_API fa_status fa_decode(const void* q, const void* kcache, const void* vcache,
+                    const int* kv_lens, void* o, float* lse,
+                    int B, int Hq, int Hkv, int max_kv_len, int d,
+                    float scale, fa_dtype dtype, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/* fa_status_string — static, human-readable name of a status code (never NULL). */
+FA_API const char* fa_status_string(fa_status s);
+
+/*
+ * fa_device_status — synchronises the current device, then returns FA_OK or the first
+ * error a kernel of this library recorded on it (FA_ERR_DEVICE_TIMEOUT). If `clear` is
+ * non-zero the recorded error is reset afterwards. FA_ERR_CUDA if the synchronisation
+ * itself fails.
+ */
+FA_API fa_status fa_device_status(int clear);
+
+/*
+ * fa_set_wait_timeout_ns — upper bound, in nanoseconds, on every device-side barrier wait
+ * of kernels launched afterwards from this process (default 2e9, i.e. 2 s). 0 restores
+ * the default. Test hook for the timeout path; normal callers never need it.
+ */
+FA_API void fa_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * fa_debug_skip_q_load — test hook for the bounded-wait path: when non-zero, fa_fwd
+ * kernels launched afterwards never issue the Q-tile load, so the barrier that waits for
+ * it is never completed and every wait that depends on it runs out. The kernel records
+ * FA_ERR_DEVICE_TIMEOUT and returns; the outputs are then unspecified. 0 restores normal
+ * operation.
+ */
+FA_API void fa_debug_skip_q_load(int enable);
+
+/* fa_build_info — static string: library version and the GPU architecture it targets. */
+FA_API const char* fa_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_FA_H_ */

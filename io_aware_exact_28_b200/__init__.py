@@ -1,0 +1,211 @@
+"""Python binding of libfa_b200.so: exact attention on B200 (sm_100a).
+
+Argument marshalling only. Every step of the computation runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback. If the shared library is missing or fails
+to load, the first call raises `FALibraryError`.
+
+Functions mirror the C ABI in ``include/fa.h``:
+
+* ``fwd(q, k, v, causal, scale)`` -> ``(o, lse)``   (``fa_fwd``)
+* ``decode(q, kcache, vcache, kv_lens, scale)`` -> ``(o, lse)``   (``fa_decode``)
+* ``decode_workspace_bytes(B, Hq, max_kv_len, d)``   (``fa_decode_workspace_bytes``)
+* ``device_status``, ``set_wait_timeout_ns``, ``debug_skip_q_load``, ``build_info``
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+from typing import Optional, Tuple
+
+__all__ = ["FAError", "FALibraryError", "LIB_PATH", "lib", "fwd", "decode",
+           "decode_workspace_bytes", "device_status", "set_wait_timeout_ns",
+           "debug_skip_q_load", "build_info", "status_string", "EXPORTED_SYMBOLS",
+           "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_ALIGNMENT",
+           "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_FP16", "FA_BF16"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
+
+FA_FP16, FA_BF16 = 0, 1
+(FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA,
+ FA_ERR_DEVICE_TIMEOUT, FA_ERR_WORKSPACE) = range(7)
+
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode", "fa_decode_workspace_bytes", "fa_status_string",
+                    "fa_device_status", "fa_set_wait_timeout_ns", "fa_debug_skip_q_load",
+                    "fa_build_info")
+
+
+class FALibraryError(RuntimeError):
+    """The CUDA library could not be loaded (not built, or built for another target)."""
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where} failed: {status_string(status)} ({status})")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfa_b200.so once and declare the C signatures."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise FALibraryError(
+                f"{LIB_PATH} is missing; build it with `python io_aware_exact_28_b200/csrc/build.py`")
+        try:
+            L = ctypes.CDLL(LIB_PATH)
+        except OSError as e:
+            raise FALibraryError(f"cannot load {LIB_PATH}: {e}") from e
+        c_int, c_float, c_void_p, c_size_t = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+        L.fa_fwd.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p] + [c_int] * 7 + \
+            [c_float, c_int, c_void_p]
+        L.fa_fwd.restype = c_int
+        L.fa_decode.argtypes = [c_void_p] * 6 + [c_int] * 5 + [c_float, c_int, c_void_p, c_size_t,
+                                                                 c_void_p]
+        L.fa_decode.restype = c_int
+        L.fa_decode_workspace_bytes.argtypes = [c_int] * 4
+        L.fa_decode_workspace_bytes.restype = c_size_t
+        L.fa_status_string.argtypes = [c_int]
+        L.fa_status_string.restype = ctypes.c_char_p
+        L.fa_device_status.argtypes = [c_int]
+        L.fa_device_status.restype = c_int
+        L.fa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+        L.fa_set_wait_timeout_ns.restype = None
+        L.fa_debug_skip_q_load.argtypes = [c_int]
+        L.fa_debug_skip_q_load.restype = None
+        L.fa_build_info.argtypes = []
+        L.fa_build_info.restype = ctypes.c_char_p
+        _lib = L
+        return L
+
+
+def status_string(status: int) -> str:
+    return lib().fa_status_string(int(status)).decode()
+
+
+def build_info() -> str:
+    return lib().fa_build_info().decode()
+
+
+def device_status(clear: bool = True) -> int:
+    return int(lib().fa_device_status(1 if clear else 0))
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    lib().fa_set_wait_timeout_ns(int(ns))
+
+
+def debug_skip_q_load(enable: bool) -> None:
+    lib().fa_debug_skip_q_load(1 if enable else 0)
+
+
+def decode_workspace_bytes(B: int, Hq: int, max_kv_len: int, d: int) -> int:
+    return int(lib().fa_decode_workspace_bytes(B, Hq, max_kv_len, d))
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float16:
+        return FA_FP16
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; expected float16 or bfloat16")
+
+
+def _check(t, name: str, ndim: int, device) -> None:
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, lse=None,
+        return_lse: bool = True, stream=None) -> Tuple[object, Optional[object]]:
+    """O = softmax(scale * Q K^T) V and the per-row natural-log LSE via ``fa_fwd``.
+
+    q [B,Hq,Nq,d], k and v [B,Hkv,Nk,d] (fp16 or bf16, contiguous, same CUDA device).
+    Returns (o [B,Hq,Nq,d], lse [B,Hq,Nq] fp32 or None).
+    """
+    import torch
+    _check(q, "q", 4, q.device)
+    _check(k, "k", 4, q.device)
+    _check(v, "v", 4, q.device)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk != d:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check(out, "out", 4, q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _check(lse, "lse", 3, q.device)
+    st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                      lse.data_ptr() if lse is not None else None,
+                      B, Hq, Hkv, Nq, Nk, d, 1 if causal else 0, float(scale), _dtype_code(q),
+                      _stream_ptr(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd")
+    return out, lse
+
+
+def decode(q, kcache, vcache, kv_lens, scale: Optional[float] = None, out=None, lse=None,
+           workspace=None, return_lse: bool = True, stream=None):
+    """Single-token decode over a KV cache via ``fa_decode``.
+
+    q [B,Hq,d]; kcache, vcache [B,Hkv,max_kv_len,d]; kv_lens int32 [B] on the device.
+    Returns (o [B,Hq,d], lse [B,Hq] fp32 or None).
+    """
+    import torch
+    _check(q, "q", 3, q.device)
+    _check(kcache, "kcache", 4, q.device)
+    _check(vcache, "vcache", 4, q.device)
+    _check(kv_lens, "kv_lens", 1, q.device)
+    if kv_lens.dtype != torch.int32:
+        raise TypeError("kv_lens must be int32")
+    if kcache.dtype != q.dtype or vcache.dtype != q.dtype:
+        raise TypeError("q and the caches must share one dtype")
+    B, Hq, d = q.shape
+    Bk, Hkv, max_len, dk = kcache.shape
+    if tuple(vcache.shape) != tuple(kcache.shape) or Bk != B or dk != d or kv_lens.shape[0] != B:
+        raise ValueError("shape mismatch between q, caches and kv_lens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_bytes(B, Hq, max_len, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = lib().fa_decode(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), kv_lens.data_ptr(),
+                         out.data_ptr(), lse.data_ptr() if lse is not None else None,
+                         B, Hq, Hkv, max_len, d, float(scale), _dtype_code(q),
+                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         _stream_ptr(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_decode")
+    return out, lse

@@ -1,0 +1,318 @@
+// fa_api.cu — host side of the C ABI declared in include/fa.h: argument checks, TMA
+// descriptors, launch configuration and status reporting. Compiled for sm_100a only.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "decode_kernel.cuh"
+#include "fwd_kernel.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;   // 2 s
+
+uint64_t g_timeout_ns = kDefaultTimeoutNs;
+int g_skip_q_load = 0;
+
+// ---------------------------------------------------------------------------------------
+// Device checks (cached per device)
+// ---------------------------------------------------------------------------------------
+enum DevState : int { kUnknown = 0, kSupported = 1, kUnsupported = 2 };
+int g_dev_state[kMaxDevices];
+std::mutex g_mu;
+
+fa_status check_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_dev_state[dev] == kUnknown) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+    g_dev_state[dev] = (major == 10 && minor == 0) ? kSupported : kUnsupported;
+  }
+  return g_dev_state[dev] == kSupported ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------------------------------
+// TMA descriptors through the driver entry point (no link-time dependency on libcuda)
+// ---------------------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [heads, rows, d] 16-bit tensor, box = 64 columns (128 bytes) x 128 rows x 1 head,
+// 128-byte swizzle; rows past `rows` read as zero and are clipped on store.
+bool make_tile_map(CUtensorMap* m, const void* ptr, int d, int rows, long long heads, bool bf16) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(rows) * d * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(fa::kBM), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+             const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------------------
+// Forward launch
+// ---------------------------------------------------------------------------------------
+template <int D, bool BF16, bool CAUSAL>
+fa_status launch_fwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const CUtensorMap& mo, const fa::FwdParams& prm, int BH, int Nq,
+                     cudaStream_t stream) {
+  using C = fa::FwdCfg<D>;
+  auto kernel = fa::fa_fwd_kernel<D, BF16, CAUSAL>;
+  static bool attr_set[kMaxDevices];
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_BYTES) != cudaSuccess)
+        return FA_ERR_CUDA;
+      attr_set[dev] = true;
+    }
+  }
+  const int n_qblocks = (Nq + fa::kQTiles * fa::kBM - 1) / (fa::kQTiles * fa::kBM);
+  dim3 grid(BH, n_qblocks, 1);
+  kernel<<<grid, fa::kFwdThreads, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+fa_status dispatch_causal(int causal, int dev, const CUtensorMap& mq, const CUtensorMap& mk,
+                          const CUtensorMap& mv, const CUtensorMap& mo, const fa::FwdParams& prm,
+                          int BH, int Nq, cudaStream_t st) {
+  return causal ? launch_fwd<D, BF16, true>(dev, mq, mk, mv, mo, prm, BH, Nq, st)
+                : launch_fwd<D, BF16, false>(dev, mq, mk, mv, mo, prm, BH, Nq, st);
+}
+
+// ---------------------------------------------------------------------------------------
+// Decode sizing: the split length depends only on (B, Hq, max_kv_len) so that the
+// workspace query and the launch always agree.
+// ---------------------------------------------------------------------------------------
+int decode_split_tokens(int B, int Hq, int max_len) {
+  const long long units = static_cast<long long>(B) * (Hq >= 4 ? Hq / 4 : 1);
+  int s = 256;
+  while (s > 64 && units * ((max_len + s - 1) / s) < 148LL * 8) s >>= 1;
+  return s;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct DecodeLayout {
+  int split_tokens, n_split;
+  size_t o_bytes, lse_off, total;
+};
+
+bool decode_layout(int B, int Hq, int max_len, int d, DecodeLayout* L) {
+  if (B <= 0 || Hq <= 0 || max_len <= 0 || d <= 0) return false;
+  L->split_tokens = decode_split_tokens(B, Hq, max_len);
+  L->n_split = (max_len + L->split_tokens - 1) / L->split_tokens;
+  const size_t rows = static_cast<size_t>(B) * Hq * L->n_split;
+  L->o_bytes = align_up(rows * d * sizeof(float), 256);
+  L->lse_off = L->o_bytes;
+  L->total = L->o_bytes + align_up(rows * sizeof(float), 256);
+  return true;
+}
+
+template <int D, int GT, bool BF16>
+fa_status launch_decode_t(const fa::DecodeParams& dp, const fa::CombineParams& cp, int B,
+                          int Hkv, int G, cudaStream_t st) {
+  const int n_gt = (G + GT - 1) / GT;
+  dim3 grid(dp.n_split, Hkv * n_gt, B);
+  fa::fa_decode_split_kernel<D, GT, BF16><<<grid, fa::kDecThreads, 0, st>>>(dp);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  fa::fa_decode_combine_kernel<D, BF16><<<B * dp.Hq, D, 0, st>>>(cp);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+fa_status launch_decode_g(const fa::DecodeParams& dp, const fa::CombineParams& cp, int B,
+                          int Hkv, int G, cudaStream_t st) {
+  if (G <= 1) return launch_decode_t<D, 1, BF16>(dp, cp, B, Hkv, G, st);
+  if (G <= 2) return launch_decode_t<D, 2, BF16>(dp, cp, B, Hkv, G, st);
+  if (G <= 4) return launch_decode_t<D, 4, BF16>(dp, cp, B, Hkv, G, st);
+  return launch_decode_t<D, 8, BF16>(dp, cp, B, Hkv, G, st);
+}
+
+fa_status common_checks(int B, int Hq, int Hkv, int d, float scale, int dtype) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                 int Hkv, int Nq, int Nk, int d, int causal, float scale, fa_dtype dtype,
+                 void* stream) {
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (Nq <= 0 || Nk <= 0 || (causal != 0 && causal != 1)) return FA_ERR_INVALID_ARG;
+  fa_status s = common_checks(B, Hq, Hkv, d, scale, dtype);
+  if (s != FA_OK) return s;
+  const long long BH = static_cast<long long>(B) * Hq;
+  const long long BHkv = static_cast<long long>(B) * Hkv;
+  if (BH >= (1LL << 31)) return FA_ERR_INVALID_ARG;
+  if ((Nq + fa::kQTiles * fa::kBM - 1) / (fa::kQTiles * fa::kBM) > 65535) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGNMENT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_ALIGNMENT;
+  int dev = 0;
+  s = check_device(&dev);
+  if (s != FA_OK) return s;
+
+  const bool bf16 = dtype == FA_BF16;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_tile_map(&mq, q, d, Nq, BH, bf16) || !make_tile_map(&mk, k, d, Nk, BHkv, bf16) ||
+      !make_tile_map(&mv, v, d, Nk, BHkv, bf16) || !make_tile_map(&mo, o, d, Nq, BH, bf16))
+    return FA_ERR_CUDA;
+
+  fa::FwdParams prm;
+  prm.lse = lse;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.causal_offset = Nk - Nq;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.timeout_ns = g_timeout_ns;
+  prm.skip_q_load = g_skip_q_load;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int bh = static_cast<int>(BH);
+  if (d == 64)
+    return bf16 ? dispatch_causal<64, true>(causal, dev, mq, mk, mv, mo, prm, bh, Nq, st)
+                : dispatch_causal<64, false>(causal, dev, mq, mk, mv, mo, prm, bh, Nq, st);
+  return bf16 ? dispatch_causal<128, true>(causal, dev, mq, mk, mv, mo, prm, bh, Nq, st)
+              : dispatch_causal<128, false>(causal, dev, mq, mk, mv, mo, prm, bh, Nq, st);
+}
+
+size_t fa_decode_workspace_bytes(int B, int Hq, int max_kv_len, int d) {
+  DecodeLayout L;
+  if (!decode_layout(B, Hq, max_kv_len, d, &L)) return 0;
+  return L.total;
+}
+
+fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const int* kv_lens,
+                    void* o, float* lse, int B, int Hq, int Hkv, int max_kv_len, int d,
+                    float scale, fa_dtype dtype, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  if (!q || !kcache || !vcache || !kv_lens || !o) return FA_ERR_INVALID_ARG;
+  if (max_kv_len <= 0) return FA_ERR_INVALID_ARG;
+  fa_status s = common_checks(B, Hq, Hkv, d, scale, dtype);
+  if (s != FA_OK) return s;
+  if (B > 65535 || static_cast<long long>(B) * Hq >= (1LL << 31)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o))
+    return FA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(kv_lens) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_ALIGNMENT;
+  DecodeLayout L;
+  decode_layout(B, Hq, max_kv_len, d, &L);
+  if (!workspace || workspace_bytes < L.total) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_ALIGNMENT;
+  const int G = Hq / Hkv;
+  if (static_cast<long long>(Hkv) * ((G + 7) / 8) > 65535) return FA_ERR_INVALID_ARG;
+  int dev = 0;
+  s = check_device(&dev);
+  if (s != FA_OK) return s;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  fa::DecodeParams dp;
+  dp.q = static_cast<const uint16_t*>(q);
+  dp.kc = static_cast<const uint16_t*>(kcache);
+  dp.vc = static_cast<const uint16_t*>(vcache);
+  dp.kv_lens = kv_lens;
+  dp.ws_o = reinterpret_cast<float*>(ws);
+  dp.ws_lse = reinterpret_cast<float*>(ws + L.lse_off);
+  dp.Hq = Hq;
+  dp.Hkv = Hkv;
+  dp.G = G;
+  dp.max_len = max_kv_len;
+  dp.split_tokens = L.split_tokens;
+  dp.n_split = L.n_split;
+  dp.scale_log2 = scale * 1.4426950408889634f;
+  fa::CombineParams cp;
+  cp.ws_o = dp.ws_o;
+  cp.ws_lse = dp.ws_lse;
+  cp.kv_lens = kv_lens;
+  cp.o = static_cast<uint16_t*>(o);
+  cp.lse = lse;
+  cp.Hq = Hq;
+  cp.max_len = max_kv_len;
+  cp.split_tokens = L.split_tokens;
+  cp.n_split = L.n_split;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == FA_BF16;
+  if (d == 64)
+    return bf16 ? launch_decode_g<64, true>(dp, cp, B, Hkv, G, st)
+                : launch_decode_g<64, false>(dp, cp, B, Hkv, G, st);
+  return bf16 ? launch_decode_g<128, true>(dp, cp, B, Hkv, G, st)
+              : launch_decode_g<128, false>(dp, cp, B, Hkv, G, st);
+}
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_ALIGNMENT: return "FA_ERR_ALIGNMENT";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+fa_status fa_device_status(int clear) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_fa_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (clear && v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return v == 0 ? FA_OK : static_cast<fa_status>(v);
+}
+
+void fa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTimeoutNs; }
+
+void fa_debug_skip_q_load(int enable) { g_skip_q_load = enable ? 1 : 0; }
+
+const char* fa_build_info(void) { return "libfa_b200 0.1 sm_100a (tcgen05/TMA prefill, split-KV decode)"; }
+
+}  // extern "C"

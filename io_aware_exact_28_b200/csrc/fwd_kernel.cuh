@@ -1,0 +1,364 @@
+// fwd_kernel.cuh — exact attention forward (prefill) for sm_100a.
+//
+// One CTA owns 256 query rows of one (batch, query head): two 128-row Q tiles that
+// take turns on the tensor core. Per K/V tile j (128 keys) and Q tile t:
+//     S_t = Q_t K_j^T                    tcgen05.mma, fp32 accumulator in TMEM
+//     softmax warps: mask, row max, lazy rescale of O_t, P_t = exp2(S*c - m) -> TMEM
+//     O_t += P_t V_j                     tcgen05.mma with A read from TMEM
+// so the 128x128 score tile lives only in tensor memory and registers and never reaches
+// device memory. This is the tiling + online-softmax scheme of page "Kotaemon
+// FlashAttention" (algorithm bullets: Q split into row blocks, K_j/V_j blocks streamed
+// through on-chip memory, running max and normaliser, result identical to the untiled
+// formula) and page "Flash Attention ... IO-aware exact" (fr), tiling pseudo-code (Q_i
+// read once, K_j/V_j per block, O_i and L written once at the end).
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax + epilogue for Q tile 0 (thread r owns row r = TMEM lane r)
+//   warps 4-7  softmax + epilogue for Q tile 1
+//   warp  8    TMA producer: Q tiles once, then K_j, V_j through an NS-stage ring
+//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+//
+// Tensor memory (512 columns): S_t at columns [128t, 128t+128) (fp32); P_t overwrites
+// the first 64 of those columns as packed 16-bit pairs; O_t at [256 + t*D, 256+(t+1)*D).
+//
+// Lazy rescaling: the running maximum m used in the exponent is only raised when a new
+// tile maximum exceeds it by more than 8 (log2 units). O and l are both accumulated
+// against the same m, so the final O/l and LSE = (m + log2 l) ln 2 are exact in real
+// arithmetic whatever m is; the bound keeps P <= 2^8.
+#pragma once
+
+#include <cuda.h>
+#include <math_constants.h>
+
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int kBM = 128;           // query rows per Q tile (one TMEM lane per row)
+constexpr int kBN = 128;           // keys per K/V tile
+constexpr int kQTiles = 2;         // Q tiles per CTA
+constexpr int kFwdThreads = 320;
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+constexpr uint64_t kDrainNs = 200000000ull;   // 0.2 s limit for abort-path drains
+
+template <int D>
+struct FwdCfg {
+  static constexpr int NCH = D / 64;                  // 128-byte swizzle chunks along d
+  static constexpr int CHUNK_BYTES = kBM * 128;       // 128 rows x 128 bytes
+  static constexpr int TILE_BYTES = kBM * D * 2;      // one 128-row tile of Q, K, V or O
+  static constexpr int NS = (D == 128) ? 4 : 8;       // K/V ring stages
+  static constexpr int Q_OFF = 0;
+  static constexpr int KV_OFF = kQTiles * TILE_BYTES;
+  static constexpr int BAR_OFF = KV_OFF + NS * TILE_BYTES;
+  static constexpr int NBARS = 1 + 2 * NS + 2 * kQTiles + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;   // + slack for 1 KB alignment
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t S_COL = 0;
+  static constexpr uint32_t O_COL = 256;
+  static_assert(O_COL + kQTiles * D <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+struct FwdParams {
+  float* lse;           // [B*Hq, Nq] or nullptr
+  int Hq, Hkv, group;   // group = Hq / Hkv
+  int Nq, Nk;
+  int causal_offset;    // Nk - Nq (bottom-right alignment)
+  float scale_log2;     // scale * log2(e)
+  uint64_t timeout_ns;
+  int skip_q_load;      // test hook
+};
+
+__device__ int g_fa_status;   // first device-side error (0 = none)
+
+template <int D>
+__device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
+#pragma unroll
+  for (int c = 0; c < D; c += 32) {
+    uint32_t v[32];
+    tmem_ld32x32b_x32(tO + c, v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+    tmem_st32x32b_x32(tO + c, v);
+  }
+  tmem_st_wait();
+}
+
+template <int D, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+              const FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;                        // b * Hq + h
+  const int b = bh / p.Hq;
+  const int h = bh - b * p.Hq;
+  const int bh_kv = b * p.Hkv + h / p.group;
+  const int qb = gridDim.y - 1 - blockIdx.y;        // heaviest (causal) blocks launch first
+  const int q0 = qb * (kQTiles * kBM);
+
+  const int n_kv_total = (p.Nk + kBN - 1) / kBN;
+  int n_kv = n_kv_total;
+  if (CAUSAL) {
+    const int q_last = min(q0 + kQTiles * kBM - 1, p.Nq - 1);
+    const int kmax = q_last + p.causal_offset;      // last key visible to this CTA
+    n_kv = kmax < 0 ? 0 : min(n_kv_total, kmax / kBN + 1);
+  }
+
+  const uint32_t bar0 = base + C::BAR_OFF;
+  auto bar_q = [&]() { return bar0; };
+  auto bar_full = [&](int i) { return bar0 + 8u * (1 + i); };
+  auto bar_empty = [&](int i) { return bar0 + 8u * (1 + C::NS + i); };
+  auto bar_s = [&](int t) { return bar0 + 8u * (1 + 2 * C::NS + t); };
+  auto bar_p = [&](int t) { return bar0 + 8u * (1 + 2 * C::NS + kQTiles + t); };
+  const uint32_t bar_drain = bar0 + 8u * (1 + 2 * C::NS + 2 * kQTiles);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + C::MISC_OFF + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q(), 1);
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(bar_full(i), 1);
+      mbar_init(bar_empty(i), 1);
+    }
+    for (int t = 0; t < kQTiles; ++t) {
+      mbar_init(bar_s(t), 1);
+      mbar_init(bar_p(t), kBM);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == kWarpMma) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+  if (warp == kWarpProducer && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{abort_flag, &g_fa_status, p.timeout_ns};
+
+  if (warp == kWarpProducer) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      bool q_issued = false;
+      // A CTA with no visible key tile writes zeros from the softmax warps and needs no Q.
+      if (!p.skip_q_load && n_kv > 0) {
+        mbar_arrive_expect_tx(bar_q(), kQTiles * C::TILE_BYTES);
+        for (int t = 0; t < kQTiles; ++t)
+          for (int ch = 0; ch < C::NCH; ++ch)
+            tma_load_3d(base + C::Q_OFF + t * C::TILE_BYTES + ch * C::CHUNK_BYTES, &tmQ, bar_q(),
+                        ch * 64, q0 + t * kBM, bh);
+        q_issued = true;
+      }
+      int it = 0;
+      bool ok = true;
+      for (int j = 0; j < n_kv && ok; ++j) {
+        for (int kv = 0; kv < 2; ++kv) {
+          const int slot = it % C::NS;
+          const int round = it / C::NS;
+          if (round > 0 && !mbar_wait(bar_empty(slot), (round - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_full(slot), C::TILE_BYTES);
+          const CUtensorMap* tm = kv ? &tmV : &tmK;
+          for (int ch = 0; ch < C::NCH; ++ch)
+            tma_load_3d(base + C::KV_OFF + slot * C::TILE_BYTES + ch * C::CHUNK_BYTES, tm,
+                        bar_full(slot), ch * 64, j * kBN, bh_kv);
+          ++it;
+        }
+      }
+      if (!ok || *abort_flag) {
+        // Loads still in flight must land before the CTA exits.
+        for (int k = max(0, it - C::NS); k < it; ++k)
+          mbar_wait_drain(bar_full(k % C::NS), (k / C::NS) & 1, kDrainNs);
+        if (q_issued) mbar_wait_drain(bar_q(), 0, kDrainNs);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_kv > 0) {
+      constexpr uint32_t IDESC_S = idesc_f16(kBM, kBN, BF16 ? 1u : 0u, 0u, 0u);
+      constexpr uint32_t IDESC_O = idesc_f16(kBM, D, BF16 ? 1u : 0u, 0u, 1u);
+      auto issue_s = [&](int t, int kslot) {
+        const uint32_t qa = base + C::Q_OFF + t * C::TILE_BYTES;
+        const uint32_t ka = base + C::KV_OFF + kslot * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+          mma_f16_ss(tmem + C::S_COL + t * kBN, sdesc_k_sw128(qa + off), sdesc_k_sw128(ka + off),
+                     IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int vslot, bool acc0) {
+        const uint32_t va = base + C::KV_OFF + vslot * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          mma_f16_ts(tmem + C::O_COL + t * D, tmem + C::S_COL + t * kBN + kk * 8,
+                     sdesc_mn_sw128(va + kk * 2048, C::CHUNK_BYTES), IDESC_O,
+                     (acc0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar_q(), 0, wc);
+      bool issued = false;
+      tc_fence_after();
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int kit = 2 * j, kslot = kit % C::NS;
+        const int vit = 2 * j - 1, vslot = (vit + C::NS) % C::NS;   // V_{j-1}
+        if (!mbar_wait(bar_full(kslot), (kit / C::NS) & 1, wc)) { ok = false; break; }
+        if (j > 0 && !mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        for (int t = 0; t < kQTiles; ++t) {
+          if (j > 0) {
+            if (!mbar_wait(bar_p(t), (j - 1) & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(t, vslot, j - 1 > 0);
+            if (t == kQTiles - 1) mma_commit(bar_empty(vslot));
+          }
+          issue_s(t, kslot);
+          issued = true;
+          mma_commit(bar_s(t));
+        }
+        if (!ok) break;
+        mma_commit(bar_empty(kslot));
+      }
+      if (ok) {
+        const int vit = 2 * n_kv - 1, vslot = vit % C::NS;
+        ok = mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc);
+        for (int t = 0; t < kQTiles && ok; ++t) {
+          if (!mbar_wait(bar_p(t), (n_kv - 1) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(t, vslot, n_kv - 1 > 0);
+          mma_commit(bar_s(t));   // final phase: O_t complete
+        }
+        if (ok) mma_commit(bar_empty(vslot));
+      }
+      if (issued) {
+        // Every MMA must have finished before TMEM is released.
+        mma_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0, kDrainNs);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int t = warp >> 2;
+    const int r = threadIdx.x & (kBM - 1);
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + C::S_COL + t * kBN;
+    const uint32_t tO = tmem + lane_base + C::O_COL + t * D;
+    const int row = q0 + t * kBM + r;
+    const int row_min = q0 + t * kBM;
+    const int lim = CAUSAL ? min(row + p.causal_offset, p.Nk - 1) : p.Nk - 1;
+    const int lim_min = CAUSAL ? min(row_min + p.causal_offset, p.Nk - 1) : p.Nk - 1;
+    const float c = p.scale_log2;
+
+    float m_used = -CUDART_INF_F;
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      if (!mbar_wait(bar_s(t), j & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[kBN];
+      tmem_ld32x32b_x128(tS, sr);
+      const int key0 = j * kBN;
+      if (key0 + kBN - 1 > lim_min) {               // tile-uniform: diagonal or ragged tile
+#pragma unroll
+        for (int k = 0; k < kBN; ++k)
+          if (key0 + k > lim) sr[k] = __float_as_uint(-CUDART_INF_F);
+      }
+      float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
+#pragma unroll
+      for (int k = 0; k < kBN; k += 2) {
+        mx0 = fmaxf(mx0, __uint_as_float(sr[k]));
+        mx1 = fmaxf(mx1, __uint_as_float(sr[k + 1]));
+      }
+      const float mx = fmaxf(mx0, mx1) * c;          // scale > 0, -inf stays -inf
+      if (mx > m_used + 8.0f) {
+        if (m_used != -CUDART_INF_F) {               // O_t and l hold earlier tiles
+          const float alpha = ex2_approx(m_used - mx);
+          l *= alpha;
+          rescale_o_row<D>(tO, alpha);
+        }
+        m_used = mx;
+      }
+      const float mref = (m_used == -CUDART_INF_F) ? 0.f : m_used;
+      uint32_t pk[kBN / 2];
+      float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+      for (int k = 0; k < kBN / 2; ++k) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * k]), c, -mref));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * k + 1]), c, -mref));
+        l0 += p0;
+        l1 += p1;
+        pk[k] = pack_half2(p0, p1, BF16);
+      }
+      l += l0 + l1;
+      tmem_st32x32b_x64(tS, pk);                    // P_t into S_t columns [0, 64)
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_p(t));
+    }
+    if (ok && n_kv > 0) {
+      ok = mbar_wait(bar_s(t), n_kv & 1, wc);       // final PV of this tile done
+      tc_fence_after();
+    }
+    uint8_t* otile = sbase + C::Q_OFF + t * C::TILE_BYTES;   // Q_t no longer read
+    if (ok) {
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+      for (int ch = 0; ch < C::NCH; ++ch) {
+        uint32_t o[64];
+        if (n_kv > 0) {
+          tmem_ld32x32b_x64(tO + ch * 64, o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) o[i] = 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          uint4 w;
+          w.x = pack_half2(__uint_as_float(o[8 * u + 0]) * inv_l, __uint_as_float(o[8 * u + 1]) * inv_l, BF16);
+          w.y = pack_half2(__uint_as_float(o[8 * u + 2]) * inv_l, __uint_as_float(o[8 * u + 3]) * inv_l, BF16);
+          w.z = pack_half2(__uint_as_float(o[8 * u + 4]) * inv_l, __uint_as_float(o[8 * u + 5]) * inv_l, BF16);
+          w.w = pack_half2(__uint_as_float(o[8 * u + 6]) * inv_l, __uint_as_float(o[8 * u + 7]) * inv_l, BF16);
+          // 128-byte swizzle: 16-byte unit u of row r sits at unit u ^ (r mod 8)
+          *reinterpret_cast<uint4*>(otile + ch * C::CHUNK_BYTES + r * 128 + ((u ^ (r & 7)) << 4)) = w;
+        }
+      }
+      if (p.lse != nullptr && row < p.Nq) {
+        p.lse[static_cast<size_t>(bh) * p.Nq + row] =
+            (l > 0.f) ? (m_used + __log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
+      }
+      fence_proxy_async_smem();
+    }
+    named_barrier_sync(1 + t, kBM);
+    if (r == 0 && ok && !*abort_flag) {
+      for (int ch = 0; ch < C::NCH; ++ch)
+        tma_store_3d(&tmO, smem_u32(otile + ch * C::CHUNK_BYTES), ch * 64, q0 + t * kBM, bh);
+      tma_store_commit_and_wait_read();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,65 @@
+"""Tolerances and comparison helpers shared by the GPU parity tests.
+
+Tolerances (stated for this workload family): output max-abs error <= 4e-3 for fp16 and
+<= 1.6e-2 for bf16, output RMS error <= 1e-3, and LSE relative error <= 1e-4 with the
+denominator max(|LSE_ref|, 1) (LSE near 0, e.g. the first causal row, is otherwise
+ill-conditioned). Rows whose reference LSE is -inf (no visible key) must come back as
+O = 0 and LSE = -inf exactly.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+MAX_ABS = {"fp16": 4e-3, "bf16": 1.6e-2}
+RMS_TOL = 1e-3
+LSE_REL = 1e-4
+
+
+def to_f64(t) -> np.ndarray:
+    import torch
+    t = t.detach().to("cpu")
+    if t.dtype in (torch.float16, torch.bfloat16):
+        t = t.float()
+    return t.double().numpy()
+
+
+def metrics(o_gpu, lse_gpu, O_ref, L_ref):
+    o = to_f64(o_gpu) if not isinstance(o_gpu, np.ndarray) else o_gpu
+    O_ref = np.asarray(O_ref)
+    err = np.abs(o - O_ref)
+    out = {"max_abs": float(err.max()) if err.size else 0.0,
+           "rms": float(np.sqrt(np.mean(err ** 2))) if err.size else 0.0}
+    if lse_gpu is not None:
+        lg = to_f64(lse_gpu) if not isinstance(lse_gpu, np.ndarray) else lse_gpu
+        L_ref = np.asarray(L_ref)
+        fin = np.isfinite(L_ref)
+        out["lse_nonfinite_mismatch"] = int(np.sum(np.isfinite(lg) != fin))
+        if fin.any():
+            rel = np.abs(lg[fin] - L_ref[fin]) / np.maximum(np.abs(L_ref[fin]), 1.0)
+            out["lse_rel"] = float(rel.max())
+        else:
+            out["lse_rel"] = 0.0
+        if (~fin).any():
+            out["empty_rows_nonzero"] = int(np.sum(np.abs(o[~fin]) > 0))
+    return out
+
+
+def assert_close(o_gpu, lse_gpu, O_ref, L_ref, dtype: str, what: str = ""):
+    m = metrics(o_gpu, lse_gpu, O_ref, L_ref)
+    assert np.all(np.isfinite(to_f64(o_gpu) if not isinstance(o_gpu, np.ndarray) else o_gpu)), \
+        f"{what}: non-finite output"
+    assert m["max_abs"] <= MAX_ABS[dtype], f"{what}: max-abs {m['max_abs']:.3e} > {MAX_ABS[dtype]} {m}"
+    assert m["rms"] <= RMS_TOL, f"{what}: rms {m['rms']:.3e} > {RMS_TOL} {m}"
+    if lse_gpu is not None:
+        assert m["lse_nonfinite_mismatch"] == 0, f"{what}: -inf pattern of LSE differs {m}"
+        assert m["lse_rel"] <= LSE_REL, f"{what}: LSE rel {m['lse_rel']:.3e} > {LSE_REL} {m}"
+        assert m.get("empty_rows_nonzero", 0) == 0, f"{what}: rows without keys must be 0 {m}"
+    return m
+
+
+def sample_rows(N: int, n_random: int, seed: int) -> np.ndarray:
+    """Edge rows of a length-N sequence (tile boundaries, both ends) plus seeded random rows."""
+    fixed = [0, 1, 2, 63, 64, 127, 128, 129, 255, 256, 257, N // 2, N - 129, N - 128, N - 2, N - 1]
+    r = np.random.default_rng(seed).choice(N, size=min(n_random, N), replace=False)
+    rows = np.unique(np.concatenate([[x for x in fixed if 0 <= x < N], r]))
+    return rows.astype(np.int64)

@@ -1,0 +1,86 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol the header declares,
+and rejects bad arguments on the host before touching CUDA (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import io_aware_exact_28_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+def header_functions():
+    with open(HEADER) as f:
+        src = f.read()
+    return re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", src)
+
+
+def test_library_loads_and_targets_sm100a():
+    assert os.path.exists(fa.LIB_PATH)
+    assert "sm_100a" in fa.build_info()
+
+
+def test_every_declared_symbol_is_exported():
+    names = header_functions()
+    assert set(names) == set(fa.EXPORTED_SYMBOLS), names
+    L = ctypes.CDLL(fa.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    for code in range(7):
+        assert fa.status_string(code).startswith("FA_")
+    assert fa.status_string(99) == "FA_ERR_UNKNOWN"
+
+
+def _fwd(L, q=16, k=16, v=16, o=16, lse=None, B=1, Hq=2, Hkv=1, Nq=128, Nk=128, d=64, causal=1,
+         scale=0.125, dtype=0):
+    return L.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, dtype, None)
+
+
+def test_fwd_rejects_bad_arguments_without_cuda():
+    L = fa.lib()
+    assert _fwd(L, q=None) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, o=None) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, B=0) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, Nq=0) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, Nk=-3) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, Hq=3, Hkv=2) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, causal=2) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, scale=float("inf")) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, scale=float("nan")) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, scale=-1.0) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, d=96) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd(L, dtype=7) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd(L, q=24) == fa.FA_ERR_ALIGNMENT
+    assert _fwd(L, lse=18) == fa.FA_ERR_ALIGNMENT
+
+
+def test_decode_rejects_bad_arguments_without_cuda():
+    L = fa.lib()
+    need = fa.decode_workspace_bytes(2, 8, 4096, 128)
+
+    def call(q=16, kc=16, vc=16, lens=16, o=16, lse=None, B=2, Hq=8, Hkv=2, max_len=4096, d=128,
+             scale=0.088, dtype=1, ws=32, ws_bytes=need):
+        return L.fa_decode(q, kc, vc, lens, o, lse, B, Hq, Hkv, max_len, d, scale, dtype, ws,
+                           ws_bytes, None)
+    assert call(lens=None) == fa.FA_ERR_INVALID_ARG
+    assert call(max_len=0) == fa.FA_ERR_INVALID_ARG
+    assert call(Hq=6, Hkv=4) == fa.FA_ERR_INVALID_ARG
+    assert call(d=80) == fa.FA_ERR_UNSUPPORTED
+    assert call(kc=8) == fa.FA_ERR_ALIGNMENT
+    assert call(ws=None) == fa.FA_ERR_WORKSPACE
+    assert call(ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE
+
+
+def test_workspace_size_covers_every_split():
+    # one fp32 row of d plus one fp32 LSE per (sequence, head, split), 256-byte aligned parts
+    for (B, Hq, max_len, d) in [(64, 32, 4096, 128), (1, 1, 1, 64), (3, 8, 1000, 128)]:
+        n = fa.decode_workspace_bytes(B, Hq, max_len, d)
+        assert n >= B * Hq * (d + 1) * 4
+        assert n % 256 == 0
+    assert fa.decode_workspace_bytes(0, 8, 128, 64) == 0

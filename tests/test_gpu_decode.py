@@ -1,0 +1,94 @@
+"""GPU parity of fa_decode (through the C ABI) against the float64 CPU oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import io_aware_exact_28_b200 as fa
+from oracle import decode_f64
+from tests.parity import assert_close
+from workloads import WORKLOADS, make_decode_inputs
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def run_decode(kv_lens, q, kc, vc, scale, workspace=None):
+    o, lse = fa.decode(q.to(DEV), kc.to(DEV), vc.to(DEV), kv_lens.to(DEV), scale=scale,
+                       workspace=workspace)
+    torch.cuda.synchronize()
+    assert fa.device_status() == fa.FA_OK
+    return o.cpu(), lse.cpu()
+
+
+def check(B, Hq, Hkv, cache, d, dtype, lens, seed=0):
+    kv_lens, q, kc, vc = make_decode_inputs(B, Hq, Hkv, cache, d, dtype, 1, cache, seed,
+                                            kv_lens=torch.tensor(lens))
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_decode(kv_lens, q, kc, vc, scale)
+    O, L = decode_f64(q, kc, vc, kv_lens, scale)
+    return assert_close(o, lse, O, L, dtype, f"decode B{B} Hq{Hq} Hkv{Hkv} d{d} {dtype} {lens}")
+
+
+def test_decode_workload_full():
+    """B=64, Hq=32, Hkv=8, d=128 bf16, kv_len ~ U[512, 4096] from seed 0: every output."""
+    w = WORKLOADS["decode"]
+    kv_lens, q, kc, vc = make_decode_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.dtype, w.kv_len_lo,
+                                            w.kv_len_hi, w.seed)
+    o, lse = run_decode(kv_lens, q, kc, vc, w.scale)
+    O, L = decode_f64(q, kc, vc, kv_lens, w.scale)
+    assert_close(o, lse, O, L, w.dtype, "decode workload")
+
+
+@pytest.mark.parametrize("lens", [[1, 2, 3, 4], [255, 256, 257, 4096], [511, 512, 513, 1000],
+                                  [4095, 4096, 1, 64], [0, 5, 0, 4096]])
+def test_lengths_at_split_edges(lens):
+    """kv_len = 0 (O = 0, LSE = -inf), 1, split boundaries +-1 and the full cache."""
+    check(4, 32, 8, 4096, 128, "bf16", lens, seed=sum(lens))
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (8, 4), (16, 2), (24, 8), (10, 2), (32, 2)])
+@pytest.mark.parametrize("d,dtype", [(64, "fp16"), (128, "bf16"), (128, "fp16")])
+def test_groupings_and_dims(Hq, Hkv, d, dtype):
+    """G = Hq/Hkv in {1, 2, 3, 5, 8, 16}; G > 8 and odd G use head tiles with masking."""
+    check(3, Hq, Hkv, 700, d, dtype, [700, 333, 1], seed=Hq + Hkv + d)
+
+
+def test_poisoned_cache_rows_beyond_length():
+    """NaN in cache rows >= kv_len must never be read."""
+    B, Hq, Hkv, cache, d = 4, 16, 4, 2048, 128
+    lens = torch.tensor([100, 2047, 1, 1500])
+    kv_lens, q, kc, vc = make_decode_inputs(B, Hq, Hkv, cache, d, "bf16", 1, cache, 21,
+                                            kv_lens=lens)
+    kcp, vcp = kc.clone(), vc.clone()
+    for b in range(B):
+        kcp[b, :, int(lens[b]):] = float("nan")
+        vcp[b, :, int(lens[b]):] = float("nan")
+    o, lse = run_decode(kv_lens, q, kcp, vcp, 1 / math.sqrt(d))
+    O, L = decode_f64(q, kc, vc, kv_lens, 1 / math.sqrt(d))
+    assert_close(o, lse, O, L, "bf16", "poisoned decode")
+
+
+def test_lengths_beyond_cache_are_clamped():
+    B, Hq, Hkv, cache, d = 2, 8, 2, 300, 64
+    kv_lens, q, kc, vc = make_decode_inputs(B, Hq, Hkv, cache, d, "fp16", 1, cache, 22,
+                                            kv_lens=torch.tensor([5000, -3]))
+    o, lse = run_decode(kv_lens, q, kc, vc, 0.125)
+    O, L = decode_f64(q, kc, vc, torch.tensor([300, 0]), 0.125)
+    assert_close(o, lse, O, L, "fp16", "clamped")
+
+
+def test_workspace_reuse_and_determinism():
+    w = WORKLOADS["decode"]
+    kv_lens, q, kc, vc = make_decode_inputs(8, w.Hq, w.Hkv, 1024, w.d, w.dtype, 1, 1024, 23)
+    ws = torch.empty(fa.decode_workspace_bytes(8, w.Hq, 1024, w.d), dtype=torch.uint8, device=DEV)
+    ws.fill_(0xFF)   # garbage (NaN patterns) in the workspace must not matter
+    args = (q.to(DEV), kc.to(DEV), vc.to(DEV), kv_lens.to(DEV))
+    o1, l1 = fa.decode(*args, workspace=ws)
+    o2, l2 = fa.decode(*args, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    O, L = decode_f64(q, kc, vc, kv_lens, w.scale)
+    assert_close(o1.cpu(), l1.cpu(), O, L, w.dtype, "reuse")

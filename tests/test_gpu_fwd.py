@@ -1,0 +1,177 @@
+"""GPU parity of fa_fwd (through the C ABI) against the float64 CPU oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import io_aware_exact_28_b200 as fa
+from oracle import attention_f64, attention_rows_f64
+from tests.parity import assert_close, sample_rows, to_f64
+from workloads import WORKLOADS, make_fwd_inputs
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def run_fwd(q, k, v, causal, scale=None):
+    o, lse = fa.fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.device_status() == fa.FA_OK
+    return o.cpu(), lse.cpu()
+
+
+def check_full(B, Hq, Hkv, Nq, Nk, d, dtype, causal, seed=0):
+    q, k, v = make_fwd_inputs(B, Hq, Hkv, Nq, Nk, d, dtype, seed)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_fwd(q, k, v, causal, scale)
+    O, L = attention_f64(q, k, v, causal, scale)
+    return assert_close(o, lse, O, L, dtype, f"B{B} Hq{Hq} Hkv{Hkv} Nq{Nq} Nk{Nk} d{d} {dtype} c{causal}")
+
+
+def test_tiny_workload():
+    w = WORKLOADS["tiny"]
+    check_full(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.causal)
+
+
+def test_mha2k_workload_full():
+    """The causal B=8 H=12 N=2048 d=64 fp16 workload, every output element."""
+    w = WORKLOADS["mha2k"]
+    check_full(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.causal)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 77, 128, 129, 256, 300, 640])
+def test_shapes_ragged(d, dtype, causal, N):
+    """Lengths that are not multiples of the 128-row tile or the 256-row CTA block."""
+    check_full(1, 2, 1, N, N, d, dtype, causal, seed=N + d)
+
+
+@pytest.mark.parametrize("Nq,Nk", [(128, 640), (77, 300), (300, 77), (1, 513), (256, 129),
+                                   (512, 1024)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_rectangular(Nq, Nk, causal):
+    """Nq != Nk, bottom-right aligned causal mask (chunked prefill against a longer prefix,
+    and the degenerate Nq > Nk case where early rows see no key)."""
+    check_full(2, 4, 2, Nq, Nk, 128, "bf16", causal, seed=Nq * 7 + Nk)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 1), (8, 2), (6, 3), (4, 4)])
+def test_gqa_groupings(Hq, Hkv):
+    check_full(2, Hq, Hkv, 384, 384, 64, "fp16", True, seed=Hq * 10 + Hkv)
+
+
+def test_first_causal_row_is_exact():
+    """Row 0 of a square causal problem sees only key 0: P = 1, l = 1, O = V[0] exactly."""
+    q, k, v = make_fwd_inputs(1, 4, 4, 512, 512, 128, "bf16", seed=11)
+    o, lse = run_fwd(q, k, v, True)
+    assert torch.equal(o[:, :, 0], v[:, :, 0])
+    s00 = (q[:, :, 0].double() * k[:, :, 0].double()).sum(-1) / math.sqrt(128)
+    assert np.allclose(lse[:, :, 0].double().numpy(), s00.numpy(), rtol=0, atol=2e-5)
+
+
+def test_constant_v_gives_constant_o():
+    q, k, _ = make_fwd_inputs(1, 2, 2, 384, 384, 64, "fp16", seed=12)
+    c = torch.randn(64, generator=torch.Generator().manual_seed(13)).half()
+    v = c.expand(1, 2, 384, 64).contiguous()
+    o, _ = run_fwd(q, k, v, True)
+    assert (o.float() - c.float()).abs().max().item() <= 2e-3
+
+
+def test_one_hot_scores_select_one_value_row():
+    """q = c e1, k_j* = e1, other keys 0, c*scale = 200: every other weight is 2^-288 (0 in
+    fp32), so O = V[j*] exactly."""
+    N, d = 256, 64
+    q = torch.zeros(1, 1, N, d, dtype=torch.bfloat16)
+    q[..., 0] = 1600.0
+    k = torch.zeros(1, 1, N, d, dtype=torch.bfloat16)
+    k[0, 0, 173, 0] = 1.0
+    v = torch.randn(1, 1, N, d, generator=torch.Generator().manual_seed(14)).bfloat16()
+    o, lse = run_fwd(q, k, v, False, scale=0.125)
+    assert torch.equal(o[0, 0], v[0, 0, 173].expand(N, d))
+    assert np.allclose(lse.numpy(), 200.0, rtol=0, atol=1e-4)
+
+
+def test_poisoned_padding_and_guard_bands():
+    """NaN in the memory right after K, V and Q must not leak into O; memory right after
+    O and LSE must stay untouched (the kernel writes only [0, Nq) rows)."""
+    N, d, pad = 200, 128, 256
+    q, k, v = make_fwd_inputs(1, 1, 1, N, N, d, "bf16", seed=15)
+    bufs = []
+    for t in (q, k, v):
+        b = torch.full((N + pad, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+        b[:N] = t[0, 0].to(DEV)
+        bufs.append(b)
+    obuf = torch.full((N + pad, d), 7.0, dtype=torch.bfloat16, device=DEV)
+    lbuf = torch.full((N + pad,), 9.0, dtype=torch.float32, device=DEV)
+    qv, kv, vv = (b[:N].view(1, 1, N, d) for b in bufs)
+    fa.fwd(qv, kv, vv, causal=True, out=obuf[:N].view(1, 1, N, d), lse=lbuf[:N].view(1, 1, N))
+    torch.cuda.synchronize()
+    assert fa.device_status() == fa.FA_OK
+    O, L = attention_f64(q, k, v, True, 1 / math.sqrt(d))
+    assert_close(obuf[:N].view(1, 1, N, d).cpu(), lbuf[:N].view(1, 1, N).cpu(), O, L, "bf16", "poison")
+    assert torch.all(obuf[N:] == 7.0) and torch.all(lbuf[N:] == 9.0)
+
+
+def test_lse_may_be_null():
+    q, k, v = make_fwd_inputs(1, 2, 2, 256, 256, 64, "fp16", seed=16)
+    o, lse = fa.fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=True, return_lse=False)
+    torch.cuda.synchronize()
+    assert lse is None
+    O, _ = attention_f64(q, k, v, True, 0.125)
+    assert_close(o.cpu(), None, O, None, "fp16", "no-lse")
+
+
+def test_repeated_calls_are_deterministic():
+    q, k, v = make_fwd_inputs(1, 4, 2, 1000, 1000, 128, "bf16", seed=17)
+    q, k, v = q.to(DEV), k.to(DEV), v.to(DEV)
+    o1, l1 = fa.fwd(q, k, v, causal=True)
+    o2, l2 = fa.fwd(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """Test hook: the Q load is never issued, so the waits on it run out after 20 ms; the
+    kernel records FA_ERR_DEVICE_TIMEOUT and returns, and the next call works."""
+    q, k, v = make_fwd_inputs(1, 1, 1, 256, 256, 64, "fp16", seed=18)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    assert fa.device_status(clear=True) == fa.FA_OK
+    fa.set_wait_timeout_ns(20_000_000)
+    fa.debug_skip_q_load(True)
+    try:
+        fa.fwd(qd, kd, vd, causal=True)
+        status = fa.device_status(clear=True)
+    finally:
+        fa.debug_skip_q_load(False)
+        fa.set_wait_timeout_ns(0)
+    assert status == fa.FA_ERR_DEVICE_TIMEOUT
+    o, lse = fa.fwd(qd, kd, vd, causal=True)
+    torch.cuda.synchronize()
+    assert fa.device_status() == fa.FA_OK
+    O, L = attention_f64(q, k, v, True, 0.125)
+    assert_close(o.cpu(), lse.cpu(), O, L, "fp16", "after-timeout")
+
+
+@pytest.mark.parametrize("name", ["gqa8k", "gqa32k"])
+def test_long_gqa_workloads_sampled_rows(name):
+    """Full-size GQA causal prefill (N = 8192 and 32768, d = 128, bf16) in the launch the
+    benchmark times; the oracle checks seeded rows of every head (tile edges included)."""
+    w = WORKLOADS[name]
+    q, k, v = make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed)
+    o, lse = run_fwd(q, k, v, True, w.scale)
+    rows = sample_rows(w.N, 48 if name == "gqa32k" else 96, seed=w.N)
+    o_s, l_s, O_s, L_s = [], [], [], []
+    for h in range(w.Hq):
+        Oh, Lh = attention_rows_f64(q, k, v, True, w.scale, 0, h, rows)
+        o_s.append(to_f64(o[0, h, rows]))
+        l_s.append(to_f64(lse[0, h, rows]))
+        O_s.append(Oh)
+        L_s.append(Lh)
+    assert_close(np.stack(o_s), np.stack(l_s), np.stack(O_s), np.stack(L_s), w.dtype, name)
+    # properties at every row: finite, and |O| bounded by max |V| (O is a convex combination)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    assert o.float().abs().max() <= v.float().abs().max() + 1e-2
