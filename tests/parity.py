@@ -44,12 +44,27 @@ def metrics(o_gpu, lse_gpu, O_ref, L_ref):
     return out
 
 
-def assert_close(o_gpu, lse_gpu, O_ref, L_ref, dtype: str, what: str = ""):
+def rounding_floor_rms(O_ref, dtype: str) -> float:
+    """RMS error of the oracle's own output after rounding it to the output dtype: the
+    smallest RMS error any implementation that returns `dtype` can have."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(O_ref, dtype=np.float64))
+    r = t.float().to({"fp16": torch.float16, "bf16": torch.bfloat16}[dtype]).double()
+    return float(torch.sqrt(torch.mean((r - t) ** 2))) if t.numel() else 0.0
+
+
+def assert_close(o_gpu, lse_gpu, O_ref, L_ref, dtype: str, what: str = "", strict: bool = True):
+    """strict=True: the stated tolerances, used for the five named workloads. strict=False
+    (edge cases: a handful of keys, so |O| ~ 1 and 16-bit output rounding alone can exceed
+    1e-3 RMS): the RMS bound becomes max(1e-3, 1.5 x the rounding floor of the exact
+    output in `dtype`); max-abs and LSE bounds are unchanged."""
     m = metrics(o_gpu, lse_gpu, O_ref, L_ref)
     assert np.all(np.isfinite(to_f64(o_gpu) if not isinstance(o_gpu, np.ndarray) else o_gpu)), \
         f"{what}: non-finite output"
     assert m["max_abs"] <= MAX_ABS[dtype], f"{what}: max-abs {m['max_abs']:.3e} > {MAX_ABS[dtype]} {m}"
-    assert m["rms"] <= RMS_TOL, f"{what}: rms {m['rms']:.3e} > {RMS_TOL} {m}"
+    rms_tol = RMS_TOL if strict else max(RMS_TOL, 1.5 * rounding_floor_rms(O_ref, dtype))
+    m["rms_tol"] = rms_tol
+    assert m["rms"] <= rms_tol, f"{what}: rms {m['rms']:.3e} > {rms_tol:.3e} {m}"
     if lse_gpu is not None:
         assert m["lse_nonfinite_mismatch"] == 0, f"{what}: -inf pattern of LSE differs {m}"
         assert m["lse_rel"] <= LSE_REL, f"{what}: LSE rel {m['lse_rel']:.3e} > {LSE_REL} {m}"
