@@ -119,6 +119,38 @@ FA_API fa_status fa_decode(const void* q, const void* kcache, const void* vcache
                     float scale, fa_dtype dtype, void* workspace, size_t workspace_bytes,
                     void* stream);
 
+/*
+ * fa_decode_noalloc — fa_decode for callers that cannot allocate device memory.
+ *
+ * Not from the pages (they have no counterpart): a convenience form of fa_decode whose
+ * split-KV scratch is a fixed array compiled into this library instead of a
+ * caller-provided workspace. Some callers cannot call cudaMalloc at the point where they
+ * decode: an inference server that has handed almost all device memory to its own pool
+ * and KV cache up front (a fresh cudaMalloc would fail or fragment that pool), a plugin
+ * that is given tensors but no allocator, or a latency-critical decode loop that must not
+ * pay cudaMalloc/cudaFree's cost and implicit device-wide synchronisation. This entry
+ * point needs nothing beyond the inputs and outputs, and it calls no allocating routine.
+ *
+ * Arguments, layouts, ownership and results are those of fa_decode, minus the workspace.
+ * Limits and behaviour:
+ *  - the scratch is FA_DECODE_NOALLOC_SCRATCH_BYTES (32 MiB) of device memory per GPU,
+ *    reserved when the library's device code is loaded on that GPU and held until the
+ *    process exits; calls whose fa_decode_workspace_bytes(B, Hq, max_kv_len, d) exceeds
+ *    it return FA_ERR_WORKSPACE without launching anything;
+ *  - the first call on each device looks up the scratch's device address (with that
+ *    device current); make that first call before any stream capture;
+ *  - every call on a device shares the one scratch array, which keeps the previous call's
+ *    contents (the kernels overwrite every slot they later read, so nothing needs
+ *    clearing); two calls whose kernels may overlap on the GPU (different streams, or
+ *    different host threads) race on it and give wrong results. Serialise them, or use
+ *    fa_decode with separate workspaces.
+ */
+#define FA_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)
+FA_API fa_status fa_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                                   const int* kv_lens, void* o, float* lse,
+                                   int B, int Hq, int Hkv, int max_kv_len, int d,
+                                   float scale, fa_dtype dtype, void* stream);
+
 /* fa_status_string — static, human-readable name of a status code (never NULL). */
 FA_API const char* fa_status_string(fa_status s);
 

@@ -23,7 +23,8 @@ __all__ = ["FAError", "FALibraryError", "LIB_PATH", "lib", "fwd", "decode",
            "decode_workspace_bytes", "device_status", "set_wait_timeout_ns",
            "debug_skip_q_load", "build_info", "status_string", "EXPORTED_SYMBOLS",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_ALIGNMENT",
-           "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_FP16", "FA_BF16"]
+           "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_FP16", "FA_BF16",
+           "decode_noalloc", "DECODE_NOALLOC_SCRATCH_BYTES"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
 
@@ -33,7 +34,10 @@ FA_FP16, FA_BF16 = 0, 1
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode", "fa_decode_workspace_bytes", "fa_status_string",
                     "fa_device_status", "fa_set_wait_timeout_ns", "fa_debug_skip_q_load",
-                    "fa_build_info")
+                    "fa_build_info", "fa_decode_noalloc")
+
+# Size of the library's fixed decode scratch (FA_DECODE_NOALLOC_SCRATCH_BYTES in fa.h).
+DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class FALibraryError(RuntimeError):
@@ -82,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.fa_debug_skip_q_load.restype = None
         L.fa_build_info.argtypes = []
         L.fa_build_info.restype = ctypes.c_char_p
+        L.fa_decode_noalloc.argtypes = [c_void_p] * 6 + [c_int] * 5 + [c_float, c_int, c_void_p]
+        L.fa_decode_noalloc.restype = c_int
         _lib = L
         return L
 
@@ -208,4 +214,43 @@ def decode(q, kcache, vcache, kv_lens, scale: Optional[float] = None, out=None, 
                          _stream_ptr(stream))
     if st != FA_OK:
         raise FAError(st, "fa_decode")
+    return out, lse
+
+
+def decode_noalloc(q, kcache, vcache, kv_lens, scale: Optional[float] = None, out=None, lse=None,
+                   return_lse: bool = True, stream=None):
+    """Decode via ``fa_decode_noalloc``: same arguments and results as `decode`, but the
+    split-KV scratch is the library's own fixed 32 MiB device array, so the library itself
+    allocates nothing (for callers that cannot call cudaMalloc: a serving process whose
+    device memory is already handed to its own pool, a plugin without an allocator, or a
+    latency-critical loop that must avoid cudaMalloc's cost and synchronisation). Calls on
+    one device share that scratch: do not let two of them overlap on the GPU. `out` and
+    `lse` are allocated here only if the caller does not pass them.
+    """
+    import torch
+    _check(q, "q", 3, q.device)
+    _check(kcache, "kcache", 4, q.device)
+    _check(vcache, "vcache", 4, q.device)
+    _check(kv_lens, "kv_lens", 1, q.device)
+    if kv_lens.dtype != torch.int32:
+        raise TypeError("kv_lens must be int32")
+    if kcache.dtype != q.dtype or vcache.dtype != q.dtype:
+        raise TypeError("q and the caches must share one dtype")
+    B, Hq, d = q.shape
+    Bk, Hkv, max_len, dk = kcache.shape
+    if tuple(vcache.shape) != tuple(kcache.shape) or Bk != B or dk != d or kv_lens.shape[0] != B:
+        raise ValueError("shape mismatch between q, caches and kv_lens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    st = lib().fa_decode_noalloc(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
+                                 kv_lens.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr() if lse is not None else None,
+                                 B, Hq, Hkv, max_len, d, float(scale), _dtype_code(q),
+                                 _stream_ptr(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_decode_noalloc")
     return out, lse

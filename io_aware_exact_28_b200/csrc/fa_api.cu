@@ -285,6 +285,52 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
               : launch_decode_g<128, false>(dp, cp, B, Hkv, G, st);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Allocation-free decode: split-KV scratch in a fixed device array of this file. In host
+// code `g_decode_noalloc_scratch` names a host-side stand-in, not device memory, so its
+// device address is looked up once per device with cudaGetSymbolAddress (with that device
+// current) and only that address is handed to the kernels.
+// ---------------------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_decode_noalloc_scratch[FA_DECODE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_scratch_ptr[kMaxDevices];
+
+fa_status noalloc_scratch_address(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_noalloc_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return FA_ERR_CUDA;
+    g_noalloc_scratch_ptr[dev] = p;
+  }
+  *out = g_noalloc_scratch_ptr[dev];
+  return FA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+fa_status fa_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                            const int* kv_lens, void* o, float* lse, int B, int Hq, int Hkv,
+                            int max_kv_len, int d, float scale, fa_dtype dtype, void* stream) {
+  const size_t need = fa_decode_workspace_bytes(B, Hq, max_kv_len, d);
+  if (need == 0)   // invalid sizes: let fa_decode report them without touching CUDA
+    return fa_decode(q, kcache, vcache, kv_lens, o, lse, B, Hq, Hkv, max_kv_len, d, scale,
+                     dtype, nullptr, 0, stream);
+  if (need > FA_DECODE_NOALLOC_SCRATCH_BYTES) return FA_ERR_WORKSPACE;
+  int dev = 0;
+  fa_status s = check_device(&dev);
+  if (s != FA_OK) return s;
+  void* scratch = nullptr;
+  s = noalloc_scratch_address(dev, &scratch);
+  if (s != FA_OK) return s;
+  return fa_decode(q, kcache, vcache, kv_lens, o, lse, B, Hq, Hkv, max_kv_len, d, scale, dtype,
+                   scratch, FA_DECODE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 const char* fa_status_string(fa_status s) {
   switch (s) {
     case FA_OK: return "FA_OK";
