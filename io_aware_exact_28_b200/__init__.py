@@ -26,7 +26,9 @@ __all__ = ["FAError", "FALibraryError", "LIB_PATH", "lib", "fwd", "decode",
            "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_FP16", "FA_BF16",
            "decode_noalloc", "DECODE_NOALLOC_SCRATCH_BYTES"]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
+# FA_B200_LIB may name another build of the same library (e.g. a variant for timing).
+LIB_PATH = os.environ.get("FA_B200_LIB") or \
+    os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
 
 FA_FP16, FA_BF16 = 0, 1
 (FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ALIGNMENT, FA_ERR_CUDA,

@@ -25,10 +25,11 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def command(verbose: bool = False) -> list[str]:
+def command(verbose: bool = False, out: str = OUT, defines=()) -> list[str]:
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo",
            "-std=c++17", "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-           "-I", os.path.join(ROOT, "include"), "-I", HERE, "-o", OUT] + SOURCES + ["-cudart", "static"]
+           "-I", os.path.join(ROOT, "include"), "-I", HERE, "-o", out] + \
+        [f"-D{d}" for d in defines] + SOURCES + ["-cudart", "static"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     return cmd
@@ -41,14 +42,15 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if force or verbose or not up_to_date():
-        proc = subprocess.run(command(verbose), capture_output=True, text=True)
+def build(force: bool = False, verbose: bool = False, out: str = OUT, defines=()) -> str:
+    """Compile (if stale) to `out`; `defines` (e.g. "FA_SOFTMAX_F32X2=0") build a variant."""
+    if force or verbose or out != OUT or defines or not up_to_date():
+        proc = subprocess.run(command(verbose, out, defines), capture_output=True, text=True)
         if proc.returncode != 0:
             raise RuntimeError(f"nvcc failed ({proc.returncode}):\n{proc.stdout}\n{proc.stderr}")
         if verbose:
             sys.stderr.write(proc.stderr)
-    return OUT
+    return out
 
 
 if __name__ == "__main__":

@@ -67,16 +67,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [heads, rows, d] 16-bit tensor, box = 64 columns (128 bytes) x 128 rows x 1 head,
+// [heads, rows, d] 16-bit tensor, box = 64 columns (128 bytes) x box_rows rows x 1 head,
 // 128-byte swizzle; rows past `rows` read as zero and are clipped on store.
-bool make_tile_map(CUtensorMap* m, const void* ptr, int d, int rows, long long heads, bool bf16) {
+bool make_tile_map(CUtensorMap* m, const void* ptr, int d, int rows, long long heads, bool bf16,
+                   int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(heads)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                                  static_cast<cuuint64_t>(rows) * d * 2};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(fa::kBM), 1};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
              const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -93,19 +94,27 @@ fa_status launch_fwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
                      cudaStream_t stream) {
   using C = fa::FwdCfg<D>;
   auto kernel = fa::fa_fwd_kernel<D, BF16, CAUSAL>;
-  static bool attr_set[kMaxDevices];
+  static int attr_state[kMaxDevices];   // 0 unknown, 1 ready, 2 unusable build
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!attr_set[dev]) {
+    if (attr_state[dev] == 0) {
       if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               C::SMEM_BYTES) != cudaSuccess)
+                               C::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return FA_ERR_CUDA;
-      attr_set[dev] = true;
+      // The in-kernel register re-split hands out exactly the launch allocation; a build
+      // whose compiled register count differs would make it wait forever, so refuse it.
+      cudaFuncAttributes fattr;
+      if (cudaFuncGetAttributes(&fattr, kernel) != cudaSuccess) return FA_ERR_CUDA;
+      attr_state[dev] =
+          (!C::REGSPLIT || static_cast<uint32_t>(fattr.numRegs) == C::REGS_LAUNCH) ? 1 : 2;
     }
+    if (attr_state[dev] != 1) return FA_ERR_UNSUPPORTED;
   }
   const int n_qblocks = (Nq + fa::kQTiles * fa::kBM - 1) / (fa::kQTiles * fa::kBM);
   dim3 grid(BH, n_qblocks, 1);
-  kernel<<<grid, fa::kFwdThreads, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
+  kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -198,8 +207,11 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
   const bool bf16 = dtype == FA_BF16;
   CUtensorMap mq, mk, mv, mo;
-  if (!make_tile_map(&mq, q, d, Nq, BH, bf16) || !make_tile_map(&mk, k, d, Nk, BHkv, bf16) ||
-      !make_tile_map(&mv, v, d, Nk, BHkv, bf16) || !make_tile_map(&mo, o, d, Nq, BH, bf16))
+  const int kv_box = (d == 64) ? fa::FwdCfg<64>::BN : fa::FwdCfg<128>::BN;
+  if (!make_tile_map(&mq, q, d, Nq, BH, bf16, fa::kBM) ||
+      !make_tile_map(&mk, k, d, Nk, BHkv, bf16, kv_box) ||
+      !make_tile_map(&mv, v, d, Nk, BHkv, bf16, kv_box) ||
+      !make_tile_map(&mo, o, d, Nq, BH, bf16, fa::kBM))
     return FA_ERR_CUDA;
 
   fa::FwdParams prm;

@@ -1,7 +1,8 @@
 // fwd_kernel.cuh — exact attention forward (prefill) for sm_100a.
 //
 // One CTA owns 256 query rows of one (batch, query head): two 128-row Q tiles that
-// take turns on the tensor core. Per K/V tile j (128 keys) and Q tile t:
+// take turns on the tensor core. Per K/V tile j (BN keys: 128 at d = 128, 64 at d = 64)
+// and Q tile t:
 //     S_t = Q_t K_j^T                    tcgen05.mma, fp32 accumulator in TMEM
 //     softmax warps: mask, row max, lazy rescale of O_t, P_t = exp2(S*c - m) -> TMEM
 //     O_t += P_t V_j                     tcgen05.mma with A read from TMEM
@@ -12,14 +13,16 @@
 // formula) and page "Flash Attention ... IO-aware exact" (fr), tiling pseudo-code (Q_i
 // read once, K_j/V_j per block, O_i and L written once at the end).
 //
-// Warp roles (320 threads):
+// Warp roles (FwdCfg::THREADS: 384 at d = 128, 320 at d = 64):
 //   warps 0-3  softmax + epilogue for Q tile 0 (thread r owns row r = TMEM lane r)
 //   warps 4-7  softmax + epilogue for Q tile 1
 //   warp  8    TMA producer: Q tiles once, then K_j, V_j through an NS-stage ring
 //   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 10-11 (d = 128 only) idle: they complete warpgroup 2 for the register re-split
 //
-// Tensor memory (512 columns): S_t at columns [128t, 128t+128) (fp32); P_t overwrites
-// the first 64 of those columns as packed 16-bit pairs; O_t at [256 + t*D, 256+(t+1)*D).
+// Tensor memory (FwdCfg::TMEM_COLS): S_t at columns [t*BN, (t+1)*BN) (fp32); P_t
+// overwrites the first BN/2 of those columns as packed 16-bit pairs; O_t at
+// [2*BN + t*D, 2*BN + (t+1)*D).
 //
 // Lazy rescaling: the running maximum m used in the exponent is only raised when a new
 // tile maximum exceeds it by more than 8 (log2 units). O and l are both accumulated
@@ -35,30 +38,66 @@
 namespace fa {
 
 constexpr int kBM = 128;           // query rows per Q tile (one TMEM lane per row)
-constexpr int kBN = 128;           // keys per K/V tile
 constexpr int kQTiles = 2;         // Q tiles per CTA
-constexpr int kFwdThreads = 320;
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
 constexpr uint64_t kDrainNs = 200000000ull;   // 0.2 s limit for abort-path drains
 
+// Polynomial-exp2 pair masks (see FwdCfg::kEmuPairs); off by default: measured slower on
+// B200 at both head dimensions, because the softmax is latency-bound, not MUFU-bound.
+#ifndef FA_EMU_PAIRS_D64
+#define FA_EMU_PAIRS_D64 0u
+#endif
+#ifndef FA_EMU_PAIRS_D128
+#define FA_EMU_PAIRS_D128 0u
+#endif
+#ifndef FA_REGSPLIT
+#define FA_REGSPLIT 1
+#endif
+
+// Per head-dimension configuration.
+//  d = 128: 128-key tiles, one CTA per SM, TMEM S 2x128 + O 2x128 = 512 columns.
+//  d = 64:  64-key tiles, two CTAs per SM (TMEM S 2x64 + O 2x64 = 256 columns each), so
+//           four Q tiles are in flight per SM and one CTA's prologue/epilogue overlaps the
+//           other's main loop: at d = 64 the per-tile softmax <-> MMA round trip, not any
+//           one pipe, is the limit.
 template <int D>
 struct FwdCfg {
+  static constexpr int BN = (D == 64) ? 64 : 128;     // keys per K/V tile
+  static constexpr int CTAS = (D == 64) ? 2 : 1;      // resident CTAs per SM
+  // d = 128: 3 warpgroups (warps 10-11 idle) so the register re-split below can apply;
+  // d = 64: 10 warps, two CTAs per SM share the register file (96 registers per thread).
+  static constexpr int THREADS = (D == 64) ? 320 : 384;
+  static constexpr bool REGSPLIT = (D == 128) && FA_REGSPLIT;
   static constexpr int NCH = D / 64;                  // 128-byte swizzle chunks along d
-  static constexpr int CHUNK_BYTES = kBM * 128;       // 128 rows x 128 bytes
-  static constexpr int TILE_BYTES = kBM * D * 2;      // one 128-row tile of Q, K, V or O
-  static constexpr int NS = (D == 128) ? 4 : 8;       // K/V ring stages
+  static constexpr int Q_CHUNK = kBM * 128;           // 128 rows x 128 bytes
+  static constexpr int KV_CHUNK = BN * 128;
+  static constexpr int Q_TILE_BYTES = kBM * D * 2;    // one 128-row tile of Q or O
+  static constexpr int KV_TILE_BYTES = BN * D * 2;
+  static constexpr int NS = (D == 64) ? 8 : 4;        // K/V ring stages
   static constexpr int Q_OFF = 0;
-  static constexpr int KV_OFF = kQTiles * TILE_BYTES;
-  static constexpr int BAR_OFF = KV_OFF + NS * TILE_BYTES;
+  static constexpr int KV_OFF = kQTiles * Q_TILE_BYTES;
+  static constexpr int BAR_OFF = KV_OFF + NS * KV_TILE_BYTES;
   static constexpr int NBARS = 1 + 2 * NS + 2 * kQTiles + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;   // + slack for 1 KB alignment
-  static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t S_COL = 0;
-  static constexpr uint32_t O_COL = 256;
+  static constexpr uint32_t TMEM_COLS = (D == 64) ? 256 : 512;
+  static constexpr uint32_t S_COL = 0;                // S_t at t * BN
+  static constexpr uint32_t O_COL = kQTiles * BN;     // O_t at O_COL + t * D
+  // Registers per thread: the launch allocation (65536 / (threads * CTAS), rounded down
+  // to 8) is re-split so that warpgroup 2 (producer, MMA, 2 idle warps) keeps REGS_OTHER
+  // and the two softmax warpgroups get REGS_SOFTMAX; the split uses exactly the launch
+  // allocation (checked on the host against the compiled register count).
+  static constexpr uint32_t REGS_LAUNCH = (D == 64) ? 96 : 168;
+  static constexpr uint32_t REGS_OTHER = 72;
+  static constexpr uint32_t REGS_SOFTMAX = 216;
+  static_assert(!REGSPLIT || 128 * REGS_OTHER + 256 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH,
+                "register split");
+  static_assert(THREADS * REGS_LAUNCH * CTAS <= 65536, "register file");
+  // Which of every 8 consecutive P column pairs use the polynomial exp2 (bit i = pair i).
+  static constexpr uint32_t kEmuPairs = (D == 64) ? FA_EMU_PAIRS_D64 : FA_EMU_PAIRS_D128;
   static_assert(O_COL + kQTiles * D <= TMEM_COLS, "TMEM budget");
-  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(SMEM_BYTES * CTAS <= 227 * 1024, "shared memory budget");
 };
 
 struct FwdParams {
@@ -87,7 +126,7 @@ __device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
 }
 
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+__global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::CTAS)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
               const FwdParams p) {
@@ -106,6 +145,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int qb = gridDim.y - 1 - blockIdx.y;        // heaviest (causal) blocks launch first
   const int q0 = qb * (kQTiles * kBM);
 
+  constexpr int kBN = C::BN;
   const int n_kv_total = (p.Nk + kBN - 1) / kBN;
   int n_kv = n_kv_total;
   if (CAUSAL) {
@@ -151,16 +191,19 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, &g_fa_status, p.timeout_ns};
 
-  if (warp == kWarpProducer) {
+  // Each role's code sits inside the branch that set its register budget.
+  if (warp >= 2 * 4) {
+    if constexpr (C::REGSPLIT) setmaxnreg_dec<C::REGS_OTHER>();
+    if (warp == kWarpProducer) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool q_issued = false;
       // A CTA with no visible key tile writes zeros from the softmax warps and needs no Q.
       if (!p.skip_q_load && n_kv > 0) {
-        mbar_arrive_expect_tx(bar_q(), kQTiles * C::TILE_BYTES);
+        mbar_arrive_expect_tx(bar_q(), kQTiles * C::Q_TILE_BYTES);
         for (int t = 0; t < kQTiles; ++t)
           for (int ch = 0; ch < C::NCH; ++ch)
-            tma_load_3d(base + C::Q_OFF + t * C::TILE_BYTES + ch * C::CHUNK_BYTES, &tmQ, bar_q(),
+            tma_load_3d(base + C::Q_OFF + t * C::Q_TILE_BYTES + ch * C::Q_CHUNK, &tmQ, bar_q(),
                         ch * 64, q0 + t * kBM, bh);
         q_issued = true;
       }
@@ -174,10 +217,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar_full(slot), C::TILE_BYTES);
+          mbar_arrive_expect_tx(bar_full(slot), C::KV_TILE_BYTES);
           const CUtensorMap* tm = kv ? &tmV : &tmK;
           for (int ch = 0; ch < C::NCH; ++ch)
-            tma_load_3d(base + C::KV_OFF + slot * C::TILE_BYTES + ch * C::CHUNK_BYTES, tm,
+            tma_load_3d(base + C::KV_OFF + slot * C::KV_TILE_BYTES + ch * C::KV_CHUNK, tm,
                         bar_full(slot), ch * 64, j * kBN, bh_kv);
           ++it;
         }
@@ -189,27 +232,28 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (q_issued) mbar_wait_drain(bar_q(), 0, kDrainNs);
       }
     }
-  } else if (warp == kWarpMma) {
+    } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_kv > 0) {
       constexpr uint32_t IDESC_S = idesc_f16(kBM, kBN, BF16 ? 1u : 0u, 0u, 0u);
       constexpr uint32_t IDESC_O = idesc_f16(kBM, D, BF16 ? 1u : 0u, 0u, 1u);
       auto issue_s = [&](int t, int kslot) {
-        const uint32_t qa = base + C::Q_OFF + t * C::TILE_BYTES;
-        const uint32_t ka = base + C::KV_OFF + kslot * C::TILE_BYTES;
+        const uint32_t qa = base + C::Q_OFF + t * C::Q_TILE_BYTES;
+        const uint32_t ka = base + C::KV_OFF + kslot * C::KV_TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-          mma_f16_ss(tmem + C::S_COL + t * kBN, sdesc_k_sw128(qa + off), sdesc_k_sw128(ka + off),
+          const uint32_t koff = (kk & 3) * 32;
+          mma_f16_ss(tmem + C::S_COL + t * kBN, sdesc_k_sw128(qa + (kk >> 2) * C::Q_CHUNK + koff),
+                     sdesc_k_sw128(ka + (kk >> 2) * C::KV_CHUNK + koff),
                      IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int vslot, bool acc0) {
-        const uint32_t va = base + C::KV_OFF + vslot * C::TILE_BYTES;
+        const uint32_t va = base + C::KV_OFF + vslot * C::KV_TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           mma_f16_ts(tmem + C::O_COL + t * D, tmem + C::S_COL + t * kBN + kk * 8,
-                     sdesc_mn_sw128(va + kk * 2048, C::CHUNK_BYTES), IDESC_O,
+                     sdesc_mn_sw128(va + kk * 2048, C::KV_CHUNK), IDESC_O,
                      (acc0 || kk > 0) ? 1u : 0u);
         }
       };
@@ -253,7 +297,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_wait_drain(bar_drain, 0, kDrainNs);
       }
     }
+    }   // warps 10-11: idle, straight to the final barrier
   } else {
+    if constexpr (C::REGSPLIT) setmaxnreg_inc<C::REGS_SOFTMAX>();
     // ------------------------------------------------------------------ softmax + epilogue
     const int t = warp >> 2;
     const int r = threadIdx.x & (kBM - 1);
@@ -272,22 +318,47 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     for (int j = 0; j < n_kv; ++j) {
       if (!mbar_wait(bar_s(t), j & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[kBN];
-      tmem_ld32x32b_x128(tS, sr);
       const int key0 = j * kBN;
-      if (key0 + kBN - 1 > lim_min) {               // tile-uniform: diagonal or ragged tile
+      const bool masked_tile = key0 + kBN - 1 > lim_min;   // tile-uniform: diagonal or ragged
+      // Scores of a 32-column chunk cc, with masked keys set to -inf.
+      auto mask_chunk = [&](uint32_t (&v)[32], int cc) {
+        if (masked_tile) {
 #pragma unroll
-        for (int k = 0; k < kBN; ++k)
-          if (key0 + k > lim) sr[k] = __float_as_uint(-CUDART_INF_F);
-      }
-      float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
+          for (int k = 0; k < 32; ++k)
+            if (key0 + 32 * cc + k > lim) v[k] = __float_as_uint(-CUDART_INF_F);
+        }
+      };
+      // Row maximum over 8 independent chains (short dependency chains).
+      float mx8[8];
 #pragma unroll
-      for (int k = 0; k < kBN; k += 2) {
-        mx0 = fmaxf(mx0, __uint_as_float(sr[k]));
-        mx1 = fmaxf(mx1, __uint_as_float(sr[k + 1]));
+      for (int i = 0; i < 8; ++i) mx8[i] = -CUDART_INF_F;
+      auto max_chunk = [&](const uint32_t (&v)[32]) {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], __uint_as_float(v[k]));
+      };
+      // d = 128 keeps the whole 128-score row in registers; d = 64 (two CTAs per SM, 96
+      // registers) reads its 64-score row from TMEM twice: once for the max, once for P.
+      constexpr bool kResident = (kBN == 128);
+      uint32_t sr[kResident ? kBN : 32];
+      if constexpr (kResident) {
+        tmem_ld32x32b_x128(tS, sr);
+#pragma unroll
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          uint32_t (&v)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]);
+          mask_chunk(v, cc);
+          max_chunk(v);
+        }
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          tmem_ld32x32b_x32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]), cc);
+          max_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        }
       }
-      const float mx = fmaxf(mx0, mx1) * c;          // scale > 0, -inf stays -inf
-      if (mx > m_used + 8.0f) {
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * c;
+      if (mx > m_used + 8.0f) {                      // scale > 0: -inf stays -inf
         if (m_used != -CUDART_INF_F) {               // O_t and l hold earlier tiles
           const float alpha = ex2_approx(m_used - mx);
           l *= alpha;
@@ -296,18 +367,47 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         m_used = mx;
       }
       const float mref = (m_used == -CUDART_INF_F) ? 0.f : m_used;
-      uint32_t pk[kBN / 2];
-      float l0 = 0.f, l1 = 0.f;
+      // P = 2^(s*c - m) in 32-column chunks, each stored to TMEM as 16 packed columns
+      // (P_t occupies S_t columns [0, BN/2); chunk cc only overwrites columns already read).
+      // In tiles without masked scores, the pairs selected by kEmuPairs are evaluated
+      // with the FMA-pipe polynomial instead of MUFU.EX2. The argument s*c - m and the
+      // row sum use packed f32x2 arithmetic.
+      const uint64_t c2 = f2_pack(c, c);
+      const uint64_t nm2 = f2_pack(-mref, -mref);
+      uint64_t l2a = f2_pack(0.f, 0.f), l2b = l2a;
 #pragma unroll
-      for (int k = 0; k < kBN / 2; ++k) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * k]), c, -mref));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * k + 1]), c, -mref));
-        l0 += p0;
-        l1 += p1;
-        pk[k] = pack_half2(p0, p1, BF16);
+      for (int cc = 0; cc < kBN / 32; ++cc) {
+        if constexpr (!kResident) {
+          tmem_ld32x32b_x32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]), cc);
+        }
+        const uint32_t* v = kResident ? &sr[32 * cc] : &sr[0];
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint64_t x2 =
+              f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2);
+          uint64_t p2;
+          if (!masked_tile && ((FwdCfg<D>::kEmuPairs >> (i & 7)) & 1u)) {
+            p2 = exp2_poly_f2(x2);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          }
+          if (i & 1) l2b = f2_add(l2b, p2); else l2a = f2_add(l2a, p2);
+          float p0, p1;
+          f2_unpack(p2, p0, p1);
+          pk[i] = pack_half2(p0, p1, BF16);
+        }
+        tmem_st32x32b_x16(tS + cc * 16, pk);
       }
-      l += l0 + l1;
-      tmem_st32x32b_x64(tS, pk);                    // P_t into S_t columns [0, 64)
+      {
+        float la, lb, lc, ld;
+        f2_unpack(l2a, la, lb);
+        f2_unpack(l2b, lc, ld);
+        l += (la + lb) + (lc + ld);
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_p(t));
@@ -316,14 +416,17 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       ok = mbar_wait(bar_s(t), n_kv & 1, wc);       // final PV of this tile done
       tc_fence_after();
     }
-    uint8_t* otile = sbase + C::Q_OFF + t * C::TILE_BYTES;   // Q_t no longer read
+    uint8_t* otile = sbase + C::Q_OFF + t * C::Q_TILE_BYTES;   // Q_t no longer read
     if (ok) {
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll
       for (int ch = 0; ch < C::NCH; ++ch) {
         uint32_t o[64];
         if (n_kv > 0) {
-          tmem_ld32x32b_x64(tO + ch * 64, o);
+          uint32_t (&o_lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
+          uint32_t (&o_hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[32]);
+          tmem_ld32x32b_x32(tO + ch * 64, o_lo);
+          tmem_ld32x32b_x32(tO + ch * 64 + 32, o_hi);
         } else {
 #pragma unroll
           for (int i = 0; i < 64; ++i) o[i] = 0u;
@@ -336,7 +439,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           w.z = pack_half2(__uint_as_float(o[8 * u + 4]) * inv_l, __uint_as_float(o[8 * u + 5]) * inv_l, BF16);
           w.w = pack_half2(__uint_as_float(o[8 * u + 6]) * inv_l, __uint_as_float(o[8 * u + 7]) * inv_l, BF16);
           // 128-byte swizzle: 16-byte unit u of row r sits at unit u ^ (r mod 8)
-          *reinterpret_cast<uint4*>(otile + ch * C::CHUNK_BYTES + r * 128 + ((u ^ (r & 7)) << 4)) = w;
+          *reinterpret_cast<uint4*>(otile + ch * C::Q_CHUNK + r * 128 + ((u ^ (r & 7)) << 4)) = w;
         }
       }
       if (p.lse != nullptr && row < p.Nq) {
@@ -348,7 +451,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     named_barrier_sync(1 + t, kBM);
     if (r == 0 && ok && !*abort_flag) {
       for (int ch = 0; ch < C::NCH; ++ch)
-        tma_store_3d(&tmO, smem_u32(otile + ch * C::CHUNK_BYTES), ch * 64, q0 + t * kBM, bh);
+        tma_store_3d(&tmO, smem_u32(otile + ch * C::Q_CHUNK), ch * 64, q0 + t * kBM, bh);
       tma_store_commit_and_wait_read();
     }
   }

@@ -40,6 +40,75 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi, bool bf16) {
   return r;
 }
 
+// ---------------------------------------------------------------------------------------
+// Packed fp32 pairs (sm_100 f32x2 instructions): one instruction, two lanes of math.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x on the FMA pipe for two values at once, for x <= 2^7 (inputs below -126 are
+// clamped to -126, giving a tiny positive result instead of 0; callers use it only where
+// no score is masked). x = j + f with j = round-to-nearest(x) (the 1.5*2^23 shifter),
+// |f| <= 1/2; 2^f is a degree-4 polynomial with minimax relative error 2.7e-6 (fp32
+// Horner), fitted by fit_exp2_poly.py (Lawson's re-weighted least squares); j is then
+// added to the result's exponent field.
+constexpr float kExp2C0 = 0x1.ffffe8p-1f;   // 0.999999285
+constexpr float kExp2C1 = 0x1.62e0dcp-1f;   // 0.693121791
+constexpr float kExp2C2 = 0x1.ec06dap-3f;   // 0.240247443
+constexpr float kExp2C3 = 0x1.ca1442p-5f;   // 0.0559178628
+constexpr float kExp2C4 = 0x1.3997d4p-7f;   // 0.00957010128
+
+__device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t shifter = f2_pack(12582912.f, 12582912.f);       // 1.5 * 2^23
+  const uint64_t t = f2_add(xc, shifter);                         // shifter + j (exact)
+  const uint64_t f = f2_sub(xc, f2_sub(t, shifter));              // x - j, exact
+  uint64_t p = f2_fma(f2_pack(kExp2C4, kExp2C4), f, f2_pack(kExp2C3, kExp2C3));
+  p = f2_fma(p, f, f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  // bits(t) = bits(shifter) + j; shifting left by 23 keeps exactly j << 23.
+  const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
+  const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
+  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+}
+
+// Warpgroup-wide register re-allocation (all four warps of a warpgroup execute it).
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(N));
+}
+
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(nthreads) : "memory");
 }
