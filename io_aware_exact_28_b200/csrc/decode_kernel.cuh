@@ -2,21 +2,26 @@
 //
 // Decode reads every valid K and V row of the cache once per step, so it is bound by
 // device-memory bandwidth (page "Empreinte mémoire et calcul des couches Transformer":
-// KV-cache size per token and the memory-bound character of cache access). The kernel
-// therefore streams the cache with coalesced 128-bit loads, reads each K/V row once for
-// all G = Hq/Hkv query heads that share it, and keeps the math in fp32 registers.
+// KV-cache size per token and the memory-bound character of cache access). The split
+// kernel therefore
+//   * streams each split's K and V rows into a shared-memory ring with bulk TMA copies
+//     (the rows of one split are contiguous, so one copy per tensor per stage), keeping
+//     many bytes in flight without spending registers on them;
+//   * reads each K/V row once for all G = Hq/Hkv query heads that share it;
+//   * computes in fp32, two lanes of math per instruction (f32x2 FMA).
 //
-// Split kernel: grid (split, kv head x head tile, sequence), 128 threads. A split covers
-// up to `split_tokens` consecutive cache rows. Each token row is read by D/8 lanes (8
-// elements = 16 bytes per lane); each warp runs its own online softmax over its tokens
-// (running max with the same lazy-rescale rule as the prefill kernel), the four warps
-// merge through shared memory, and the CTA writes a normalised partial O row and its
-// log2-domain logsumexp per query head.
+// Split kernel: grid (split, kv head x head tile, sequence), 128 threads (4 warps). A
+// split covers up to `split_tokens` consecutive cache rows in stages of 32 tokens. Each
+// token row is read from shared memory by LPT lanes (DPL = D/LPT elements per lane), the
+// LPT partial dot products are summed with xor-shuffles, and each warp runs its own online
+// softmax over its tokens (running max with the lazy-rescale rule of the prefill kernel).
+// The four warps merge through shared memory and the CTA writes, per query head, a
+// normalised partial O row and its log2-domain logsumexp.
 //
-// Combine kernel: grid (sequence x query head), D threads. Merges the valid splits with
-// weights 2^(lse_s - max) (the online-softmax rescaling identity, page "Kotaemon
-// FlashAttention", running max and normaliser bullet) and writes O (16-bit) and the
-// natural-log LSE.
+// Combine kernel: grid (sequence x query head), D threads, launched as a programmatic
+// dependent of the split kernel. It merges the valid splits with weights 2^(lse_s - max)
+// (the online-softmax rescaling identity, page "Kotaemon FlashAttention", running max and
+// normaliser bullet) and writes O (16-bit) and the natural-log LSE.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -29,7 +34,8 @@ namespace fa {
 
 constexpr int kDecThreads = 128;
 constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kDecUnroll = 4;       // token groups per warp per batch (loads in flight)
+constexpr int kDecStageTok = 32;     // tokens per ring stage
+constexpr int kDecStages = 4;        // ring depth
 
 struct DecodeParams {
   const uint16_t* q;      // [B, Hq, D]
@@ -41,41 +47,63 @@ struct DecodeParams {
   int Hq, Hkv, G;         // G = Hq / Hkv
   int max_len, split_tokens, n_split;
   float scale_log2;
+  uint64_t timeout_ns;
 };
-
-__device__ __forceinline__ uint4 ld_stream_u4(const void* ptr) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(ptr));
-  return v;
-}
-
-template <bool BF16>
-__device__ __forceinline__ void unpack8(const uint4& w, float (&f)[8]) {
-  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (BF16) {
-      f[2 * i] = __uint_as_float(u[i] << 16);
-      f[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
-    } else {
-      const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&u[i]));
-      f[2 * i] = x.x;
-      f[2 * i + 1] = x.y;
-    }
-  }
-}
 
 __device__ __forceinline__ int clamp_len(int n, int max_len) {
   return n < 0 ? 0 : (n > max_len ? max_len : n);
 }
 
+// 16-byte shared-memory load.
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// Bulk (non-tensor) TMA copy global -> shared, completing on an mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar) : "memory");
+}
+
+// Two 16-bit values in one 32-bit word -> an f32x2 pair (low element first).
+template <bool BF16>
+__device__ __forceinline__ uint64_t half2_to_f2(uint32_t w) {
+  if (BF16) return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&w));
+  return f2_pack(x.x, x.y);
+}
+
+template <int D, int GT>
+struct DecCfg {
+  // Lanes per token row: 8 while GT*D/8 registers of q and of the accumulator stay <= 64
+  // per lane, otherwise 16.
+  static constexpr int LPT = (GT * (D / 8) <= 64) ? 8 : 16;
+  static constexpr int DPL = D / LPT;                 // elements per lane (8 or 16)
+  static constexpr int NV = DPL / 8;                  // 16-byte loads per lane per row
+  static constexpr int TPI = 32 / LPT;                // tokens per warp instruction
+  static constexpr int TPW = kDecStageTok / kDecWarps;  // tokens per warp per stage
+  static constexpr int GROUPS = TPW / TPI;            // token groups per warp per stage
+  static constexpr int ROW = D * 2;                   // bytes per token row
+  static constexpr int STAGE_BYTES = kDecStageTok * ROW;
+  static constexpr int SMEM_BYTES = 2 * kDecStages * STAGE_BYTES + 2 * kDecStages * 8 + 16;
+  // Three CTAs per SM (<= 168 registers) where the head tile allows it without spills.
+  static constexpr int MIN_BLOCKS = (GT == 8) ? 2 : 3;
+  static_assert(GROUPS >= 1 && TPW % TPI == 0, "stage split");
+};
+
 template <int D, int GT, bool BF16>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, DecCfg<D, GT>::MIN_BLOCKS)
 fa_decode_split_kernel(const DecodeParams p) {
-  constexpr int LPT = D / 8;           // lanes per token row
-  constexpr int TPI = 32 / LPT;        // tokens per warp per load instruction
-  constexpr int TOK_PER_BATCH = kDecUnroll * kDecWarps * TPI;
+  using C = DecCfg<D, GT>;
+  extern __shared__ __align__(128) uint8_t dsmem[];
+
+  // Let the dependent combine kernel launch as soon as every split CTA has started; it
+  // waits for this grid to finish before reading anything.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int split = blockIdx.x;
   const int n_gt = (p.G + GT - 1) / GT;
@@ -86,140 +114,225 @@ fa_decode_split_kernel(const DecodeParams p) {
   const int t0 = split * p.split_tokens;
   if (t0 >= len) return;                               // this split is never merged
   const int t1 = min(len, t0 + p.split_tokens);
+  const int n_stages = (t1 - t0 + kDecStageTok - 1) / kDecStageTok;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int sub = lane / LPT;                          // which token of the instruction
-  const int dofs = (lane % LPT) * 8;
+  const int sub = lane / C::LPT;                       // token of the instruction
+  const int li = lane % C::LPT;                        // lane within the token's group
+
+  const uint32_t sK = smem_u32(dsmem);
+  const uint32_t sV = sK + kDecStages * C::STAGE_BYTES;
+  const uint32_t bar_full = sV + kDecStages * C::STAGE_BYTES;   // kDecStages x 8 bytes
+  const uint32_t bar_empty = bar_full + kDecStages * 8;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(dsmem + 2 * kDecStages * C::STAGE_BYTES +
+                                                             2 * kDecStages * 8);
+  const WaitCtl wc{abort_flag, &g_fa_status, p.timeout_ns};
 
   const size_t kv_base = (static_cast<size_t>(b) * p.Hkv + kvh) * p.max_len * D;
-  const uint16_t* kp = p.kc + kv_base + dofs;
-  const uint16_t* vp = p.vc + kv_base + dofs;
+  const uint16_t* kg = p.kc + kv_base + static_cast<size_t>(t0) * D;
+  const uint16_t* vg = p.vc + kv_base + static_cast<size_t>(t0) * D;
 
-  // This lane's slice of the query rows, pre-multiplied by scale*log2(e).
-  float qf[GT][8];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, kDecWarps);
+    }
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  auto issue = [&](int st) {               // thread 0: fill ring slot st % kDecStages
+    const int slot = st % kDecStages;
+    const int n = min(kDecStageTok, t1 - (t0 + st * kDecStageTok));
+    const uint32_t bytes = static_cast<uint32_t>(n) * C::ROW;
+    mbar_arrive_expect_tx(bar_full + 8 * slot, 2 * bytes);
+    bulk_load(sK + slot * C::STAGE_BYTES, kg + static_cast<size_t>(st) * kDecStageTok * D, bytes,
+              bar_full + 8 * slot);
+    bulk_load(sV + slot * C::STAGE_BYTES, vg + static_cast<size_t>(st) * kDecStageTok * D, bytes,
+              bar_full + 8 * slot);
+  };
+  int issued = 0;
+  if (threadIdx.x == 0) {
+    for (; issued < min(kDecStages, n_stages); ++issued) issue(issued);
+  }
+
+  // This lane's slice of the query rows (pre-multiplied by scale*log2(e)) as f32x2 pairs:
+  // elements [8*li, 8*li+8) (+64 for the second half when DPL = 16).
+  uint64_t q2[GT][C::DPL / 2];
 #pragma unroll
   for (int g = 0; g < GT; ++g) {
+    const bool hv = g0 + g < p.G;
     const int h = kvh * p.G + g0 + g;
-    if (g0 + g < p.G) {
-      const uint4 w = *reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.Hq + h) * D + dofs);
-      unpack8<BF16>(w, qf[g]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) qf[g][e] *= p.scale_log2;
-    } else {
+    for (int nv = 0; nv < C::NV; ++nv) {
+      uint4 w = make_uint4(0, 0, 0, 0);
+      if (hv) w = *reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.Hq + h) * D +
+                                                  nv * (D / 2) + li * 8);
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) qf[g][e] = 0.f;
+      for (int e = 0; e < 4; ++e) {
+        float a, c;
+        f2_unpack(half2_to_f2<BF16>(u[e]), a, c);
+        q2[g][nv * 4 + e] = f2_pack(a * p.scale_log2, c * p.scale_log2);
+      }
     }
   }
 
-  float m[GT], l[GT], acc[GT][8];
+  float m[GT], l[GT];
+  uint64_t acc[GT][C::DPL / 2];
 #pragma unroll
   for (int g = 0; g < GT; ++g) {
     m[g] = -CUDART_INF_F;
     l[g] = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+    for (int e = 0; e < C::DPL / 2; ++e) acc[g][e] = f2_pack(0.f, 0.f);
   }
 
-  for (int base = t0; base < t1; base += TOK_PER_BATCH) {
-    uint4 kw[kDecUnroll], vw[kDecUnroll];
-    bool valid[kDecUnroll];
+  bool ok = true;
+  for (int st = 0; st < n_stages; ++st) {
+    const int slot = st % kDecStages;
+    if (lane == 0) ok = mbar_wait(bar_full + 8 * slot, (st / kDecStages) & 1, wc);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    if (!ok) break;
+    const int base_tok = t0 + st * kDecStageTok + warp * C::TPW;   // first token of this warp
+    const uint32_t kst = sK + slot * C::STAGE_BYTES + (warp * C::TPW) * C::ROW;
+    const uint32_t vst = sV + slot * C::STAGE_BYTES + (warp * C::TPW) * C::ROW;
+
+    float s[C::GROUPS][GT];
+    bool valid[C::GROUPS];
 #pragma unroll
-    for (int u = 0; u < kDecUnroll; ++u) {
-      const int tok = base + (u * kDecWarps + warp) * TPI + sub;
-      valid[u] = tok < t1;
-      if (valid[u]) {
-        kw[u] = ld_stream_u4(kp + static_cast<size_t>(tok) * D);
-        vw[u] = ld_stream_u4(vp + static_cast<size_t>(tok) * D);
-      } else {
-        kw[u] = make_uint4(0, 0, 0, 0);
-        vw[u] = make_uint4(0, 0, 0, 0);
+    for (int u = 0; u < C::GROUPS; ++u) {
+      const int tl = u * C::TPI + sub;                 // token within the warp's slice
+      valid[u] = base_tok + tl < t1;
+      uint32_t kw[C::DPL / 2];
+#pragma unroll
+      for (int nv = 0; nv < C::NV; ++nv) {
+        const uint4 w = lds128(kst + tl * C::ROW + nv * (C::ROW / 2) + li * 16);
+        kw[nv * 4 + 0] = w.x; kw[nv * 4 + 1] = w.y; kw[nv * 4 + 2] = w.z; kw[nv * 4 + 3] = w.w;
       }
-    }
-    float s[kDecUnroll][GT];
-#pragma unroll
-    for (int u = 0; u < kDecUnroll; ++u) {
-      float kf[8];
-      unpack8<BF16>(kw[u], kf);
 #pragma unroll
       for (int g = 0; g < GT; ++g) {
-        float a = 0.f;
+        uint64_t a2 = f2_pack(0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) a = fmaf(qf[g][e], kf[e], a);
-        s[u][g] = a;
+        for (int e = 0; e < C::DPL / 2; ++e) a2 = f2_fma(q2[g][e], half2_to_f2<BF16>(kw[e]), a2);
+        float x, y;
+        f2_unpack(a2, x, y);
+        s[u][g] = x + y;
       }
     }
-    // Sum the partial dot products over the LPT lanes that share a token.
+    // Sum the partial dot products over the LPT lanes of each token.
 #pragma unroll
-    for (int o = 1; o < LPT; o <<= 1) {
+    for (int o = 1; o < C::LPT; o <<= 1) {
 #pragma unroll
-      for (int u = 0; u < kDecUnroll; ++u)
+      for (int u = 0; u < C::GROUPS; ++u)
 #pragma unroll
         for (int g = 0; g < GT; ++g) s[u][g] += __shfl_xor_sync(0xffffffffu, s[u][g], o);
     }
+    // Online softmax over the warp's tokens of this stage (lazy rescale, threshold 2^8).
 #pragma unroll
     for (int g = 0; g < GT; ++g) {
       float mb = -CUDART_INF_F;
 #pragma unroll
-      for (int u = 0; u < kDecUnroll; ++u) {
+      for (int u = 0; u < C::GROUPS; ++u) {
         if (!valid[u]) s[u][g] = -CUDART_INF_F;
         mb = fmaxf(mb, s[u][g]);
       }
 #pragma unroll
-      for (int o = LPT; o < 32; o <<= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-      if (mb > m[g] + 8.0f) {                          // warp-uniform lazy rescale
+      for (int o = C::LPT; o < 32; o <<= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+      if (mb > m[g] + 8.0f) {                          // warp-uniform
         const float alpha = (m[g] == -CUDART_INF_F) ? 0.f : ex2_approx(m[g] - mb);
         l[g] *= alpha;
+        const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] *= alpha;
+        for (int e = 0; e < C::DPL / 2; ++e) acc[g][e] = f2_fma(acc[g][e], a2, f2_pack(0.f, 0.f));
         m[g] = mb;
       }
     }
 #pragma unroll
-    for (int u = 0; u < kDecUnroll; ++u) {
-      float vf[8];
-      unpack8<BF16>(vw[u], vf);
+    for (int u = 0; u < C::GROUPS; ++u) {
+      const int tl = u * C::TPI + sub;
+      uint32_t vw[C::DPL / 2];
+#pragma unroll
+      for (int nv = 0; nv < C::NV; ++nv) {
+        uint4 w = lds128(vst + tl * C::ROW + nv * (C::ROW / 2) + li * 16);
+        if (!valid[u]) w = make_uint4(0, 0, 0, 0);     // slot bytes past the split: never used
+        vw[nv * 4 + 0] = w.x; vw[nv * 4 + 1] = w.y; vw[nv * 4 + 2] = w.z; vw[nv * 4 + 3] = w.w;
+      }
 #pragma unroll
       for (int g = 0; g < GT; ++g) {
         // A warp whose tokens were all past the end still has m = -inf: use 0 there.
         const float mref = (m[g] == -CUDART_INF_F) ? 0.f : m[g];
         const float pr = ex2_approx(s[u][g] - mref);   // 0 for invalid tokens (s = -inf)
         l[g] += pr;
+        const uint64_t p2 = f2_pack(pr, pr);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pr, vf[e], acc[g][e]);
+        for (int e = 0; e < C::DPL / 2; ++e) acc[g][e] = f2_fma(p2, half2_to_f2<BF16>(vw[e]), acc[g][e]);
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_empty + 8 * slot);
+    // Refill the slot the whole CTA has finished with.
+    if (threadIdx.x == 0 && issued < n_stages) {
+      const int rs = issued % kDecStages;              // == slot of stage issued - kDecStages
+      if (mbar_wait(bar_empty + 8 * rs, ((issued / kDecStages) - 1) & 1, wc)) {
+        issue(issued);
+        ++issued;
+      }
+    }
+  }
+  if (threadIdx.x == 0 && *abort_flag) {
+    // Copies still in flight must land before the CTA exits.
+    for (int k = max(0, issued - kDecStages); k < issued; ++k)
+      mbar_wait_drain(bar_full + 8 * (k % kDecStages), (k / kDecStages) & 1, 200000000ull);
   }
 
   // Merge the token sub-groups of the warp (they share m).
 #pragma unroll
-  for (int o = LPT; o < 32; o <<= 1) {
+  for (int o = C::LPT; o < 32; o <<= 1) {
 #pragma unroll
     for (int g = 0; g < GT; ++g) {
       l[g] += __shfl_xor_sync(0xffffffffu, l[g], o);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], o);
+      for (int e = 0; e < C::DPL / 2; ++e) {
+        float x, y;
+        f2_unpack(acc[g][e], x, y);
+        x += __shfl_xor_sync(0xffffffffu, x, o);
+        y += __shfl_xor_sync(0xffffffffu, y, o);
+        acc[g][e] = f2_pack(x, y);
+      }
     }
   }
 
-  __shared__ float sm_m[kDecWarps][GT];
-  __shared__ float sm_l[kDecWarps][GT];
-  __shared__ __align__(16) float sm_acc[kDecWarps][GT][D];
-  if (lane < LPT) {
+  // Cross-warp merge through shared memory (the K ring is free now).
+  __syncthreads();
+  float* sm_acc = reinterpret_cast<float*>(dsmem);                      // [warps][GT][D]
+  float* sm_m = sm_acc + kDecWarps * GT * D;                            // [warps][GT]
+  float* sm_l = sm_m + kDecWarps * GT;
+  if (lane < C::LPT) {
 #pragma unroll
-    for (int g = 0; g < GT; ++g) {
+    for (int g = 0; g < GT; ++g)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) sm_acc[warp][g][dofs + e] = acc[g][e];
-    }
+      for (int nv = 0; nv < C::NV; ++nv)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float x, y;
+          f2_unpack(acc[g][nv * 4 + e], x, y);
+          const int d0 = nv * (D / 2) + li * 8 + 2 * e;
+          sm_acc[(warp * GT + g) * D + d0] = x;
+          sm_acc[(warp * GT + g) * D + d0 + 1] = y;
+        }
   }
   if (lane == 0) {
 #pragma unroll
     for (int g = 0; g < GT; ++g) {
-      sm_m[warp][g] = m[g];
-      sm_l[warp][g] = l[g];
+      sm_m[warp * GT + g] = m[g];
+      sm_l[warp * GT + g] = l[g];
     }
   }
   __syncthreads();
+  if (!ok || *abort_flag) return;
 
   for (int idx = threadIdx.x; idx < GT * D; idx += kDecThreads) {
     const int g = idx / D;
@@ -227,13 +340,14 @@ fa_decode_split_kernel(const DecodeParams p) {
     if (g0 + g >= p.G) continue;
     float M = -CUDART_INF_F;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm_m[w][g]);
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm_m[w * GT + g]);
     float L = 0.f, O = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecWarps; ++w) {
-      const float wt = (sm_m[w][g] == -CUDART_INF_F) ? 0.f : ex2_approx(sm_m[w][g] - M);
-      L = fmaf(wt, sm_l[w][g], L);
-      O = fmaf(wt, sm_acc[w][g][e], O);
+      const float mw = sm_m[w * GT + g];
+      const float wt = (mw == -CUDART_INF_F) ? 0.f : ex2_approx(mw - M);
+      L = fmaf(wt, sm_l[w * GT + g], L);
+      O = fmaf(wt, sm_acc[(w * GT + g) * D + e], O);
     }
     const int h = kvh * p.G + g0 + g;
     const size_t row = (static_cast<size_t>(b) * p.Hq + h) * p.n_split + split;
@@ -254,6 +368,9 @@ struct CombineParams {
 template <int D, bool BF16>
 __global__ void __launch_bounds__(D)
 fa_decode_combine_kernel(const CombineParams p) {
+  // Launched as a programmatic dependent of the split kernel: wait until it has finished
+  // and its writes are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x;
   const int b = bh / p.Hq;
   const int e = threadIdx.x;

@@ -156,23 +156,48 @@ bool decode_layout(int B, int Hq, int max_len, int d, DecodeLayout* L) {
 }
 
 template <int D, int GT, bool BF16>
-fa_status launch_decode_t(const fa::DecodeParams& dp, const fa::CombineParams& cp, int B,
-                          int Hkv, int G, cudaStream_t st) {
+fa_status launch_decode_t(int dev, const fa::DecodeParams& dp, const fa::CombineParams& cp,
+                          int B, int Hkv, int G, cudaStream_t st) {
+  using C = fa::DecCfg<D, GT>;
+  auto split_kernel = fa::fa_decode_split_kernel<D, GT, BF16>;
+  static bool attr_set[kMaxDevices];
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_BYTES) != cudaSuccess)
+        return FA_ERR_CUDA;
+      attr_set[dev] = true;
+    }
+  }
   const int n_gt = (G + GT - 1) / GT;
   dim3 grid(dp.n_split, Hkv * n_gt, B);
-  fa::fa_decode_split_kernel<D, GT, BF16><<<grid, fa::kDecThreads, 0, st>>>(dp);
+  split_kernel<<<grid, fa::kDecThreads, C::SMEM_BYTES, st>>>(dp);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  fa::fa_decode_combine_kernel<D, BF16><<<B * dp.Hq, D, 0, st>>>(cp);
+  // The combine is a programmatic dependent launch: it is scheduled while the split
+  // kernel's last CTAs run and waits (griddepcontrol.wait) for its results.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(B * dp.Hq, 1, 1);
+  cfg.blockDim = dim3(D, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fa::fa_decode_combine_kernel<D, BF16>, cp) != cudaSuccess)
+    return FA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 template <int D, bool BF16>
-fa_status launch_decode_g(const fa::DecodeParams& dp, const fa::CombineParams& cp, int B,
-                          int Hkv, int G, cudaStream_t st) {
-  if (G <= 1) return launch_decode_t<D, 1, BF16>(dp, cp, B, Hkv, G, st);
-  if (G <= 2) return launch_decode_t<D, 2, BF16>(dp, cp, B, Hkv, G, st);
-  if (G <= 4) return launch_decode_t<D, 4, BF16>(dp, cp, B, Hkv, G, st);
-  return launch_decode_t<D, 8, BF16>(dp, cp, B, Hkv, G, st);
+fa_status launch_decode_g(int dev, const fa::DecodeParams& dp, const fa::CombineParams& cp,
+                          int B, int Hkv, int G, cudaStream_t st) {
+  if (G <= 1) return launch_decode_t<D, 1, BF16>(dev, dp, cp, B, Hkv, G, st);
+  if (G <= 2) return launch_decode_t<D, 2, BF16>(dev, dp, cp, B, Hkv, G, st);
+  if (G <= 4) return launch_decode_t<D, 4, BF16>(dev, dp, cp, B, Hkv, G, st);
+  return launch_decode_t<D, 8, BF16>(dev, dp, cp, B, Hkv, G, st);
 }
 
 fa_status common_checks(int B, int Hq, int Hkv, int d, float scale, int dtype) {
@@ -278,6 +303,7 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
   dp.split_tokens = L.split_tokens;
   dp.n_split = L.n_split;
   dp.scale_log2 = scale * 1.4426950408889634f;
+  dp.timeout_ns = g_timeout_ns;
   fa::CombineParams cp;
   cp.ws_o = dp.ws_o;
   cp.ws_lse = dp.ws_lse;
@@ -291,10 +317,10 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == FA_BF16;
   if (d == 64)
-    return bf16 ? launch_decode_g<64, true>(dp, cp, B, Hkv, G, st)
-                : launch_decode_g<64, false>(dp, cp, B, Hkv, G, st);
-  return bf16 ? launch_decode_g<128, true>(dp, cp, B, Hkv, G, st)
-              : launch_decode_g<128, false>(dp, cp, B, Hkv, G, st);
+    return bf16 ? launch_decode_g<64, true>(dev, dp, cp, B, Hkv, G, st)
+                : launch_decode_g<64, false>(dev, dp, cp, B, Hkv, G, st);
+  return bf16 ? launch_decode_g<128, true>(dev, dp, cp, B, Hkv, G, st)
+              : launch_decode_g<128, false>(dev, dp, cp, B, Hkv, G, st);
 }
 
 }  // extern "C"

@@ -110,8 +110,6 @@ struct FwdParams {
   int skip_q_load;      // test hook
 };
 
-__device__ int g_fa_status;   // first device-side error (0 = none)
-
 template <int D>
 __device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
 #pragma unroll

@@ -153,6 +153,10 @@ struct WaitCtl {
 
 constexpr int kStatusTimeout = 5;   // == FA_ERR_DEVICE_TIMEOUT
 
+// First device-side error recorded by any kernel of the library (0 = none). The library
+// is a single translation unit, so this is the one definition.
+__device__ int g_fa_status;
+
 __device__ __forceinline__ void raise_abort(const WaitCtl& c) {
   *c.abort = 1;
   atomicCAS(c.status, 0, kStatusTimeout);
