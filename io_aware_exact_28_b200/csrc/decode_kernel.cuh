@@ -69,19 +69,42 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       :: "r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar) : "memory");
 }
 
-// Two 16-bit values in one 32-bit word -> an f32x2 pair (low element first).
+// A pair of fp32 values: one packed f32x2 register pair (FA_DEC_F32X2 = 1, default) or
+// two scalar floats.
+#ifndef FA_DEC_F32X2
+#define FA_DEC_F32X2 1
+#endif
+#if FA_DEC_F32X2
+using pair_t = uint64_t;
+__device__ __forceinline__ pair_t pmake(float a, float b) { return f2_pack(a, b); }
+__device__ __forceinline__ void psplit(pair_t v, float& a, float& b) { f2_unpack(v, a, b); }
+__device__ __forceinline__ pair_t pfma(pair_t a, pair_t b, pair_t c) { return f2_fma(a, b, c); }
+#else
+using pair_t = float2;
+__device__ __forceinline__ pair_t pmake(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ void psplit(pair_t v, float& a, float& b) { a = v.x; b = v.y; }
+__device__ __forceinline__ pair_t pfma(pair_t a, pair_t b, pair_t c) {
+  return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+}
+#endif
+
+// Two 16-bit values in one 32-bit word -> a pair (low element first).
 template <bool BF16>
-__device__ __forceinline__ uint64_t half2_to_f2(uint32_t w) {
-  if (BF16) return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+__device__ __forceinline__ pair_t half2_to_pair(uint32_t w) {
+  if (BF16) return pmake(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
   const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&w));
-  return f2_pack(x.x, x.y);
+  return pmake(x.x, x.y);
 }
 
 template <int D, int GT>
 struct DecCfg {
   // Lanes per token row: 8 while GT*D/8 registers of q and of the accumulator stay <= 64
   // per lane, otherwise 16.
+#ifdef FA_DEC_LPT
+  static constexpr int LPT = FA_DEC_LPT;
+#else
   static constexpr int LPT = (GT * (D / 8) <= 64) ? 8 : 16;
+#endif
   static constexpr int DPL = D / LPT;                 // elements per lane (8 or 16)
   static constexpr int NV = DPL / 8;                  // 16-byte loads per lane per row
   static constexpr int TPI = 32 / LPT;                // tokens per warp instruction
@@ -160,7 +183,7 @@ fa_decode_split_kernel(const DecodeParams p) {
 
   // This lane's slice of the query rows (pre-multiplied by scale*log2(e)) as f32x2 pairs:
   // elements [8*li, 8*li+8) (+64 for the second half when DPL = 16).
-  uint64_t q2[GT][C::DPL / 2];
+  pair_t q2[GT][C::DPL / 2];
 #pragma unroll
   for (int g = 0; g < GT; ++g) {
     const bool hv = g0 + g < p.G;
@@ -174,20 +197,20 @@ fa_decode_split_kernel(const DecodeParams p) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         float a, c;
-        f2_unpack(half2_to_f2<BF16>(u[e]), a, c);
-        q2[g][nv * 4 + e] = f2_pack(a * p.scale_log2, c * p.scale_log2);
+        psplit(half2_to_pair<BF16>(u[e]), a, c);
+        q2[g][nv * 4 + e] = pmake(a * p.scale_log2, c * p.scale_log2);
       }
     }
   }
 
   float m[GT], l[GT];
-  uint64_t acc[GT][C::DPL / 2];
+  pair_t acc[GT][C::DPL / 2];
 #pragma unroll
   for (int g = 0; g < GT; ++g) {
     m[g] = -CUDART_INF_F;
     l[g] = 0.f;
 #pragma unroll
-    for (int e = 0; e < C::DPL / 2; ++e) acc[g][e] = f2_pack(0.f, 0.f);
+    for (int e = 0; e < C::DPL / 2; ++e) acc[g][e] = pmake(0.f, 0.f);
   }
 
   bool ok = true;
@@ -214,11 +237,11 @@ fa_decode_split_kernel(const DecodeParams p) {
       }
 #pragma unroll
       for (int g = 0; g < GT; ++g) {
-        uint64_t a2 = f2_pack(0.f, 0.f);
+        pair_t a2 = pmake(0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < C::DPL / 2; ++e) a2 = f2_fma(q2[g][e], half2_to_f2<BF16>(kw[e]), a2);
+        for (int e = 0; e < C::DPL / 2; ++e) a2 = pfma(q2[g][e], half2_to_pair<BF16>(kw[e]), a2);
         float x, y;
-        f2_unpack(a2, x, y);
+        psplit(a2, x, y);
         s[u][g] = x + y;
       }
     }
@@ -244,9 +267,9 @@ fa_decode_split_kernel(const DecodeParams p) {
       if (mb > m[g] + 8.0f) {                          // warp-uniform
         const float alpha = (m[g] == -CUDART_INF_F) ? 0.f : ex2_approx(m[g] - mb);
         l[g] *= alpha;
-        const uint64_t a2 = f2_pack(alpha, alpha);
+        const pair_t a2 = pmake(alpha, alpha);
 #pragma unroll
-        for (int e = 0; e < C::DPL / 2; ++e) acc[g][e] = f2_fma(acc[g][e], a2, f2_pack(0.f, 0.f));
+        for (int e = 0; e < C::DPL / 2; ++e) acc[g][e] = pfma(acc[g][e], a2, pmake(0.f, 0.f));
         m[g] = mb;
       }
     }
@@ -266,9 +289,9 @@ fa_decode_split_kernel(const DecodeParams p) {
         const float mref = (m[g] == -CUDART_INF_F) ? 0.f : m[g];
         const float pr = ex2_approx(s[u][g] - mref);   // 0 for invalid tokens (s = -inf)
         l[g] += pr;
-        const uint64_t p2 = f2_pack(pr, pr);
+        const pair_t p2 = pmake(pr, pr);
 #pragma unroll
-        for (int e = 0; e < C::DPL / 2; ++e) acc[g][e] = f2_fma(p2, half2_to_f2<BF16>(vw[e]), acc[g][e]);
+        for (int e = 0; e < C::DPL / 2; ++e) acc[g][e] = pfma(p2, half2_to_pair<BF16>(vw[e]), acc[g][e]);
       }
     }
     __syncwarp();
@@ -297,10 +320,10 @@ fa_decode_split_kernel(const DecodeParams p) {
 #pragma unroll
       for (int e = 0; e < C::DPL / 2; ++e) {
         float x, y;
-        f2_unpack(acc[g][e], x, y);
+        psplit(acc[g][e], x, y);
         x += __shfl_xor_sync(0xffffffffu, x, o);
         y += __shfl_xor_sync(0xffffffffu, y, o);
-        acc[g][e] = f2_pack(x, y);
+        acc[g][e] = pmake(x, y);
       }
     }
   }
@@ -318,7 +341,7 @@ fa_decode_split_kernel(const DecodeParams p) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float x, y;
-          f2_unpack(acc[g][nv * 4 + e], x, y);
+          psplit(acc[g][nv * 4 + e], x, y);
           const int d0 = nv * (D / 2) + li * 8 + 2 * e;
           sm_acc[(warp * GT + g) * D + d0] = x;
           sm_acc[(warp * GT + g) * D + d0 + 1] = y;

@@ -5,11 +5,13 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
 #include "fa.h"
 #include "decode_kernel.cuh"
+#include "decode_tc_kernel.cuh"
 #include "fwd_kernel.cuh"
 
 namespace {
@@ -130,7 +132,19 @@ fa_status dispatch_causal(int causal, int dev, const CUtensorMap& mq, const CUte
 // Decode sizing: the split length depends only on (B, Hq, max_kv_len) so that the
 // workspace query and the launch always agree.
 // ---------------------------------------------------------------------------------------
+// FA_DECODE_SPLIT_TOKENS (a power of two in [32, 4096]) overrides the choice; it is read
+// once per process, so the workspace query and the launch still agree.
+int split_tokens_override() {
+  static int v = [] {
+    const char* e = std::getenv("FA_DECODE_SPLIT_TOKENS");
+    const int x = e ? std::atoi(e) : 0;
+    return (x >= 32 && x <= 4096 && (x & (x - 1)) == 0) ? x : 0;
+  }();
+  return v;
+}
+
 int decode_split_tokens(int B, int Hq, int max_len) {
+  if (split_tokens_override()) return split_tokens_override();
   const long long units = static_cast<long long>(B) * (Hq >= 4 ? Hq / 4 : 1);
   int s = 256;
   while (s > 64 && units * ((max_len + s - 1) / s) < 148LL * 8) s >>= 1;
@@ -144,15 +158,51 @@ struct DecodeLayout {
   size_t o_bytes, lse_off, total;
 };
 
+// d = 128 decodes on the tensor cores in 128-token tiles (decode_tc_kernel.cuh) unless
+// FA_DECODE_CUDA_CORES=1 selects the CUDA-core kernel (decode_kernel.cuh).
+bool use_tc_decode(int d) {
+  static const bool cuda_cores = [] {
+    const char* e = std::getenv("FA_DECODE_CUDA_CORES");
+    return e && std::atoi(e) == 1;
+  }();
+  return d == fa::kTcD && !cuda_cores;
+}
+
 bool decode_layout(int B, int Hq, int max_len, int d, DecodeLayout* L) {
   if (B <= 0 || Hq <= 0 || max_len <= 0 || d <= 0) return false;
-  L->split_tokens = decode_split_tokens(B, Hq, max_len);
+  if (use_tc_decode(d)) {
+    // Splits of whole 128-token tiles; 1024 tokens (8 tiles) unless overridden (measured
+    // best on the 4096-token-cache workload: fewer unit boundaries per CTA).
+    const int o = split_tokens_override();
+    L->split_tokens = o ? ((o + fa::kTcTile - 1) / fa::kTcTile) * fa::kTcTile : 8 * fa::kTcTile;
+  } else {
+    L->split_tokens = decode_split_tokens(B, Hq, max_len);
+  }
   L->n_split = (max_len + L->split_tokens - 1) / L->split_tokens;
   const size_t rows = static_cast<size_t>(B) * Hq * L->n_split;
   L->o_bytes = align_up(rows * d * sizeof(float), 256);
   L->lse_off = L->o_bytes;
   L->total = L->o_bytes + align_up(rows * sizeof(float), 256);
   return true;
+}
+
+// The combine is a programmatic dependent launch: it is scheduled while the split
+// kernel's last CTAs run and waits (griddepcontrol.wait) for its results.
+template <int D, bool BF16>
+fa_status launch_combine_pdl(const fa::CombineParams& cp, int B, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(B * cp.Hq, 1, 1);
+  cfg.blockDim = dim3(D, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fa::fa_decode_combine_kernel<D, BF16>, cp) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 template <int D, int GT, bool BF16>
@@ -174,21 +224,7 @@ fa_status launch_decode_t(int dev, const fa::DecodeParams& dp, const fa::Combine
   dim3 grid(dp.n_split, Hkv * n_gt, B);
   split_kernel<<<grid, fa::kDecThreads, C::SMEM_BYTES, st>>>(dp);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  // The combine is a programmatic dependent launch: it is scheduled while the split
-  // kernel's last CTAs run and waits (griddepcontrol.wait) for its results.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(B * dp.Hq, 1, 1);
-  cfg.blockDim = dim3(D, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, fa::fa_decode_combine_kernel<D, BF16>, cp) != cudaSuccess)
-    return FA_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return launch_combine_pdl<D, BF16>(cp, B, st);
 }
 
 template <int D, bool BF16>
@@ -198,6 +234,74 @@ fa_status launch_decode_g(int dev, const fa::DecodeParams& dp, const fa::Combine
   if (G <= 2) return launch_decode_t<D, 2, BF16>(dev, dp, cp, B, Hkv, G, st);
   if (G <= 4) return launch_decode_t<D, 4, BF16>(dev, dp, cp, B, Hkv, G, st);
   return launch_decode_t<D, 8, BF16>(dev, dp, cp, B, Hkv, G, st);
+}
+
+template <bool BF16, int GT>
+fa_status launch_decode_tc_t(int dev, const void* q, const void* kc, const void* vc,
+                           const int* kv_lens, uint8_t* ws, const DecodeLayout& L, int B, int Hq,
+                           int Hkv, int max_len, float scale, const fa::CombineParams& cp,
+                           cudaStream_t st) {
+  auto kernel = fa::fa_decode_tc_kernel<BF16, GT>;
+  static int sm_count[kMaxDevices];
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (sm_count[dev] == 0) {
+      int n = 0;
+      if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+          cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::kTcSmemBytes) != cudaSuccess)
+        return FA_ERR_CUDA;
+      sm_count[dev] = n;
+    }
+  }
+  CUtensorMap mk, mv, mq;
+  const long long BHkv = static_cast<long long>(B) * Hkv;
+  // q as [1, B*Hq, 128]: 16-row boxes, one per work unit (rows past B*Hq read as zero).
+  if (!make_tile_map(&mk, kc, fa::kTcD, max_len, BHkv, BF16, fa::kTcTile) ||
+      !make_tile_map(&mv, vc, fa::kTcD, max_len, BHkv, BF16, fa::kTcTile) ||
+      !make_tile_map(&mq, q, fa::kTcD, B * Hq, 1, BF16, fa::kTcN))
+    return FA_ERR_CUDA;
+  fa::DecodeTcParams tp;
+  tp.kc = static_cast<const uint16_t*>(kc);
+  tp.vc = static_cast<const uint16_t*>(vc);
+  tp.kv_lens = kv_lens;
+  tp.ws_o = reinterpret_cast<float*>(ws);
+  tp.ws_lse = reinterpret_cast<float*>(ws + L.lse_off);
+  tp.B = B;
+  tp.Hq = Hq;
+  tp.Hkv = Hkv;
+  tp.G = Hq / Hkv;
+  tp.GT = GT;
+  tp.n_gt = (tp.G + tp.GT - 1) / tp.GT;
+  tp.max_len = max_len;
+  tp.split_tokens = L.split_tokens;
+  tp.n_split = L.n_split;
+  tp.scale_log2 = scale * 1.4426950408889634f;
+  tp.timeout_ns = g_timeout_ns;
+  const long long n_units = static_cast<long long>(L.n_split) * B * Hkv * tp.n_gt;
+  if (n_units >= (1LL << 31)) return FA_ERR_INVALID_ARG;
+  const int grid = static_cast<int>(n_units < sm_count[dev] ? n_units : sm_count[dev]);
+  kernel<<<grid, fa::kTcThreads, fa::kTcSmemBytes, st>>>(mk, mv, mq, tp);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  return launch_combine_pdl<fa::kTcD, BF16>(cp, B, st);
+}
+
+// Head tile = the smallest of 1, 2, 4, 8, 16 that holds G (16 tiles larger groups).
+template <bool BF16>
+fa_status launch_decode_tc(int dev, const void* q, const void* kc, const void* vc,
+                           const int* kv_lens, uint8_t* ws, const DecodeLayout& L, int B, int Hq,
+                           int Hkv, int max_len, float scale, const fa::CombineParams& cp,
+                           cudaStream_t st) {
+  const int G = Hq / Hkv;
+#define FA_TC_CASE(GT_)                                                                    \
+  return launch_decode_tc_t<BF16, GT_>(dev, q, kc, vc, kv_lens, ws, L, B, Hq, Hkv, max_len, \
+                                       scale, cp, st)
+  if (G <= 1) FA_TC_CASE(1);
+  if (G <= 2) FA_TC_CASE(2);
+  if (G <= 4) FA_TC_CASE(4);
+  if (G <= 8) FA_TC_CASE(8);
+  FA_TC_CASE(16);
+#undef FA_TC_CASE
 }
 
 fa_status common_checks(int B, int Hq, int Hkv, int d, float scale, int dtype) {
@@ -289,6 +393,23 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
   if (s != FA_OK) return s;
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == FA_BF16;
+  fa::CombineParams cp;
+  cp.ws_o = reinterpret_cast<float*>(ws);
+  cp.ws_lse = reinterpret_cast<float*>(ws + L.lse_off);
+  cp.kv_lens = kv_lens;
+  cp.o = static_cast<uint16_t*>(o);
+  cp.lse = lse;
+  cp.Hq = Hq;
+  cp.max_len = max_kv_len;
+  cp.split_tokens = L.split_tokens;
+  cp.n_split = L.n_split;
+  if (use_tc_decode(d))
+    return bf16 ? launch_decode_tc<true>(dev, q, kcache, vcache, kv_lens, ws, L, B, Hq, Hkv,
+                                         max_kv_len, scale, cp, st)
+                : launch_decode_tc<false>(dev, q, kcache, vcache, kv_lens, ws, L, B, Hq, Hkv,
+                                          max_kv_len, scale, cp, st);
   fa::DecodeParams dp;
   dp.q = static_cast<const uint16_t*>(q);
   dp.kc = static_cast<const uint16_t*>(kcache);
@@ -304,18 +425,6 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
   dp.n_split = L.n_split;
   dp.scale_log2 = scale * 1.4426950408889634f;
   dp.timeout_ns = g_timeout_ns;
-  fa::CombineParams cp;
-  cp.ws_o = dp.ws_o;
-  cp.ws_lse = dp.ws_lse;
-  cp.kv_lens = kv_lens;
-  cp.o = static_cast<uint16_t*>(o);
-  cp.lse = lse;
-  cp.Hq = Hq;
-  cp.max_len = max_kv_len;
-  cp.split_tokens = L.split_tokens;
-  cp.n_split = L.n_split;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool bf16 = dtype == FA_BF16;
   if (d == 64)
     return bf16 ? launch_decode_g<64, true>(dev, dp, cp, B, Hkv, G, st)
                 : launch_decode_g<64, false>(dev, dp, cp, B, Hkv, G, st);
@@ -396,6 +505,15 @@ fa_status fa_device_status(int clear) {
 void fa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTimeoutNs; }
 
 void fa_debug_skip_q_load(int enable) { g_skip_q_load = enable ? 1 : 0; }
+
+#ifdef FA_TC_TRACE
+// Debug builds only: copy the tensor-core decode trace (8 events x 1024 tiles of clock64).
+FA_API int fa_debug_tc_trace(long long* host, int n) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  const size_t bytes = sizeof(long long) * static_cast<size_t>(n < 8 * 1024 ? n : 8 * 1024);
+  return cudaMemcpyFromSymbol(host, fa::g_fa_tc_trace, bytes) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 const char* fa_build_info(void) { return "libfa_b200 0.1 sm_100a (tcgen05/TMA prefill, split-KV decode)"; }
 

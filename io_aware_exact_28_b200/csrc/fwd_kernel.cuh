@@ -41,7 +41,6 @@ constexpr int kBM = 128;           // query rows per Q tile (one TMEM lane per r
 constexpr int kQTiles = 2;         // Q tiles per CTA
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
-constexpr uint64_t kDrainNs = 200000000ull;   // 0.2 s limit for abort-path drains
 
 // Polynomial-exp2 pair masks (see FwdCfg::kEmuPairs); off by default: measured slower on
 // B200 at both head dimensions, because the softmax is latency-bound, not MUFU-bound.
