@@ -144,12 +144,22 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
   constexpr int kBN = C::BN;
   const int n_kv_total = (p.Nk + kBN - 1) / kBN;
-  int n_kv = n_kv_total;
-  if (CAUSAL) {
-    const int q_last = min(q0 + kQTiles * kBM - 1, p.Nq - 1);
-    const int kmax = q_last + p.causal_offset;      // last key visible to this CTA
-    n_kv = kmax < 0 ? 0 : min(n_kv_total, kmax / kBN + 1);
+  // Key tiles each query tile visits: a tile past the last query row visits none, and
+  // under the causal mask a tile stops at the key tile holding its last row's diagonal.
+  int n_kv_t[kQTiles];
+#pragma unroll
+  for (int t = 0; t < kQTiles; ++t) {
+    const int row_first = q0 + t * kBM;
+    int n = row_first < p.Nq ? n_kv_total : 0;
+    if (CAUSAL && n > 0) {
+      const int kmax = min(row_first + kBM - 1, p.Nq - 1) + p.causal_offset;
+      n = kmax < 0 ? 0 : min(n_kv_total, kmax / kBN + 1);
+    }
+    n_kv_t[t] = n;
   }
+  int n_kv = 0;                                     // key tiles the CTA loads
+#pragma unroll
+  for (int t = 0; t < kQTiles; ++t) n_kv = max(n_kv, n_kv_t[t]);
 
   const uint32_t bar0 = base + C::BAR_OFF;
   auto bar_q = [&]() { return bar0; };
@@ -195,13 +205,20 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool q_issued = false;
-      // A CTA with no visible key tile writes zeros from the softmax warps and needs no Q.
+      // A query tile with no visible key tile writes zeros from its softmax warps straight
+      // into its Q buffer, so that buffer must not be loaded.
       if (!p.skip_q_load && n_kv > 0) {
-        mbar_arrive_expect_tx(bar_q(), kQTiles * C::Q_TILE_BYTES);
-        for (int t = 0; t < kQTiles; ++t)
+        int q_tiles = 0;
+#pragma unroll
+        for (int t = 0; t < kQTiles; ++t) q_tiles += n_kv_t[t] > 0 ? 1 : 0;
+        mbar_arrive_expect_tx(bar_q(), q_tiles * C::Q_TILE_BYTES);
+#pragma unroll
+        for (int t = 0; t < kQTiles; ++t) {
+          if (n_kv_t[t] == 0) continue;
           for (int ch = 0; ch < C::NCH; ++ch)
             tma_load_3d(base + C::Q_OFF + t * C::Q_TILE_BYTES + ch * C::Q_CHUNK, &tmQ, bar_q(),
                         ch * 64, q0 + t * kBM, bh);
+        }
         q_issued = true;
       }
       int it = 0;
@@ -257,6 +274,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       bool ok = mbar_wait(bar_q(), 0, wc);
       bool issued = false;
       tc_fence_after();
+      // Commits on bar_s(t): one per S_t(j), j < n_kv_t[t], then one after the last PV_t
+      // (O_t complete). A tile that stops early gets its last PV in the next iteration.
       for (int j = 0; j < n_kv && ok; ++j) {
         const int kit = 2 * j, kslot = kit % C::NS;
         const int vit = 2 * j - 1, vslot = (vit + C::NS) % C::NS;   // V_{j-1}
@@ -264,23 +283,27 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (j > 0 && !mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc)) { ok = false; break; }
         tc_fence_after();
         for (int t = 0; t < kQTiles; ++t) {
-          if (j > 0) {
+          if (j > 0 && j - 1 < n_kv_t[t]) {
             if (!mbar_wait(bar_p(t), (j - 1) & 1, wc)) { ok = false; break; }
             tc_fence_after();
             issue_pv(t, vslot, j - 1 > 0);
-            if (t == kQTiles - 1) mma_commit(bar_empty(vslot));
+            if (j == n_kv_t[t]) mma_commit(bar_s(t));   // final phase: O_t complete
           }
-          issue_s(t, kslot);
-          issued = true;
-          mma_commit(bar_s(t));
+          if (j < n_kv_t[t]) {
+            issue_s(t, kslot);
+            issued = true;
+            mma_commit(bar_s(t));
+          }
         }
         if (!ok) break;
+        if (j > 0) mma_commit(bar_empty(vslot));
         mma_commit(bar_empty(kslot));
       }
       if (ok) {
         const int vit = 2 * n_kv - 1, vslot = vit % C::NS;
         ok = mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc);
         for (int t = 0; t < kQTiles && ok; ++t) {
+          if (n_kv_t[t] != n_kv) continue;
           if (!mbar_wait(bar_p(t), (n_kv - 1) & 1, wc)) { ok = false; break; }
           tc_fence_after();
           issue_pv(t, vslot, n_kv - 1 > 0);
@@ -309,10 +332,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int lim_min = CAUSAL ? min(row_min + p.causal_offset, p.Nk - 1) : p.Nk - 1;
     const float c = p.scale_log2;
 
+    const int n_t = t == 0 ? n_kv_t[0] : n_kv_t[kQTiles - 1];
     float m_used = -CUDART_INF_F;
     float l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
+    for (int j = 0; j < n_t; ++j) {
       if (!mbar_wait(bar_s(t), j & 1, wc)) { ok = false; break; }
       tc_fence_after();
       const int key0 = j * kBN;
@@ -409,8 +433,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tc_fence_before();
       mbar_arrive(bar_p(t));
     }
-    if (ok && n_kv > 0) {
-      ok = mbar_wait(bar_s(t), n_kv & 1, wc);       // final PV of this tile done
+    if (ok && n_t > 0) {
+      ok = mbar_wait(bar_s(t), n_t & 1, wc);        // final PV of this tile done
       tc_fence_after();
     }
     uint8_t* otile = sbase + C::Q_OFF + t * C::Q_TILE_BYTES;   // Q_t no longer read
@@ -419,7 +443,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
       for (int ch = 0; ch < C::NCH; ++ch) {
         uint32_t o[64];
-        if (n_kv > 0) {
+        if (n_t > 0) {
           uint32_t (&o_lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
           uint32_t (&o_hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[32]);
           tmem_ld32x32b_x32(tO + ch * 64, o_lo);
@@ -446,7 +470,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       fence_proxy_async_smem();
     }
     named_barrier_sync(1 + t, kBM);
-    if (r == 0 && ok && !*abort_flag) {
+    if (r == 0 && ok && !*abort_flag && row_min < p.Nq) {
       for (int ch = 0; ch < C::NCH; ++ch)
         tma_store_3d(&tmO, smem_u32(otile + ch * C::Q_CHUNK), ch * 64, q0 + t * kBM, bh);
       tma_store_commit_and_wait_read();

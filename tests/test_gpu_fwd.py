@@ -60,6 +60,14 @@ def test_rectangular(Nq, Nk, causal):
     check_full(2, 4, 2, Nq, Nk, 128, "bf16", causal, seed=Nq * 7 + Nk)
 
 
+@pytest.mark.parametrize("Nq,Nk", [(300, 77), (640, 200), (512, 1024), (200, 1000)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_rectangular_d64(Nq, Nk, causal):
+    """The d = 64 kernel (64-key tiles) on rectangular shapes, including causal CTAs whose
+    first query tile sees no key while the second does."""
+    check_full(2, 4, 2, Nq, Nk, 64, "fp16", causal, seed=Nq * 5 + Nk)
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(8, 1), (8, 2), (6, 3), (4, 4)])
 def test_gqa_groupings(Hq, Hkv):
     check_full(2, Hq, Hkv, 384, 384, 64, "fp16", True, seed=Hq * 10 + Hkv)
