@@ -92,8 +92,7 @@ bool make_tile_map(CUtensorMap* m, const void* ptr, int d, int rows, long long h
 // ---------------------------------------------------------------------------------------
 template <int D, bool BF16, bool CAUSAL>
 fa_status launch_fwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const CUtensorMap& mo, const fa::FwdParams& prm, int BH, int Nq,
-                     cudaStream_t stream) {
+                     const fa::FwdParams& prm, cudaStream_t stream) {
   using C = fa::FwdCfg<D>;
   auto kernel = fa::fa_fwd_kernel<D, BF16, CAUSAL>;
   static int attr_state[kMaxDevices];   // 0 unknown, 1 ready, 2 unusable build
@@ -114,18 +113,18 @@ fa_status launch_fwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
     }
     if (attr_state[dev] != 1) return FA_ERR_UNSUPPORTED;
   }
-  const int n_qblocks = (Nq + fa::kQTiles * fa::kBM - 1) / (fa::kQTiles * fa::kBM);
-  dim3 grid(BH, n_qblocks, 1);
-  kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
+  // One CTA per work unit (query block of a (batch, head)); running CTAs take over the
+  // ones that have not started, so the grid size only bounds the work, not the residency.
+  const unsigned n_units = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_qb);
+  kernel<<<n_units, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 template <int D, bool BF16>
 fa_status dispatch_causal(int causal, int dev, const CUtensorMap& mq, const CUtensorMap& mk,
-                          const CUtensorMap& mv, const CUtensorMap& mo, const fa::FwdParams& prm,
-                          int BH, int Nq, cudaStream_t st) {
-  return causal ? launch_fwd<D, BF16, true>(dev, mq, mk, mv, mo, prm, BH, Nq, st)
-                : launch_fwd<D, BF16, false>(dev, mq, mk, mv, mo, prm, BH, Nq, st);
+                          const CUtensorMap& mv, const fa::FwdParams& prm, cudaStream_t st) {
+  return causal ? launch_fwd<D, BF16, true>(dev, mq, mk, mv, prm, st)
+                : launch_fwd<D, BF16, false>(dev, mq, mk, mv, prm, st);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -327,7 +326,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   const long long BH = static_cast<long long>(B) * Hq;
   const long long BHkv = static_cast<long long>(B) * Hkv;
   if (BH >= (1LL << 31)) return FA_ERR_INVALID_ARG;
-  if ((Nq + fa::kQTiles * fa::kBM - 1) / (fa::kQTiles * fa::kBM) > 65535) return FA_ERR_INVALID_ARG;
+  const long long n_qb = (Nq + fa::kQTiles * fa::kBM - 1) / (fa::kQTiles * fa::kBM);
+  if (BH * n_qb >= (1LL << 31)) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGNMENT;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_ALIGNMENT;
   int dev = 0;
@@ -335,16 +335,18 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (s != FA_OK) return s;
 
   const bool bf16 = dtype == FA_BF16;
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv;
   const int kv_box = (d == 64) ? fa::FwdCfg<64>::BN : fa::FwdCfg<128>::BN;
   if (!make_tile_map(&mq, q, d, Nq, BH, bf16, fa::kBM) ||
       !make_tile_map(&mk, k, d, Nk, BHkv, bf16, kv_box) ||
-      !make_tile_map(&mv, v, d, Nk, BHkv, bf16, kv_box) ||
-      !make_tile_map(&mo, o, d, Nq, BH, bf16, fa::kBM))
+      !make_tile_map(&mv, v, d, Nk, BHkv, bf16, kv_box))
     return FA_ERR_CUDA;
 
   fa::FwdParams prm;
+  prm.o = o;
   prm.lse = lse;
+  prm.BH = static_cast<int>(BH);
+  prm.n_qb = static_cast<int>(n_qb);
   prm.Hq = Hq;
   prm.Hkv = Hkv;
   prm.group = Hq / Hkv;
@@ -355,12 +357,11 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   prm.timeout_ns = g_timeout_ns;
   prm.skip_q_load = g_skip_q_load;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int bh = static_cast<int>(BH);
   if (d == 64)
-    return bf16 ? dispatch_causal<64, true>(causal, dev, mq, mk, mv, mo, prm, bh, Nq, st)
-                : dispatch_causal<64, false>(causal, dev, mq, mk, mv, mo, prm, bh, Nq, st);
-  return bf16 ? dispatch_causal<128, true>(causal, dev, mq, mk, mv, mo, prm, bh, Nq, st)
-              : dispatch_causal<128, false>(causal, dev, mq, mk, mv, mo, prm, bh, Nq, st);
+    return bf16 ? dispatch_causal<64, true>(causal, dev, mq, mk, mv, prm, st)
+                : dispatch_causal<64, false>(causal, dev, mq, mk, mv, prm, st);
+  return bf16 ? dispatch_causal<128, true>(causal, dev, mq, mk, mv, prm, st)
+              : dispatch_causal<128, false>(causal, dev, mq, mk, mv, prm, st);
 }
 
 size_t fa_decode_workspace_bytes(int B, int Hq, int max_kv_len, int d) {

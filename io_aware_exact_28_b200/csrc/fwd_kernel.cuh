@@ -77,8 +77,10 @@ struct FwdCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = kQTiles * Q_TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NS * KV_TILE_BYTES;
-  static constexpr int NBARS = 1 + 2 * NS + 2 * kQTiles + 1;
-  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  // q, full[NS], empty[NS], s[2], p[2], o[2], qempty, clc_full[2], clc_empty[2], drain
+  static constexpr int NBARS = 1 + 2 * NS + 3 * kQTiles + 1 + 4 + 1;
+  static constexpr int CLC_OFF = BAR_OFF + ((NBARS * 8 + 15) / 16) * 16;   // 2 x 16-byte responses
+  static constexpr int MISC_OFF = CLC_OFF + 32;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;   // + slack for 1 KB alignment
   static constexpr uint32_t TMEM_COLS = (D == 64) ? 256 : 512;
   static constexpr uint32_t S_COL = 0;                // S_t at t * BN
@@ -100,7 +102,10 @@ struct FwdCfg {
 };
 
 struct FwdParams {
+  void* o;              // [B*Hq, Nq, D], 16-bit
   float* lse;           // [B*Hq, Nq] or nullptr
+  int BH;               // B * Hq
+  int n_qb;             // query blocks of kQTiles * kBM rows per (batch, head)
   int Hq, Hkv, group;   // group = Hq / Hkv
   int Nq, Nk;
   int causal_offset;    // Nk - Nq (bottom-right alignment)
@@ -125,8 +130,7 @@ __device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
 template <int D, bool BF16, bool CAUSAL>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::CTAS)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-              const FwdParams p) {
+              const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -135,31 +139,39 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;                        // b * Hq + h
-  const int b = bh / p.Hq;
-  const int h = bh - b * p.Hq;
-  const int bh_kv = b * p.Hkv + h / p.group;
-  const int qb = gridDim.y - 1 - blockIdx.y;        // heaviest (causal) blocks launch first
-  const int q0 = qb * (kQTiles * kBM);
-
   constexpr int kBN = C::BN;
   const int n_kv_total = (p.Nk + kBN - 1) / kBN;
-  // Key tiles each query tile visits: a tile past the last query row visits none, and
-  // under the causal mask a tile stops at the key tile holding its last row's diagonal.
-  int n_kv_t[kQTiles];
+
+  // Work unit u covers query block qb of (batch, head) bh; units are numbered heaviest
+  // causal block first, which is also the order in which the hardware starts CTAs and
+  // hands out not-yet-started CTAs to running ones.
+  // n_t[t]: key tiles query tile t visits. A tile past the last query row visits none,
+  // and under the causal mask a tile stops at the key tile of its last row's diagonal.
+  struct Unit {
+    int bh, bh_kv, q0;
+    int n_t[kQTiles];
+    int n_kv;           // key tiles the unit loads: max over its query tiles
+  };
+  auto decode_unit = [&](int u) {
+    Unit w;
+    const int qb = p.n_qb - 1 - u / p.BH;
+    w.bh = u - (u / p.BH) * p.BH;
+    w.bh_kv = (w.bh / p.Hq) * p.Hkv + (w.bh % p.Hq) / p.group;
+    w.q0 = qb * (kQTiles * kBM);
+    w.n_kv = 0;
 #pragma unroll
-  for (int t = 0; t < kQTiles; ++t) {
-    const int row_first = q0 + t * kBM;
-    int n = row_first < p.Nq ? n_kv_total : 0;
-    if (CAUSAL && n > 0) {
-      const int kmax = min(row_first + kBM - 1, p.Nq - 1) + p.causal_offset;
-      n = kmax < 0 ? 0 : min(n_kv_total, kmax / kBN + 1);
+    for (int t = 0; t < kQTiles; ++t) {
+      const int row_first = w.q0 + t * kBM;
+      int n = row_first < p.Nq ? n_kv_total : 0;
+      if (CAUSAL && n > 0) {
+        const int kmax = min(row_first + kBM - 1, p.Nq - 1) + p.causal_offset;
+        n = kmax < 0 ? 0 : min(n_kv_total, kmax / kBN + 1);
+      }
+      w.n_t[t] = n;
+      w.n_kv = max(w.n_kv, n);
     }
-    n_kv_t[t] = n;
-  }
-  int n_kv = 0;                                     // key tiles the CTA loads
-#pragma unroll
-  for (int t = 0; t < kQTiles; ++t) n_kv = max(n_kv, n_kv_t[t]);
+    return w;
+  };
 
   const uint32_t bar0 = base + C::BAR_OFF;
   auto bar_q = [&]() { return bar0; };
@@ -167,9 +179,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   auto bar_empty = [&](int i) { return bar0 + 8u * (1 + C::NS + i); };
   auto bar_s = [&](int t) { return bar0 + 8u * (1 + 2 * C::NS + t); };
   auto bar_p = [&](int t) { return bar0 + 8u * (1 + 2 * C::NS + kQTiles + t); };
-  const uint32_t bar_drain = bar0 + 8u * (1 + 2 * C::NS + 2 * kQTiles);
+  auto bar_o = [&](int t) { return bar0 + 8u * (1 + 2 * C::NS + 2 * kQTiles + t); };
+  const uint32_t bar_qempty = bar0 + 8u * (1 + 2 * C::NS + 3 * kQTiles);
+  auto bar_clc_full = [&](int i) { return bar0 + 8u * (2 + 2 * C::NS + 3 * kQTiles + i); };
+  auto bar_clc_empty = [&](int i) { return bar0 + 8u * (4 + 2 * C::NS + 3 * kQTiles + i); };
+  const uint32_t bar_drain = bar0 + 8u * (6 + 2 * C::NS + 3 * kQTiles);
+  auto clc_resp = [&](int i) { return base + C::CLC_OFF + 16u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + C::MISC_OFF + 4);
+  // Readers of each scheduling response: the MMA thread and the 8 softmax warps.
+  constexpr int kClcReaders = 1 + 2 * kQTiles * 2;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q(), 1);
@@ -180,6 +199,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     for (int t = 0; t < kQTiles; ++t) {
       mbar_init(bar_s(t), 1);
       mbar_init(bar_p(t), kBM);
+      mbar_init(bar_o(t), 1);
+    }
+    mbar_init(bar_qempty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_clc_full(i), 1);
+      mbar_init(bar_clc_empty(i), kClcReaders);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -190,7 +215,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
-    prefetch_tmap(&tmO);
   }
   tc_fence_before();
   __syncthreads();
@@ -198,57 +222,77 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, &g_fa_status, p.timeout_ns};
 
-  // Each role's code sits inside the branch that set its register budget.
+  // Each role's code sits inside the branch that set its register budget. Every role
+  // walks the same unit sequence: its own blockIdx.x, then the CTAs the producer takes
+  // over, published through clc_resp[k & 1] (k = units finished).
   if (warp >= 2 * 4) {
     if constexpr (C::REGSPLIT) setmaxnreg_dec<C::REGS_OTHER>();
     if (warp == kWarpProducer) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      bool q_issued = false;
-      // A query tile with no visible key tile writes zeros from its softmax warps straight
-      // into its Q buffer, so that buffer must not be loaded.
-      if (!p.skip_q_load && n_kv > 0) {
-        int q_tiles = 0;
+      int unit = blockIdx.x, k = 0, it = 0, q_loads = 0;
+      bool ok = true, clc_pending = false;
+      while (true) {
+        const Unit w = decode_unit(unit);
+        // A query tile with no visible key writes zeros and needs no Q.
+        if (!p.skip_q_load && w.n_kv > 0) {
+          // Q is reloaded once the previous unit's S products have all read it.
+          if (q_loads > 0 && !mbar_wait(bar_qempty, (q_loads - 1) & 1, wc)) { ok = false; break; }
+          int q_tiles = 0;
 #pragma unroll
-        for (int t = 0; t < kQTiles; ++t) q_tiles += n_kv_t[t] > 0 ? 1 : 0;
-        mbar_arrive_expect_tx(bar_q(), q_tiles * C::Q_TILE_BYTES);
+          for (int t = 0; t < kQTiles; ++t) q_tiles += w.n_t[t] > 0 ? 1 : 0;
+          mbar_arrive_expect_tx(bar_q(), q_tiles * C::Q_TILE_BYTES);
 #pragma unroll
-        for (int t = 0; t < kQTiles; ++t) {
-          if (n_kv_t[t] == 0) continue;
-          for (int ch = 0; ch < C::NCH; ++ch)
-            tma_load_3d(base + C::Q_OFF + t * C::Q_TILE_BYTES + ch * C::Q_CHUNK, &tmQ, bar_q(),
-                        ch * 64, q0 + t * kBM, bh);
-        }
-        q_issued = true;
-      }
-      int it = 0;
-      bool ok = true;
-      for (int j = 0; j < n_kv && ok; ++j) {
-        for (int kv = 0; kv < 2; ++kv) {
-          const int slot = it % C::NS;
-          const int round = it / C::NS;
-          if (round > 0 && !mbar_wait(bar_empty(slot), (round - 1) & 1, wc)) {
-            ok = false;
-            break;
+          for (int t = 0; t < kQTiles; ++t) {
+            if (w.n_t[t] == 0) continue;
+            for (int ch = 0; ch < C::NCH; ++ch)
+              tma_load_3d(base + C::Q_OFF + t * C::Q_TILE_BYTES + ch * C::Q_CHUNK, &tmQ, bar_q(),
+                          ch * 64, w.q0 + t * kBM, w.bh);
           }
-          mbar_arrive_expect_tx(bar_full(slot), C::KV_TILE_BYTES);
-          const CUtensorMap* tm = kv ? &tmV : &tmK;
-          for (int ch = 0; ch < C::NCH; ++ch)
-            tma_load_3d(base + C::KV_OFF + slot * C::KV_TILE_BYTES + ch * C::KV_CHUNK, tm,
-                        bar_full(slot), ch * 64, j * kBN, bh_kv);
-          ++it;
+          ++q_loads;
         }
+        for (int j = 0; j < w.n_kv && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const int slot = it % C::NS;
+            const int round = it / C::NS;
+            if (round > 0 && !mbar_wait(bar_empty(slot), (round - 1) & 1, wc)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar_full(slot), C::KV_TILE_BYTES);
+            const CUtensorMap* tm = kv ? &tmV : &tmK;
+            for (int ch = 0; ch < C::NCH; ++ch)
+              tma_load_3d(base + C::KV_OFF + slot * C::KV_TILE_BYTES + ch * C::KV_CHUNK, tm,
+                          bar_full(slot), ch * 64, j * kBN, w.bh_kv);
+            ++it;
+          }
+        }
+        if (!ok) break;
+        // All loads of this unit are issued: take over the next CTA that has not started.
+        const int sl = k & 1;
+        if (k >= 2 && !mbar_wait(bar_clc_empty(sl), ((k >> 1) - 1) & 1, wc)) { ok = false; break; }
+        mbar_arrive_expect_tx(bar_clc_full(sl), 16);
+        clc_try_cancel(clc_resp(sl), bar_clc_full(sl));
+        clc_pending = true;
+        if (!mbar_wait(bar_clc_full(sl), (k >> 1) & 1, wc)) { ok = false; break; }
+        clc_pending = false;
+        uint32_t next;
+        const bool more = clc_query(clc_resp(sl), next);
+        ++k;
+        if (!more) break;
+        unit = static_cast<int>(next);
       }
       if (!ok || *abort_flag) {
-        // Loads still in flight must land before the CTA exits.
-        for (int k = max(0, it - C::NS); k < it; ++k)
-          mbar_wait_drain(bar_full(k % C::NS), (k / C::NS) & 1, kDrainNs);
-        if (q_issued) mbar_wait_drain(bar_q(), 0, kDrainNs);
+        // Copies still in flight must land before the CTA exits.
+        for (int i = max(0, it - C::NS); i < it; ++i)
+          mbar_wait_drain(bar_full(i % C::NS), (i / C::NS) & 1, kDrainNs);
+        if (q_loads > 0) mbar_wait_drain(bar_q(), (q_loads - 1) & 1, kDrainNs);
+        if (clc_pending) mbar_wait_drain(bar_clc_full(k & 1), (k >> 1) & 1, kDrainNs);
       }
     }
     } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_kv > 0) {
+    if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_f16(kBM, kBN, BF16 ? 1u : 0u, 0u, 0u);
       constexpr uint32_t IDESC_O = idesc_f16(kBM, D, BF16 ? 1u : 0u, 0u, 1u);
       auto issue_s = [&](int t, int kslot) {
@@ -271,45 +315,71 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                      (acc0 || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar_q(), 0, wc);
-      bool issued = false;
-      tc_fence_after();
-      // Commits on bar_s(t): one per S_t(j), j < n_kv_t[t], then one after the last PV_t
-      // (O_t complete). A tile that stops early gets its last PV in the next iteration.
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int kit = 2 * j, kslot = kit % C::NS;
-        const int vit = 2 * j - 1, vslot = (vit + C::NS) % C::NS;   // V_{j-1}
-        if (!mbar_wait(bar_full(kslot), (kit / C::NS) & 1, wc)) { ok = false; break; }
-        if (j > 0 && !mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        for (int t = 0; t < kQTiles; ++t) {
-          if (j > 0 && j - 1 < n_kv_t[t]) {
-            if (!mbar_wait(bar_p(t), (j - 1) & 1, wc)) { ok = false; break; }
+      int unit = blockIdx.x, k = 0, it = 0, q_uses = 0;
+      int p_seen[kQTiles];
+#pragma unroll
+      for (int t = 0; t < kQTiles; ++t) p_seen[t] = 0;
+      bool ok = true, issued = false;
+      while (ok) {
+        const Unit w = decode_unit(unit);
+        if (w.n_kv > 0) {
+          ok = mbar_wait(bar_q(), q_uses & 1, wc);
+          ++q_uses;
+          tc_fence_after();
+          // Per key tile j and query tile t: the PV of tile j-1 (its last one completes
+          // O_t: commit bar_o), then S_t(j) (commit bar_s). MMAs of one thread run in
+          // order, so S_t(j) never overwrites P_t(j-1) before that PV has read it.
+          for (int j = 0; j < w.n_kv && ok; ++j) {
+            const int kit = it + 2 * j, kslot = kit % C::NS;
+            const int vit = kit - 1, vslot = (vit + C::NS) % C::NS;   // V_{j-1}
+            if (!mbar_wait(bar_full(kslot), (kit / C::NS) & 1, wc)) { ok = false; break; }
+            if (j > 0 && !mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            issue_pv(t, vslot, j - 1 > 0);
-            if (j == n_kv_t[t]) mma_commit(bar_s(t));   // final phase: O_t complete
+#pragma unroll
+            for (int t = 0; t < kQTiles; ++t) {
+              if (j > 0 && j - 1 < w.n_t[t]) {
+                if (!mbar_wait(bar_p(t), p_seen[t] & 1, wc)) { ok = false; break; }
+                ++p_seen[t];
+                tc_fence_after();
+                issue_pv(t, vslot, j - 1 > 0);
+                if (j == w.n_t[t]) mma_commit(bar_o(t));
+              }
+              if (j < w.n_t[t]) {
+                issue_s(t, kslot);
+                issued = true;
+                mma_commit(bar_s(t));
+              }
+            }
+            if (!ok) break;
+            if (j == w.n_kv - 1) mma_commit(bar_qempty);    // every S of the unit issued
+            if (j > 0) mma_commit(bar_empty(vslot));
+            mma_commit(bar_empty(kslot));
           }
-          if (j < n_kv_t[t]) {
-            issue_s(t, kslot);
-            issued = true;
-            mma_commit(bar_s(t));
+          if (ok) {
+            const int vit = it + 2 * w.n_kv - 1, vslot = vit % C::NS;
+            ok = mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc);
+#pragma unroll
+            for (int t = 0; t < kQTiles; ++t) {
+              if (!ok || w.n_t[t] != w.n_kv) continue;
+              if (!mbar_wait(bar_p(t), p_seen[t] & 1, wc)) { ok = false; break; }
+              ++p_seen[t];
+              tc_fence_after();
+              issue_pv(t, vslot, w.n_kv - 1 > 0);
+              mma_commit(bar_o(t));
+            }
+            if (ok) mma_commit(bar_empty(vslot));
           }
+          it += 2 * w.n_kv;
         }
         if (!ok) break;
-        if (j > 0) mma_commit(bar_empty(vslot));
-        mma_commit(bar_empty(kslot));
-      }
-      if (ok) {
-        const int vit = 2 * n_kv - 1, vslot = vit % C::NS;
-        ok = mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc);
-        for (int t = 0; t < kQTiles && ok; ++t) {
-          if (n_kv_t[t] != n_kv) continue;
-          if (!mbar_wait(bar_p(t), (n_kv - 1) & 1, wc)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(t, vslot, n_kv - 1 > 0);
-          mma_commit(bar_s(t));   // final phase: O_t complete
-        }
-        if (ok) mma_commit(bar_empty(vslot));
+        const int sl = k & 1;
+        if (!mbar_wait(bar_clc_full(sl), (k >> 1) & 1, wc)) { ok = false; break; }
+        uint32_t next;
+        const bool more = clc_query(clc_resp(sl), next);
+        mbar_arrive(bar_clc_empty(sl));
+        ++k;
+        if (!more) break;
+        unit = static_cast<int>(next);
       }
       if (issued) {
         // Every MMA must have finished before TMEM is released.
@@ -326,154 +396,174 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + C::S_COL + t * kBN;
     const uint32_t tO = tmem + lane_base + C::O_COL + t * D;
-    const int row = q0 + t * kBM + r;
-    const int row_min = q0 + t * kBM;
-    const int lim = CAUSAL ? min(row + p.causal_offset, p.Nk - 1) : p.Nk - 1;
-    const int lim_min = CAUSAL ? min(row_min + p.causal_offset, p.Nk - 1) : p.Nk - 1;
     const float c = p.scale_log2;
-
-    const int n_t = t == 0 ? n_kv_t[0] : n_kv_t[kQTiles - 1];
-    float m_used = -CUDART_INF_F;
-    float l = 0.f;
+    int unit = blockIdx.x, k = 0, s_seen = 0, o_seen = 0;
     bool ok = true;
-    for (int j = 0; j < n_t; ++j) {
-      if (!mbar_wait(bar_s(t), j & 1, wc)) { ok = false; break; }
-      tc_fence_after();
-      const int key0 = j * kBN;
-      const bool masked_tile = key0 + kBN - 1 > lim_min;   // tile-uniform: diagonal or ragged
-      // Scores of a 32-column chunk cc, with masked keys set to -inf.
-      auto mask_chunk = [&](uint32_t (&v)[32], int cc) {
-        if (masked_tile) {
+    while (true) {
+      const Unit w = decode_unit(unit);
+      const int n_t = t == 0 ? w.n_t[0] : w.n_t[kQTiles - 1];
+      const int row = w.q0 + t * kBM + r;
+      const int row_min = w.q0 + t * kBM;
+      const int lim = CAUSAL ? min(row + p.causal_offset, p.Nk - 1) : p.Nk - 1;
+      const int lim_min = CAUSAL ? min(row_min + p.causal_offset, p.Nk - 1) : p.Nk - 1;
+
+      float m_used = -CUDART_INF_F;
+      float l = 0.f;
+      for (int j = 0; j < n_t; ++j) {
+        // Wait results are made warp-uniform: the TMEM loads and stores below are
+        // warp-collective, so a warp must never split on an aborted wait.
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_s(t), s_seen & 1, wc))) { ok = false; break; }
+        ++s_seen;
+        tc_fence_after();
+        const int key0 = j * kBN;
+        const bool masked_tile = key0 + kBN - 1 > lim_min;   // tile-uniform: diagonal or ragged
+        // Scores of a 32-column chunk cc, with masked keys set to -inf.
+        auto mask_chunk = [&](uint32_t (&v)[32], int cc) {
+          if (masked_tile) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (key0 + 32 * cc + k > lim) v[k] = __float_as_uint(-CUDART_INF_F);
+            for (int kk = 0; kk < 32; ++kk)
+              if (key0 + 32 * cc + kk > lim) v[kk] = __float_as_uint(-CUDART_INF_F);
+          }
+        };
+        // Row maximum over 8 independent chains (short dependency chains).
+        float mx8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = -CUDART_INF_F;
+        auto max_chunk = [&](const uint32_t (&v)[32]) {
+#pragma unroll
+          for (int kk = 0; kk < 32; kk += 2)
+            mx8[(kk >> 1) & 7] = fmax3(mx8[(kk >> 1) & 7], __uint_as_float(v[kk]), __uint_as_float(v[kk + 1]));
+        };
+        // d = 128 keeps the whole 128-score row in registers; d = 64 (two CTAs per SM, 96
+        // registers) reads its 64-score row from TMEM twice: once for the max, once for P.
+        constexpr bool kResident = (kBN == 128);
+        uint32_t sr[kResident ? kBN : 32];
+        if constexpr (kResident) {
+          tmem_ld32x32b_x128(tS, sr);
+#pragma unroll
+          for (int cc = 0; cc < kBN / 32; ++cc) {
+            uint32_t (&v)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]);
+            mask_chunk(v, cc);
+            max_chunk(v);
+          }
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < kBN / 32; ++cc) {
+            tmem_ld32x32b_x32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]), cc);
+            max_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          }
         }
-      };
-      // Row maximum over 8 independent chains (short dependency chains).
-      float mx8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = -CUDART_INF_F;
-      auto max_chunk = [&](const uint32_t (&v)[32]) {
-#pragma unroll
-        for (int k = 0; k < 32; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], __uint_as_float(v[k]));
-      };
-      // d = 128 keeps the whole 128-score row in registers; d = 64 (two CTAs per SM, 96
-      // registers) reads its 64-score row from TMEM twice: once for the max, once for P.
-      constexpr bool kResident = (kBN == 128);
-      uint32_t sr[kResident ? kBN : 32];
-      if constexpr (kResident) {
-        tmem_ld32x32b_x128(tS, sr);
-#pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          uint32_t (&v)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]);
-          mask_chunk(v, cc);
-          max_chunk(v);
-        }
-      } else {
-#pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          tmem_ld32x32b_x32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-          mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]), cc);
-          max_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        }
-      }
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * c;
-      if (mx > m_used + 8.0f) {                      // scale > 0: -inf stays -inf
-        if (m_used != -CUDART_INF_F) {               // O_t and l hold earlier tiles
-          const float alpha = ex2_approx(m_used - mx);
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7])) * c;
+        // Raise m only when the tile max exceeds it by more than 8 (scale > 0: -inf stays
+        // -inf). Rows that already hold earlier tiles rescale O_t and l. The TMEM rescale
+        // is warp-collective: the warp runs it if any row needs it, with factor 1 elsewhere.
+        const bool grow = mx > m_used + 8.0f;
+        const bool rescale = grow && m_used != -CUDART_INF_F;
+        if (__any_sync(0xffffffffu, rescale)) {
+          const float alpha = rescale ? ex2_approx(m_used - mx) : 1.0f;
           l *= alpha;
           rescale_o_row<D>(tO, alpha);
         }
-        m_used = mx;
-      }
-      const float mref = (m_used == -CUDART_INF_F) ? 0.f : m_used;
-      // P = 2^(s*c - m) in 32-column chunks, each stored to TMEM as 16 packed columns
-      // (P_t occupies S_t columns [0, BN/2); chunk cc only overwrites columns already read).
-      // In tiles without masked scores, the pairs selected by kEmuPairs are evaluated
-      // with the FMA-pipe polynomial instead of MUFU.EX2. The argument s*c - m and the
-      // row sum use packed f32x2 arithmetic.
-      const uint64_t c2 = f2_pack(c, c);
-      const uint64_t nm2 = f2_pack(-mref, -mref);
-      uint64_t l2a = f2_pack(0.f, 0.f), l2b = l2a;
+        if (grow) m_used = mx;
+        const float mref = (m_used == -CUDART_INF_F) ? 0.f : m_used;
+        // P = 2^(s*c - m) in 32-column chunks, each stored to TMEM as 16 packed columns
+        // (P_t occupies S_t columns [0, BN/2); chunk cc only overwrites columns already read).
+        // In tiles without masked scores, the pairs selected by kEmuPairs are evaluated
+        // with the FMA-pipe polynomial instead of MUFU.EX2. The argument s*c - m and the
+        // row sum use packed f32x2 arithmetic.
+        const uint64_t c2 = f2_pack(c, c);
+        const uint64_t nm2 = f2_pack(-mref, -mref);
+        uint64_t l2a = f2_pack(0.f, 0.f), l2b = l2a;
 #pragma unroll
-      for (int cc = 0; cc < kBN / 32; ++cc) {
-        if constexpr (!kResident) {
-          tmem_ld32x32b_x32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-          mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]), cc);
-        }
-        const uint32_t* v = kResident ? &sr[32 * cc] : &sr[0];
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint64_t x2 =
-              f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2);
-          uint64_t p2;
-          if (!masked_tile && ((FwdCfg<D>::kEmuPairs >> (i & 7)) & 1u)) {
-            p2 = exp2_poly_f2(x2);
-          } else {
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+        for (int cc = 0; cc < kBN / 32; ++cc) {
+          if constexpr (!kResident) {
+            tmem_ld32x32b_x32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]), cc);
           }
-          if (i & 1) l2b = f2_add(l2b, p2); else l2a = f2_add(l2a, p2);
-          float p0, p1;
-          f2_unpack(p2, p0, p1);
-          pk[i] = pack_half2(p0, p1, BF16);
+          const uint32_t* v = kResident ? &sr[32 * cc] : &sr[0];
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint64_t x2 =
+                f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2);
+            uint64_t p2;
+            if (!masked_tile && ((FwdCfg<D>::kEmuPairs >> (i & 7)) & 1u)) {
+              p2 = exp2_poly_f2(x2);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+            }
+            if (i & 1) l2b = f2_add(l2b, p2); else l2a = f2_add(l2a, p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            pk[i] = pack_half2(p0, p1, BF16);
+          }
+          tmem_st32x32b_x16(tS + cc * 16, pk);
         }
-        tmem_st32x32b_x16(tS + cc * 16, pk);
+        {
+          float la, lb, lc, ld;
+          f2_unpack(l2a, la, lb);
+          f2_unpack(l2b, lc, ld);
+          l += (la + lb) + (lc + ld);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_p(t));
       }
+      if (ok && n_t > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_o(t), o_seen & 1, wc));   // last PV done
+        ++o_seen;
+        tc_fence_after();
+      }
+      if (!ok) break;
+      // Epilogue: O / l straight from registers to global memory (one 2*D-byte row per
+      // thread), then LSE = (m + log2 l) ln 2. A tile that saw no key writes zeros / -inf.
+      // Every lane loads from TMEM (warp-collective); rows past Nq store nothing.
       {
-        float la, lb, lc, ld;
-        f2_unpack(l2a, la, lb);
-        f2_unpack(l2b, lc, ld);
-        l += (la + lb) + (lc + ld);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar_p(t));
-    }
-    if (ok && n_t > 0) {
-      ok = mbar_wait(bar_s(t), n_t & 1, wc);        // final PV of this tile done
-      tc_fence_after();
-    }
-    uint8_t* otile = sbase + C::Q_OFF + t * C::Q_TILE_BYTES;   // Q_t no longer read
-    if (ok) {
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const bool row_ok = row < p.Nq;
+        uint16_t* orow = static_cast<uint16_t*>(p.o) +
+                         (static_cast<size_t>(w.bh) * p.Nq + (row_ok ? row : 0)) * D;
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll
-      for (int ch = 0; ch < C::NCH; ++ch) {
-        uint32_t o[64];
-        if (n_t > 0) {
-          uint32_t (&o_lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
-          uint32_t (&o_hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[32]);
-          tmem_ld32x32b_x32(tO + ch * 64, o_lo);
-          tmem_ld32x32b_x32(tO + ch * 64 + 32, o_hi);
-        } else {
+        for (int ch = 0; ch < C::NCH; ++ch) {
+          uint32_t o[64];
+          if (n_t > 0) {
+            uint32_t (&o_lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
+            uint32_t (&o_hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[32]);
+            tmem_ld32x32b_x32(tO + ch * 64, o_lo);
+            tmem_ld32x32b_x32(tO + ch * 64 + 32, o_hi);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) o[i] = 0u;
+            for (int i = 0; i < 64; ++i) o[i] = 0u;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            uint4 v4;
+            v4.x = pack_half2(__uint_as_float(o[8 * u + 0]) * inv_l, __uint_as_float(o[8 * u + 1]) * inv_l, BF16);
+            v4.y = pack_half2(__uint_as_float(o[8 * u + 2]) * inv_l, __uint_as_float(o[8 * u + 3]) * inv_l, BF16);
+            v4.z = pack_half2(__uint_as_float(o[8 * u + 4]) * inv_l, __uint_as_float(o[8 * u + 5]) * inv_l, BF16);
+            v4.w = pack_half2(__uint_as_float(o[8 * u + 6]) * inv_l, __uint_as_float(o[8 * u + 7]) * inv_l, BF16);
+            if (row_ok) *reinterpret_cast<uint4*>(orow + ch * 64 + u * 8) = v4;
+          }
         }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          uint4 w;
-          w.x = pack_half2(__uint_as_float(o[8 * u + 0]) * inv_l, __uint_as_float(o[8 * u + 1]) * inv_l, BF16);
-          w.y = pack_half2(__uint_as_float(o[8 * u + 2]) * inv_l, __uint_as_float(o[8 * u + 3]) * inv_l, BF16);
-          w.z = pack_half2(__uint_as_float(o[8 * u + 4]) * inv_l, __uint_as_float(o[8 * u + 5]) * inv_l, BF16);
-          w.w = pack_half2(__uint_as_float(o[8 * u + 6]) * inv_l, __uint_as_float(o[8 * u + 7]) * inv_l, BF16);
-          // 128-byte swizzle: 16-byte unit u of row r sits at unit u ^ (r mod 8)
-          *reinterpret_cast<uint4*>(otile + ch * C::Q_CHUNK + r * 128 + ((u ^ (r & 7)) << 4)) = w;
+        if (row_ok && p.lse != nullptr) {
+          p.lse[static_cast<size_t>(w.bh) * p.Nq + row] =
+              (l > 0.f) ? (m_used + __log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
         }
       }
-      if (p.lse != nullptr && row < p.Nq) {
-        p.lse[static_cast<size_t>(bh) * p.Nq + row] =
-            (l > 0.f) ? (m_used + __log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
-      }
-      fence_proxy_async_smem();
-    }
-    named_barrier_sync(1 + t, kBM);
-    if (r == 0 && ok && !*abort_flag && row_min < p.Nq) {
-      for (int ch = 0; ch < C::NCH; ++ch)
-        tma_store_3d(&tmO, smem_u32(otile + ch * C::Q_CHUNK), ch * 64, q0 + t * kBM, bh);
-      tma_store_commit_and_wait_read();
+      // The next unit: every lane reads the response, then one arrival per warp.
+      const int sl = k & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_clc_full(sl), (k >> 1) & 1, wc))) { ok = false; break; }
+      uint32_t next;
+      const bool more = clc_query(clc_resp(sl), next);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_clc_empty(sl));
+      ++k;
+      if (!more) break;
+      unit = static_cast<int>(next);
     }
   }
 

@@ -30,6 +30,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction (three-operand form of max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi, bool bf16) {
   uint32_t r;
   if (bf16) {
@@ -97,6 +104,28 @@ __device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t x2) {
   const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
   const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
   return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+}
+
+// Cluster launch control (sm_100): ask the hardware scheduler for the work of a CTA of
+// this grid that has not started yet. The 16-byte response lands in shared memory and
+// completes 16 transaction bytes on the mbarrier; a CTA taken this way never launches.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp_smem, uint32_t bar) {
+  asm volatile(
+      "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];"
+      :: "r"(resp_smem), "r"(bar) : "memory");
+}
+
+// Decode a response: true and the taken CTA's x index, or false once no CTA is left.
+__device__ __forceinline__ bool clc_query(uint32_t resp_smem, uint32_t& cta_x) {
+  uint32_t ok, x;
+  asm volatile(
+      "{\n\t.reg .b128 r;\n\t.reg .pred p;\n\tld.shared.b128 r, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\tmov.u32 %1, 0;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+      : "=r"(ok), "=r"(x) : "r"(resp_smem) : "memory");
+  cta_x = x;
+  return ok != 0;
 }
 
 // Warpgroup-wide register re-allocation (all four warps of a warpgroup execute it).
