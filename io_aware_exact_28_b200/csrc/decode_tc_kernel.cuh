@@ -12,10 +12,14 @@
 //     O^T[d x heads]     += V_tile^T . P^T                (M = d = 128, N = 16, K = 128)
 // Q holds up to 16 query heads of one KV head (rows past the group are never stored).
 //
-// Persistent CTAs (one per SM). CTA c takes work units u = c, c + grid, ... of the list
-// (split, sequence, KV-head tile) in split-major order, so every CTA gets nearly the same
-// number of full units; empty units (split start past kv_len) are skipped by every role
-// alike. Warps:
+// Persistent CTAs (one per SM). A work unit is one split (up to split_tokens tokens) of
+// one (sequence, KV-head tile); its weight is 4 per 128-token tile plus 1 for its fixed
+// work (query load, epilogue). Units are ordered (sequence, head tile, split), splits past
+// kv_len do not exist, and CTA c takes the units whose weight prefix starts in
+// [c W / grid, (c+1) W / grid), W the total: each CTA gets a contiguous run of units within
+// one unit's weight of the average, whatever the kv_len mix. Warp 0 locates the run's
+// first unit with a scan over the sequences' weights (a closed form per kv_len) and every
+// role walks the same run (TcSched). Warps:
 //   0-3  softmax: thread t owns token t of the tile (TMEM lane t of S^T) and row d = t
 //        of O^T; warp-level max, cross-warp max through shared memory + an mbarrier,
 //        lazy rescale of O^T (threshold 2^8), P^T written to shared memory in the
@@ -40,11 +44,6 @@ namespace fa {
 constexpr int kTcD = 128;
 constexpr int kTcTile = 128;                 // tokens per tile (MMA M for S^T)
 constexpr int kTcStages = 3;
-// Next-unit L2 prefetch: measured slower on B200 (the prefetch traffic competes with the
-// ring's own loads), so off unless built with -DFA_TC_UNIT_PREFETCH=1.
-#ifndef FA_TC_UNIT_PREFETCH
-#define FA_TC_UNIT_PREFETCH 0
-#endif
 constexpr int kTcThreads = 224;
 constexpr int kTcWarpKProd = 4;
 constexpr int kTcWarpMma = 5;
@@ -63,7 +62,8 @@ constexpr int kTcOffBar = kTcOffRed + 2 * 4 * kTcN * 4;
 // barriers: kfull[3] kempty[3] vfull[3] vempty[3] qfull[2] qempty[2] s[2] p[2] o x pv drain
 constexpr int kTcNBars = 4 * kTcStages + 12;
 constexpr int kTcOffMisc = kTcOffBar + kTcNBars * 8;
-constexpr int kTcSmemBytes = kTcOffMisc + 16 + 1024;
+constexpr int kTcOffSched = kTcOffMisc + 16;              // the CTA's first unit (TcSched)
+constexpr int kTcSmemBytes = kTcOffSched + 48 + 1024;
 constexpr uint32_t kTcTmemCols = 64;                      // S^T x2 [0,32), O^T [32,48)
 static_assert(kTcSmemBytes <= 227 * 1024, "shared memory budget");
 
@@ -78,8 +78,6 @@ __device__ long long g_fa_tc_trace[8][1024];
 #endif
 
 struct DecodeTcParams {
-  const uint16_t* kc;     // [B, Hkv, max_len, 128] (for L2 prefetch of whole units)
-  const uint16_t* vc;
   const int* kv_lens;     // [B]
   float* ws_o;            // [B, Hq, n_split, 128]
   float* ws_lse;          // [B, Hq, n_split]
@@ -94,39 +92,123 @@ struct TcUnit {
   int b, kvh, g0, split, t0, t1;
 };
 
-// Work unit u in split-major order: u = (split * B + b) * (Hkv * n_gt) + kv-head tile.
-__device__ __forceinline__ bool tc_unit(const DecodeTcParams& p, int u, TcUnit& w) {
-  const int per_split = p.B * p.Hkv * p.n_gt;
-  w.split = u / per_split;
-  const int rem = u - w.split * per_split;
-  w.b = rem / (p.Hkv * p.n_gt);
-  const int r2 = rem - w.b * (p.Hkv * p.n_gt);
-  w.kvh = r2 / p.n_gt;
-  w.g0 = (r2 - w.kvh * p.n_gt) * p.GT;
-  int len = p.kv_lens[w.b];
-  len = len < 0 ? 0 : (len > p.max_len ? p.max_len : len);
-  w.t0 = w.split * p.split_tokens;
-  w.t1 = min(len, w.t0 + p.split_tokens);
-  return w.t0 < w.t1;
+__device__ __forceinline__ int tc_seq_len(const DecodeTcParams& p, int b) {
+  const int len = p.kv_lens[b];
+  return len < 0 ? 0 : (len > p.max_len ? p.max_len : len);
 }
 
-// Walks the tiles of this CTA's work units in order (units u = blockIdx.x + k * gridDim.x
-// with t0 < kv_len; tiles of 128 tokens from t0 to t1).
+// Weight of split s of a sequence of length len (0 if the split does not exist).
+__device__ __forceinline__ int tc_split_weight(const DecodeTcParams& p, int len, int s) {
+  const int t0 = s * p.split_tokens;
+  const int n = min(len, t0 + p.split_tokens) - t0;
+  return n > 0 ? 4 * ((n + kTcTile - 1) / kTcTile) + 1 : 0;
+}
+
+// Weight of all splits of one (sequence, head tile).
+__device__ __forceinline__ long long tc_seq_weight(const DecodeTcParams& p, int len) {
+  const int full = len / p.split_tokens;
+  const long long wf = 4 * (p.split_tokens / kTcTile) + 1;
+  return full * wf + tc_split_weight(p, len, full);
+}
+
+// Position in this CTA's run of units: sequence b, head tile hg (KV head hg / n_gt), split
+// s; pre = weight prefix at the unit's start; the run ends at the first unit with pre >= hi.
+struct TcSched {
+  int b, hg, s, len;
+  long long pre, hi;
+  __device__ __forceinline__ bool valid(const DecodeTcParams& p) const { return b < p.B && pre < hi; }
+  __device__ __forceinline__ void advance(const DecodeTcParams& p) {
+    pre += tc_split_weight(p, len, s);
+    if (++s * p.split_tokens < len) return;
+    s = 0;
+    if (++hg < p.Hkv * p.n_gt) return;
+    hg = 0;
+    for (++b; b < p.B; ++b) {
+      len = tc_seq_len(p, b);
+      if (len > 0) break;
+    }
+  }
+  __device__ __forceinline__ void unit(const DecodeTcParams& p, TcUnit& w) const {
+    w.b = b;
+    w.kvh = hg / p.n_gt;
+    w.g0 = (hg - w.kvh * p.n_gt) * p.GT;
+    w.split = s;
+    w.t0 = s * p.split_tokens;
+    w.t1 = min(len, w.t0 + p.split_tokens);
+  }
+};
+
+// The first unit of CTA blockIdx.x's run (executed by one full warp; lane 0's result).
+__device__ __forceinline__ TcSched tc_sched_start(const DecodeTcParams& p) {
+  const int lane = threadIdx.x & 31;
+  const long long HT = static_cast<long long>(p.Hkv) * p.n_gt;
+  long long total = 0;
+  for (int b0 = 0; b0 < p.B; b0 += 32) {
+    long long v = (b0 + lane < p.B) ? tc_seq_weight(p, tc_seq_len(p, b0 + lane)) : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    total += v;
+  }
+  total *= HT;
+  const long long lo = total * blockIdx.x / gridDim.x;
+  TcSched sc;
+  sc.b = p.B;
+  sc.hg = sc.s = sc.len = 0;
+  sc.pre = total;
+  sc.hi = total * (blockIdx.x + 1) / gridDim.x;
+  long long run = 0;                                   // weight before sequence b0
+  for (int b0 = 0; b0 < p.B; b0 += 32) {
+    const int b = b0 + lane;
+    const int len = b < p.B ? tc_seq_len(p, b) : 0;
+    const long long wb = b < p.B ? tc_seq_weight(p, len) * HT : 0;
+    long long incl = wb;                               // inclusive scan over the lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, wb > 0 && run + incl > lo);
+    if (hit) {
+      const int src = __ffs(hit) - 1;
+      const long long before = run + __shfl_sync(0xffffffffu, incl - wb, src);
+      const int len_b = __shfl_sync(0xffffffffu, len, src);
+      const long long w1 = tc_seq_weight(p, len_b);    // one head tile's splits
+      const long long q = lo - before;
+      sc.b = b0 + src;
+      sc.len = len_b;
+      sc.hg = static_cast<int>(q / w1);
+      const long long r = q - sc.hg * w1;
+      const long long wf = 4 * (p.split_tokens / kTcTile) + 1;
+      sc.s = static_cast<int>(r / wf);
+      sc.pre = before + sc.hg * w1 + sc.s * wf;
+      if (sc.pre < lo) sc.advance(p);                  // starts in the previous CTA's share
+      break;
+    }
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return sc;
+}
+
+// Walks the tiles (128 tokens from t0 to t1) of the units of this CTA's run.
 struct TcTiles {
-  int u, t;
+  TcSched sc;
+  int t;
   TcUnit w;
-  __device__ __forceinline__ bool first_unit_from(const DecodeTcParams& p, int u0, int n_units) {
-    for (u = u0; u < n_units; u += gridDim.x)
-      if (tc_unit(p, u, w)) { t = w.t0; return true; }
-    return false;
+  __device__ __forceinline__ bool first(const DecodeTcParams& p, const TcSched& start) {
+    sc = start;
+    if (!sc.valid(p)) return false;
+    sc.unit(p, w);
+    t = w.t0;
+    return true;
   }
-  __device__ __forceinline__ bool first(const DecodeTcParams& p, int n_units) {
-    return first_unit_from(p, blockIdx.x, n_units);
-  }
-  __device__ __forceinline__ bool next(const DecodeTcParams& p, int n_units) {
+  __device__ __forceinline__ bool next(const DecodeTcParams& p) {
     t += kTcTile;
     if (t < w.t1) return true;
-    return first_unit_from(p, u + gridDim.x, n_units);
+    sc.advance(p);
+    if (!sc.valid(p)) return false;
+    sc.unit(p, w);
+    t = w.t0;
+    return true;
   }
   __device__ __forceinline__ bool unit_first() const { return t == w.t0; }
   __device__ __forceinline__ bool unit_last() const { return t + kTcTile >= w.t1; }
@@ -185,6 +267,11 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   // P^T buffers start at zero: rows past the head tile stay zero for the whole kernel.
   for (int i = threadIdx.x; i < (2 * kTcPBytes) / 16; i += kTcThreads)
     reinterpret_cast<uint4*>(sbase + kTcOffP)[i] = make_uint4(0, 0, 0, 0);
+  TcSched* sched0 = reinterpret_cast<TcSched*>(sbase + kTcOffSched);
+  if (warp == 0) {
+    const TcSched sc = tc_sched_start(p);
+    if (lane == 0) *sched0 = sc;
+  }
   if (warp == kTcWarpMma) tmem_alloc(smem_u32(tmem_slot), kTcTmemCols);
   if (warp == kTcWarpKProd && lane == 0) {
     prefetch_tmap(&tmK);
@@ -197,7 +284,7 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, &g_fa_status, p.timeout_ns};
-  const int n_units = p.n_split * p.B * p.Hkv * p.n_gt;
+  const TcSched start = *sched0;
 
   if (warp == kTcWarpKProd || warp == kTcWarpVProd) {
     // ---------------------------------------------------------------- TMA producers
@@ -205,20 +292,10 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       const bool is_k = warp == kTcWarpKProd;
       const CUtensorMap* tm = is_k ? &tmK : &tmV;
       TcTiles cur;
-      bool have = cur.first(p, n_units);
+      bool have = cur.first(p, start);
       int jg = 0, uc = 0;
       bool ok = true;
       for (; have && ok; ++jg) {
-        if (cur.unit_first() && FA_TC_UNIT_PREFETCH) {
-          // L2 prefetch of the next unit's rows (contiguous per tensor): its tile loads
-          // then hit L2 instead of paying the full DRAM latency under load.
-          TcTiles nu = cur;
-          if (nu.first_unit_from(p, cur.u + gridDim.x, n_units)) {
-            const size_t row0 = (static_cast<size_t>(nu.w.b) * p.Hkv + nu.w.kvh) * p.max_len + nu.w.t0;
-            const uint32_t bytes = static_cast<uint32_t>(nu.w.t1 - nu.w.t0) * kTcD * 2;
-            bulk_prefetch_l2((is_k ? p.kc : p.vc) + row0 * kTcD, bytes);
-          }
-        }
         if (is_k && cur.unit_first()) {
           // Query rows of the unit: 16 rows from head (b, kvh*G + g0) on (rows past the
           // head tile are loaded but never used); Q buffer uc % 2.
@@ -243,7 +320,7 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const uint32_t dst = base + st * kTcStageBytes + (is_k ? 0 : kTcTileBytes);
         const int bhkv = cur.w.b * p.Hkv + cur.w.kvh;
         for (int ch = 0; ch < 2; ++ch) tma_load_3d(dst + ch * kTcChunk, tm, full, ch * 64, cur.t, bhkv);
-        have = cur.next(p, n_units);
+        have = cur.next(p);
       }
       if (!ok || *abort_flag) {
         // Loads still in flight must land before the CTA exits.
@@ -288,7 +365,7 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         return true;
       };
       TcTiles cur;
-      bool have = cur.first(p, n_units);
+      bool have = cur.first(p, start);
       if (have) {
         ok = wait_s_inputs(0, cur);
         if (ok) {
@@ -298,7 +375,7 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       }
       for (int j = 0; have && ok; ++j) {
         TcTiles nxt = cur;
-        const bool have_next = nxt.next(p, n_units);
+        const bool have_next = nxt.next(p);
         if (have_next) {
           if (!wait_s_inputs(j + 1, nxt)) { ok = false; break; }
           FA_TC_EVENT(1, j + 1);
@@ -369,9 +446,9 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       return true;
     };
 
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    for (TcSched sc = start; sc.valid(p) && ok; sc.advance(p)) {
       TcUnit w;
-      if (!tc_unit(p, u, w)) continue;
+      sc.unit(p, w);
       float m[GT], l[GT];
 #pragma unroll
       for (int h = 0; h < GT; ++h) { m[h] = -CUDART_INF_F; l[h] = 0.f; }

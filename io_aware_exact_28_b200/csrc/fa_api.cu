@@ -261,8 +261,6 @@ fa_status launch_decode_tc_t(int dev, const void* q, const void* kc, const void*
       !make_tile_map(&mq, q, fa::kTcD, B * Hq, 1, BF16, fa::kTcN))
     return FA_ERR_CUDA;
   fa::DecodeTcParams tp;
-  tp.kc = static_cast<const uint16_t*>(kc);
-  tp.vc = static_cast<const uint16_t*>(vc);
   tp.kv_lens = kv_lens;
   tp.ws_o = reinterpret_cast<float*>(ws);
   tp.ws_lse = reinterpret_cast<float*>(ws + L.lse_off);
