@@ -100,7 +100,9 @@ FA_API size_t fa_decode_workspace_bytes(int B, int Hq, int max_kv_len, int d);
  *
  *   q         [B, Hq, d]               fp16/bf16
  *   kcache,
- *   vcache    [B, Hkv, max_kv_len, d]  fp16/bf16; rows >= kv_lens[b] are never read
+ *   vcache    [B, Hkv, max_kv_len, d]  fp16/bf16; rows >= kv_lens[b] never affect the
+ *                                      result, whatever they hold (the d = 128 kernel may
+ *                                      fetch them as part of a 128-row tile, then masks them)
  *   kv_lens   [B] int32, device memory; values are clamped to [0, max_kv_len]
  *   o         [B, Hq, d]               same dtype as q
  *   lse       [B, Hq] fp32, may be NULL

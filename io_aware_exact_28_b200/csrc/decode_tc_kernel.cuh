@@ -12,18 +12,19 @@
 //     O^T[d x heads]     += V_tile^T . P^T                (M = d = 128, N = 16, K = 128)
 // Q holds up to 16 query heads of one KV head (rows past the group are never stored).
 //
-// Persistent CTAs (one per SM). A work unit is one split (up to split_tokens tokens) of
-// one (sequence, KV-head tile); its weight is 4 per 128-token tile plus 1 for its fixed
-// work (query load, epilogue). Units are ordered (sequence, head tile, split), splits past
-// kv_len do not exist, and CTA c takes the units whose weight prefix starts in
-// [c W / grid, (c+1) W / grid), W the total: each CTA gets a contiguous run of units within
-// one unit's weight of the average, whatever the kv_len mix. Warp 0 locates the run's
-// first unit with a scan over the sequences' weights (a closed form per kv_len) and every
-// role walks the same run (TcSched). Warps:
+// Persistent CTAs (one per SM), scheduled dynamically. A work unit is one split (up to
+// split_tokens tokens) of one (sequence, KV-head tile); the units that exist (splits
+// before kv_len) are numbered in (sequence, head tile, split) order. CTA c starts with
+// unit c; each further unit is a ticket from an atomic counter in the workspace (zeroed
+// before the launch), so a CTA that streams slower simply takes fewer units. The K
+// producer takes the tickets and hands each unit to the other roles through a 4-deep
+// shared-memory ring of unit descriptors. Warps:
 //   0-3  softmax: thread t owns token t of the tile (TMEM lane t of S^T) and row d = t
 //        of O^T; warp-level max, cross-warp max through shared memory + an mbarrier,
 //        lazy rescale of O^T (threshold 2^8), P^T written to shared memory in the
-//        canonical K-major 128-byte-swizzle layout; per-unit epilogue writes the partial.
+//        canonical K-major 128-byte-swizzle layout. The epilogue of unit k (normalised
+//        partial row + LSE) runs after unit k + 1's first P^T: unit k accumulates in
+//        O^T[k & 1], so its last P.V completes while the next unit already streams.
 //   4    K producer: the unit's query rows (TMA, double-buffered) and K tiles.
 //   5    TMEM allocator and single-thread tcgen05.mma issuer. S^T of tile j+1 is issued
 //        before P.V of tile j, so scores are ready when the softmax warps need them.
@@ -59,18 +60,26 @@ constexpr int kTcOffQ = kTcStages * kTcStageBytes;        // Q[2]
 constexpr int kTcOffP = kTcOffQ + 2 * kTcQBytes;          // P[2]
 constexpr int kTcOffRed = kTcOffP + 2 * kTcPBytes;        // float [2][4 warps][16]
 constexpr int kTcOffBar = kTcOffRed + 2 * 4 * kTcN * 4;
-// barriers: kfull[3] kempty[3] vfull[3] vempty[3] qfull[2] qempty[2] s[2] p[2] o x pv drain
-constexpr int kTcNBars = 4 * kTcStages + 12;
-constexpr int kTcOffMisc = kTcOffBar + kTcNBars * 8;
-constexpr int kTcOffSched = kTcOffMisc + 16;              // the CTA's first unit (TcSched)
-constexpr int kTcSmemBytes = kTcOffSched + 48 + 1024;
-constexpr uint32_t kTcTmemCols = 64;                      // S^T x2 [0,32), O^T [32,48)
+// barriers: kfull[3] kempty[3] vfull[3] vempty[3] qfull[2] qempty[2] s[2] p[2] o[2] x pv drain
+// + unit ring: ufull[4] uempty[4]
+constexpr int kTcUnitRing = 4;
+constexpr int kTcNBars = 4 * kTcStages + 13 + 2 * kTcUnitRing;
+constexpr int kTcOffMisc = (kTcOffBar + kTcNBars * 8 + 15) / 16 * 16;
+constexpr int kTcOffSched = kTcOffMisc + 16;              // TcStart (8-byte fields)
+constexpr int kTcOffRing = kTcOffSched + 64;               // unit descriptors (int4 each)
+constexpr int kTcSmemBytes = kTcOffRing + 16 * kTcUnitRing + 1024;
+static_assert(kTcOffQ % 1024 == 0 && kTcOffP % 1024 == 0, "128-byte-swizzle operands need 1 KB alignment");
+static_assert(kTcOffRed % 16 == 0 && kTcOffBar % 8 == 0, "reduction / barrier alignment");
+static_assert(kTcOffMisc % 16 == 0 && kTcOffSched % 16 == 0 && kTcOffRing % 16 == 0,
+              "16-byte shared accesses (descriptor ring, TcStart) need 16-byte alignment");
+constexpr uint32_t kTcTmemCols = 64;                      // S^T x2 [0,32), O^T x2 [32,64)
 static_assert(kTcSmemBytes <= 227 * 1024, "shared memory budget");
 
 // Debug builds only (-DFA_TC_TRACE): CTA 0 records clock64() at pipeline events of its
 // first 1024 tiles into g_fa_tc_trace[event][tile], read back with fa_debug_tc_trace().
 #ifdef FA_TC_TRACE
 __device__ long long g_fa_tc_trace[8][1024];
+__device__ long long g_fa_tc_clock[148][6];   // per CTA: clock64 / globaltimer at start and end, tiles, SM
 #define FA_TC_EVENT(ev, idx) \
   do { if (blockIdx.x == 0 && (idx) < 1024) g_fa_tc_trace[ev][idx] = clock64(); } while (0)
 #else
@@ -79,6 +88,7 @@ __device__ long long g_fa_tc_trace[8][1024];
 
 struct DecodeTcParams {
   const int* kv_lens;     // [B]
+  unsigned* tickets;      // unit counter, zero at launch
   float* ws_o;            // [B, Hq, n_split, 128]
   float* ws_lse;          // [B, Hq, n_split]
   int B, Hq, Hkv, G, GT;  // GT = heads per tile (<= 16), n_gt tiles per KV head
@@ -97,122 +107,77 @@ __device__ __forceinline__ int tc_seq_len(const DecodeTcParams& p, int b) {
   return len < 0 ? 0 : (len > p.max_len ? p.max_len : len);
 }
 
-// Weight of split s of a sequence of length len (0 if the split does not exist).
-__device__ __forceinline__ int tc_split_weight(const DecodeTcParams& p, int len, int s) {
-  const int t0 = s * p.split_tokens;
-  const int n = min(len, t0 + p.split_tokens) - t0;
-  return n > 0 ? 4 * ((n + kTcTile - 1) / kTcTile) + 1 : 0;
-}
-
-// Weight of all splits of one (sequence, head tile).
-__device__ __forceinline__ long long tc_seq_weight(const DecodeTcParams& p, int len) {
-  const int full = len / p.split_tokens;
-  const long long wf = 4 * (p.split_tokens / kTcTile) + 1;
-  return full * wf + tc_split_weight(p, len, full);
-}
-
-// Position in this CTA's run of units: sequence b, head tile hg (KV head hg / n_gt), split
-// s; pre = weight prefix at the unit's start; the run ends at the first unit with pre >= hi.
-struct TcSched {
-  int b, hg, s, len;
-  long long pre, hi;
-  __device__ __forceinline__ bool valid(const DecodeTcParams& p) const { return b < p.B && pre < hi; }
-  __device__ __forceinline__ void advance(const DecodeTcParams& p) {
-    pre += tc_split_weight(p, len, s);
-    if (++s * p.split_tokens < len) return;
-    s = 0;
-    if (++hg < p.Hkv * p.n_gt) return;
-    hg = 0;
-    for (++b; b < p.B; ++b) {
+// Position of a unit in the numbering: sequence b (length len, ns splits) whose first unit
+// is number base; unit base + hg * ns + s is split s of head tile hg.
+struct TcCursor {
+  int b, len, ns;
+  long long base;
+  // Move forward to unit k (k >= base, k below the total) and decode it.
+  __device__ __forceinline__ void locate(const DecodeTcParams& p, long long k, TcUnit& w) {
+    const int HT = p.Hkv * p.n_gt;
+    while (k >= base + static_cast<long long>(HT) * ns) {
+      base += static_cast<long long>(HT) * ns;
+      ++b;
       len = tc_seq_len(p, b);
-      if (len > 0) break;
+      ns = (len + p.split_tokens - 1) / p.split_tokens;
     }
-  }
-  __device__ __forceinline__ void unit(const DecodeTcParams& p, TcUnit& w) const {
+    const int r = static_cast<int>(k - base);
+    const int hg = r / ns, sp = r - hg * ns;
     w.b = b;
     w.kvh = hg / p.n_gt;
     w.g0 = (hg - w.kvh * p.n_gt) * p.GT;
-    w.split = s;
-    w.t0 = s * p.split_tokens;
+    w.split = sp;
+    w.t0 = sp * p.split_tokens;
     w.t1 = min(len, w.t0 + p.split_tokens);
   }
 };
 
-// The first unit of CTA blockIdx.x's run (executed by one full warp; lane 0's result).
-__device__ __forceinline__ TcSched tc_sched_start(const DecodeTcParams& p) {
+struct TcStart {
+  TcCursor cur;           // positioned at or before unit blockIdx.x
+  long long total;        // units that exist
+};
+
+// Total unit count and a cursor at sequence 0 (executed by one full warp).
+__device__ __forceinline__ TcStart tc_start(const DecodeTcParams& p) {
   const int lane = threadIdx.x & 31;
-  const long long HT = static_cast<long long>(p.Hkv) * p.n_gt;
   long long total = 0;
   for (int b0 = 0; b0 < p.B; b0 += 32) {
-    long long v = (b0 + lane < p.B) ? tc_seq_weight(p, tc_seq_len(p, b0 + lane)) : 0;
+    const int len = (b0 + lane < p.B) ? tc_seq_len(p, b0 + lane) : 0;
+    long long v = (len + p.split_tokens - 1) / p.split_tokens;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     total += v;
   }
-  total *= HT;
-  const long long lo = total * blockIdx.x / gridDim.x;
-  TcSched sc;
-  sc.b = p.B;
-  sc.hg = sc.s = sc.len = 0;
-  sc.pre = total;
-  sc.hi = total * (blockIdx.x + 1) / gridDim.x;
-  long long run = 0;                                   // weight before sequence b0
-  for (int b0 = 0; b0 < p.B; b0 += 32) {
-    const int b = b0 + lane;
-    const int len = b < p.B ? tc_seq_len(p, b) : 0;
-    const long long wb = b < p.B ? tc_seq_weight(p, len) * HT : 0;
-    long long incl = wb;                               // inclusive scan over the lanes
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const long long y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const unsigned hit = __ballot_sync(0xffffffffu, wb > 0 && run + incl > lo);
-    if (hit) {
-      const int src = __ffs(hit) - 1;
-      const long long before = run + __shfl_sync(0xffffffffu, incl - wb, src);
-      const int len_b = __shfl_sync(0xffffffffu, len, src);
-      const long long w1 = tc_seq_weight(p, len_b);    // one head tile's splits
-      const long long q = lo - before;
-      sc.b = b0 + src;
-      sc.len = len_b;
-      sc.hg = static_cast<int>(q / w1);
-      const long long r = q - sc.hg * w1;
-      const long long wf = 4 * (p.split_tokens / kTcTile) + 1;
-      sc.s = static_cast<int>(r / wf);
-      sc.pre = before + sc.hg * w1 + sc.s * wf;
-      if (sc.pre < lo) sc.advance(p);                  // starts in the previous CTA's share
-      break;
-    }
-    run += __shfl_sync(0xffffffffu, incl, 31);
-  }
-  return sc;
+  TcStart st;
+  st.total = total * p.Hkv * p.n_gt;
+  st.cur.b = 0;
+  st.cur.len = tc_seq_len(p, 0);
+  st.cur.ns = (st.cur.len + p.split_tokens - 1) / p.split_tokens;
+  st.cur.base = 0;
+  return st;
 }
 
-// Walks the tiles (128 tokens from t0 to t1) of the units of this CTA's run.
+// Unit descriptor passed from the K producer to the other roles (b < 0: no more units).
+struct TcDesc {
+  int b, kvh, g0, split;
+};
+
+// The tiles (128 tokens from t0 to t1) of one unit.
 struct TcTiles {
-  TcSched sc;
-  int t;
   TcUnit w;
-  __device__ __forceinline__ bool first(const DecodeTcParams& p, const TcSched& start) {
-    sc = start;
-    if (!sc.valid(p)) return false;
-    sc.unit(p, w);
-    t = w.t0;
-    return true;
-  }
-  __device__ __forceinline__ bool next(const DecodeTcParams& p) {
-    t += kTcTile;
-    if (t < w.t1) return true;
-    sc.advance(p);
-    if (!sc.valid(p)) return false;
-    sc.unit(p, w);
-    t = w.t0;
-    return true;
-  }
+  int t;
   __device__ __forceinline__ bool unit_first() const { return t == w.t0; }
   __device__ __forceinline__ bool unit_last() const { return t + kTcTile >= w.t1; }
 };
+
+__device__ __forceinline__ void tc_unit_from(const DecodeTcParams& p, const TcDesc& d, TcUnit& w) {
+  w.b = d.b;
+  w.kvh = d.kvh;
+  w.g0 = d.g0;
+  w.split = d.split;
+  w.t0 = d.split * p.split_tokens;
+  w.t1 = min(tc_seq_len(p, d.b), w.t0 + p.split_tokens);
+}
 
 template <bool BF16, int GT>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -224,6 +189,12 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   uint8_t* sbase = smem_raw + (base - raw);
 
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#ifdef FA_TC_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 148) {
+    g_fa_tc_clock[blockIdx.x][0] = clock64();
+    g_fa_tc_clock[blockIdx.x][1] = static_cast<long long>(globaltimer_ns());
+  }
+#endif
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -236,10 +207,20 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   auto bar_qempty = [&](int b) { return bar0 + 8u * (4 * kTcStages + 2 + b); };
   auto bar_s = [&](int b) { return bar0 + 8u * (4 * kTcStages + 4 + b); };   // S^T[b] ready
   auto bar_p = [&](int b) { return bar0 + 8u * (4 * kTcStages + 6 + b); };   // P^T[b] written
-  const uint32_t bar_o = bar0 + 8u * (4 * kTcStages + 8);    // O^T of a unit complete
-  const uint32_t bar_x = bar0 + 8u * (4 * kTcStages + 9);    // cross-warp exchange (4)
-  const uint32_t bar_pv = bar0 + 8u * (4 * kTcStages + 10);  // each P.V done
-  const uint32_t bar_drain = bar0 + 8u * (4 * kTcStages + 11);
+  // O^T[b] of a unit complete (unit k of the CTA accumulates in O^T[k & 1])
+  auto bar_o = [&](int b) { return bar0 + 8u * (4 * kTcStages + 8 + b); };
+  const uint32_t bar_x = bar0 + 8u * (4 * kTcStages + 10);   // cross-warp exchange (4)
+  const uint32_t bar_pv = bar0 + 8u * (4 * kTcStages + 11);  // each P.V done
+  const uint32_t bar_drain = bar0 + 8u * (4 * kTcStages + 12);
+  // Unit ring: slot n % 4 holds the descriptor of the CTA's n-th unit.
+  auto bar_ufull = [&](int n) { return bar0 + 8u * (4 * kTcStages + 13 + (n & (kTcUnitRing - 1))); };
+  auto bar_uempty = [&](int n) {
+    return bar0 + 8u * (4 * kTcStages + 13 + kTcUnitRing + (n & (kTcUnitRing - 1)));
+  };
+  // Plain shared accesses: mbarrier arrive / wait (asm with memory clobbers) order them.
+  int4* ring = reinterpret_cast<int4*>(sbase + kTcOffRing);
+  // Readers of each descriptor: V producer, MMA thread, 4 softmax warps.
+  constexpr int kTcRingReaders = 6;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + kTcOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + kTcOffMisc + 4);
   float* red = reinterpret_cast<float*>(sbase + kTcOffRed);  // [2][4][16]
@@ -257,20 +238,25 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       mbar_init(bar_s(b), 1);
       mbar_init(bar_p(b), 128);
     }
-    mbar_init(bar_o, 1);
+    mbar_init(bar_o(0), 1);
+    mbar_init(bar_o(1), 1);
     mbar_init(bar_x, 4);
     mbar_init(bar_pv, 1);
     mbar_init(bar_drain, 1);
+    for (int n = 0; n < kTcUnitRing; ++n) {
+      mbar_init(bar_ufull(n), 1);
+      mbar_init(bar_uempty(n), kTcRingReaders);
+    }
     *abort_flag = 0;
     fence_mbarrier_init();
   }
   // P^T buffers start at zero: rows past the head tile stay zero for the whole kernel.
   for (int i = threadIdx.x; i < (2 * kTcPBytes) / 16; i += kTcThreads)
     reinterpret_cast<uint4*>(sbase + kTcOffP)[i] = make_uint4(0, 0, 0, 0);
-  TcSched* sched0 = reinterpret_cast<TcSched*>(sbase + kTcOffSched);
+  TcStart* start0 = reinterpret_cast<TcStart*>(sbase + kTcOffSched);
   if (warp == 0) {
-    const TcSched sc = tc_sched_start(p);
-    if (lane == 0) *sched0 = sc;
+    const TcStart st = tc_start(p);
+    if (lane == 0) *start0 = st;
   }
   if (warp == kTcWarpMma) tmem_alloc(smem_u32(tmem_slot), kTcTmemCols);
   if (warp == kTcWarpKProd && lane == 0) {
@@ -284,44 +270,91 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, &g_fa_status, p.timeout_ns};
-  const TcSched start = *sched0;
+  // Reader side of the unit ring: the n-th unit's descriptor (false if the wait ran out).
+  auto ring_read = [&](int n, TcDesc& d) -> bool {
+    if (!mbar_wait(bar_ufull(n), (n / kTcUnitRing) & 1, wc)) return false;
+    const int4 v = ring[n & (kTcUnitRing - 1)];
+    d.b = v.x;
+    d.kvh = v.y;
+    d.g0 = v.z;
+    d.split = v.w;
+    return true;
+  };
 
   if (warp == kTcWarpKProd || warp == kTcWarpVProd) {
     // ---------------------------------------------------------------- TMA producers
     if (lane == 0) {
       const bool is_k = warp == kTcWarpKProd;
       const CUtensorMap* tm = is_k ? &tmK : &tmV;
-      TcTiles cur;
-      bool have = cur.first(p, start);
-      int jg = 0, uc = 0;
+      int jg = 0, uc = 0, n = 0;
       bool ok = true;
-      for (; have && ok; ++jg) {
-        if (is_k && cur.unit_first()) {
+      const TcStart st = *start0;
+      TcCursor cursor = st.cur;
+      long long ticket = blockIdx.x;                 // unit of the CTA's first ticket
+      while (ok) {
+        TcUnit w;
+        if (is_k) {
+          // Publish unit n (or the end) to the other roles.
+          const bool have = ticket < st.total;
+          if (have) cursor.locate(p, ticket, w);
+          if (n >= kTcUnitRing && !mbar_wait(bar_uempty(n), (n / kTcUnitRing - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          ring[n & (kTcUnitRing - 1)] = have ? make_int4(w.b, w.kvh, w.g0, w.split) : make_int4(-1, 0, 0, 0);
+          mbar_arrive(bar_ufull(n));
+          ++n;
+          if (!have) break;
           // Query rows of the unit: 16 rows from head (b, kvh*G + g0) on (rows past the
           // head tile are loaded but never used); Q buffer uc % 2.
           const int qb = uc & 1;
           if (uc >= 2 && !mbar_wait(bar_qempty(qb), ((uc >> 1) - 1) & 1, wc)) { ok = false; break; }
           mbar_arrive_expect_tx(bar_qfull(qb), kTcQBytes);
-          const int row0 = cur.w.b * p.Hq + cur.w.kvh * p.G + cur.w.g0;
+          const int row0 = w.b * p.Hq + w.kvh * p.G + w.g0;
           for (int ch = 0; ch < 2; ++ch)
             tma_load_3d(base + kTcOffQ + qb * kTcQBytes + ch * kTcSmallChunk, &tmQ, bar_qfull(qb),
                         ch * 64, row0, 0);
           ++uc;
+        } else {
+          TcDesc d;
+          if (!ring_read(n, d)) { ok = false; break; }
+          mbar_arrive(bar_uempty(n));
+          ++n;
+          if (d.b < 0) break;
+          tc_unit_from(p, d, w);
         }
-        const int st = jg % kTcStages;
-        const uint32_t empty = is_k ? bar_kempty(st) : bar_vempty(st);
-        const uint32_t full = is_k ? bar_kfull(st) : bar_vfull(st);
-        if (jg >= kTcStages && !mbar_wait(empty, ((jg / kTcStages) - 1) & 1, wc)) {
-          ok = false;
-          break;
+        unsigned next_ticket = 0;
+        bool asked = false;
+        const int bhkv = w.b * p.Hkv + w.kvh;
+        for (int t = w.t0; t < w.t1; t += kTcTile, ++jg) {
+          // The next ticket is drawn two tiles before this unit's loads end: late enough to
+          // balance, early enough that its latency hides behind these loads.
+          if (is_k && !asked && t + 2 * kTcTile >= w.t1) {
+            next_ticket = atomicAdd(p.tickets, 1u);
+            asked = true;
+          }
+          const int stg = jg % kTcStages;
+          const uint32_t empty = is_k ? bar_kempty(stg) : bar_vempty(stg);
+          const uint32_t full = is_k ? bar_kfull(stg) : bar_vfull(stg);
+          if (jg >= kTcStages && !mbar_wait(empty, ((jg / kTcStages) - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          if (is_k) FA_TC_EVENT(0, jg); else FA_TC_EVENT(6, jg);
+          mbar_arrive_expect_tx(full, kTcTileBytes);
+          const uint32_t dst = base + stg * kTcStageBytes + (is_k ? 0 : kTcTileBytes);
+          for (int ch = 0; ch < 2; ++ch) tma_load_3d(dst + ch * kTcChunk, tm, full, ch * 64, t, bhkv);
         }
-        if (is_k) FA_TC_EVENT(0, jg);
-        mbar_arrive_expect_tx(full, kTcTileBytes);
-        const uint32_t dst = base + st * kTcStageBytes + (is_k ? 0 : kTcTileBytes);
-        const int bhkv = cur.w.b * p.Hkv + cur.w.kvh;
-        for (int ch = 0; ch < 2; ++ch) tma_load_3d(dst + ch * kTcChunk, tm, full, ch * 64, cur.t, bhkv);
-        have = cur.next(p);
+        if (is_k) ticket = static_cast<long long>(gridDim.x) + next_ticket;
       }
+#ifdef FA_TC_TRACE
+      if (is_k && blockIdx.x < 148) {
+        uint32_t smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        g_fa_tc_clock[blockIdx.x][4] = jg;
+        g_fa_tc_clock[blockIdx.x][5] = smid;
+      }
+#endif
       if (!ok || *abort_flag) {
         // Loads still in flight must land before the CTA exits.
         for (int k = max(0, jg - kTcStages); k < jg; ++k)
@@ -338,7 +371,8 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       constexpr uint32_t IDESC_S = idesc_f16(kTcTile, kTcN, FMT, 0u, 0u);   // K-major A, B
       constexpr uint32_t IDESC_O = idesc_f16(kTcD, kTcN, FMT, 1u, 0u);      // A = V^T, MN-major
       bool ok = true, issued = false;
-      int uc = -1;                                   // unit counter (Q buffer uc % 2)
+      int uc = -1;                                   // unit of the S side (Q buffer uc % 2)
+      int uo = 0;                                    // unit of the P.V side (O^T buffer uo % 2)
       // S^T for tile j (K slot j % 3) with the current unit's Q; frees the K slot (and, on the
       // unit's last tile, the Q buffer) when it completes.
       auto issue_s = [&](int j, bool last_of_unit) {
@@ -364,8 +398,26 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         tc_fence_after();
         return true;
       };
+      // Next tile of the unit stream: 1 = a tile, 0 = no more units, -1 = a wait ran out.
+      int nu = 0;
+      auto advance = [&](TcTiles& it, bool first) -> int {
+        if (!first) {
+          it.t += kTcTile;
+          if (it.t < it.w.t1) return 1;
+        }
+        TcDesc d;
+        if (!ring_read(nu, d)) return -1;
+        mbar_arrive(bar_uempty(nu));
+        ++nu;
+        if (d.b < 0) return 0;
+        tc_unit_from(p, d, it.w);
+        it.t = it.w.t0;
+        return 1;
+      };
       TcTiles cur;
-      bool have = cur.first(p, start);
+      const int r0 = advance(cur, true);
+      bool have = r0 == 1;
+      if (r0 < 0) ok = false;
       if (have) {
         ok = wait_s_inputs(0, cur);
         if (ok) {
@@ -375,7 +427,9 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       }
       for (int j = 0; have && ok; ++j) {
         TcTiles nxt = cur;
-        const bool have_next = nxt.next(p);
+        const int rn = advance(nxt, false);
+        if (rn < 0) { ok = false; break; }
+        const bool have_next = rn == 1;
         if (have_next) {
           if (!wait_s_inputs(j + 1, nxt)) { ok = false; break; }
           FA_TC_EVENT(1, j + 1);
@@ -384,19 +438,23 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         if (!mbar_wait(bar_p(j & 1), (j >> 1) & 1, wc)) { ok = false; break; }
         FA_TC_EVENT(2, j);
         if (!mbar_wait(bar_vfull(j % kTcStages), (j / kTcStages) & 1, wc)) { ok = false; break; }
+        FA_TC_EVENT(7, j);
         tc_fence_after();
         const uint32_t va = base + (j % kTcStages) * kTcStageBytes + kTcTileBytes;
         const uint32_t pa = base + kTcOffP + (j & 1) * kTcPBytes;
         const bool acc0 = !cur.unit_first();
 #pragma unroll
         for (int kk = 0; kk < kTcTile / 16; ++kk) {
-          mma_f16_ss(tmem + 32, sdesc_mn_sw128(va + kk * 2048, kTcChunk),
+          mma_f16_ss(tmem + 32 + 16 * (uo & 1), sdesc_mn_sw128(va + kk * 2048, kTcChunk),
                      sdesc_k_sw128(pa + (kk >> 2) * kTcSmallChunk + (kk & 3) * 32), IDESC_O,
                      (acc0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar_vempty(j % kTcStages));
         mma_commit(bar_pv);
-        if (cur.unit_last()) mma_commit(bar_o);
+        if (cur.unit_last()) {
+          mma_commit(bar_o(uo & 1));
+          ++uo;
+        }
         cur = nxt;
         have = have_next;
       }
@@ -410,7 +468,7 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     const int t = threadIdx.x;                       // token of the tile / row d of O^T
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t tS = tmem + lane_base;            // S^T[b] at column 16 * b
-    const uint32_t tO = tmem + lane_base + 32;
+    const uint32_t tO0 = tmem + lane_base + 32;      // O^T[b] at column 32 + 16 b
     const float c = p.scale_log2;
     uint8_t* pbuf = sbase + kTcOffP;
     int jg = 0, uc = 0, xc = 0;
@@ -446,9 +504,53 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       return true;
     };
 
-    for (TcSched sc = start; sc.valid(p) && ok; sc.advance(p)) {
+    // The epilogue of unit k runs after the first P of unit k + 1 (or at the end), so the
+    // softmax warps never idle on unit k's last P.V: that product accumulates in O^T[k & 1]
+    // while unit k + 1 starts in O^T[(k + 1) & 1].
+    TcUnit w_prev;
+    float m_prev[GT], l_prev[GT];
+    bool have_prev = false;
+    auto epilogue = [&]() -> bool {
+      const int b = uc & 1;
+      bool got = true;
+      if (lane == 0) got = mbar_wait(bar_o(b), (uc >> 1) & 1, wc);
+      got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+      ++uc;
+      have_prev = false;
+      if (!got) return false;
+      tc_fence_after();
+      uint32_t ov[kTcN];
+      tmem_ld32x32b_x16(tO0 + 16 * b, ov);           // row d = t of O^T
+      float L[GT];
+#pragma unroll
+      for (int h = 0; h < GT; ++h) L[h] = l_prev[h];
+      if (!exchange(L, false)) return false;
+#pragma unroll
+      for (int h = 0; h < GT; ++h) {
+        if (w_prev.g0 + h >= p.G) break;
+        const int hq = w_prev.kvh * p.G + w_prev.g0 + h;
+        const size_t row = (static_cast<size_t>(w_prev.b) * p.Hq + hq) * p.n_split + w_prev.split;
+        p.ws_o[row * kTcD + t] = __uint_as_float(ov[h]) / L[h];
+        if (t == 0) p.ws_lse[row] = m_prev[h] + __log2f(L[h]);
+      }
+      return true;
+    };
+    int nu = 0;                                      // descriptors read
+    for (int uk = 0; ok; ++uk) {                     // uk: units started (O^T buffer uk % 2)
+      TcDesc d;
+      bool got_d = true;
+      if (lane == 0) got_d = ring_read(nu, d);
+      if (!__shfl_sync(0xffffffffu, got_d ? 1 : 0, 0)) { ok = false; break; }
+      d.b = __shfl_sync(0xffffffffu, d.b, 0);
+      d.kvh = __shfl_sync(0xffffffffu, d.kvh, 0);
+      d.g0 = __shfl_sync(0xffffffffu, d.g0, 0);
+      d.split = __shfl_sync(0xffffffffu, d.split, 0);
+      if (lane == 0) mbar_arrive(bar_uempty(nu));
+      ++nu;
+      if (d.b < 0) break;
       TcUnit w;
-      sc.unit(p, w);
+      tc_unit_from(p, d, w);
+      const uint32_t tO = tO0 + 16 * (uk & 1);
       float m[GT], l[GT];
 #pragma unroll
       for (int h = 0; h < GT; ++h) { m[h] = -CUDART_INF_F; l[h] = 0.f; }
@@ -531,34 +633,25 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         tc_fence_before();
         mbar_arrive(bar_p(jg & 1));
         if (t == 0) FA_TC_EVENT(5, jg);
+        if (tile == 0 && have_prev && !epilogue()) { ok = false; break; }
       }
       if (!ok) break;
-      // ------------------------------------------------------------ unit epilogue
-      bool got = true;
-      if (lane == 0) got = mbar_wait(bar_o, uc & 1, wc);
-      got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
-      ++uc;
-      if (!got) { ok = false; break; }
-      tc_fence_after();
-      uint32_t ov[kTcN];
-      tmem_ld32x32b_x16(tO, ov);                     // row d = t of O^T
-      float L[GT];
+      w_prev = w;
 #pragma unroll
-      for (int h = 0; h < GT; ++h) L[h] = l[h];
-      if (!exchange(L, false)) { ok = false; break; }
-#pragma unroll
-      for (int h = 0; h < GT; ++h) {
-        if (w.g0 + h >= p.G) break;
-        const int hq = w.kvh * p.G + w.g0 + h;
-        const size_t row = (static_cast<size_t>(w.b) * p.Hq + hq) * p.n_split + w.split;
-        p.ws_o[row * kTcD + t] = __uint_as_float(ov[h]) / L[h];
-        if (t == 0) p.ws_lse[row] = m[h] + __log2f(L[h]);
-      }
+      for (int h = 0; h < GT; ++h) { m_prev[h] = m[h]; l_prev[h] = l[h]; }
+      have_prev = true;
     }
+    if (ok && have_prev) epilogue();
   }
 
   tc_fence_before();
   __syncthreads();
+#ifdef FA_TC_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 148) {
+    g_fa_tc_clock[blockIdx.x][2] = clock64();
+    g_fa_tc_clock[blockIdx.x][3] = static_cast<long long>(globaltimer_ns());
+  }
+#endif
   if (warp == kTcWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTcTmemCols);

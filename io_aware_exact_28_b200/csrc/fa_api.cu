@@ -154,7 +154,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct DecodeLayout {
   int split_tokens, n_split;
-  size_t o_bytes, lse_off, total;
+  size_t o_bytes, lse_off, ticket_off, total;
 };
 
 // d = 128 decodes on the tensor cores in 128-token tiles (decode_tc_kernel.cuh) unless
@@ -181,7 +181,8 @@ bool decode_layout(int B, int Hq, int max_len, int d, DecodeLayout* L) {
   const size_t rows = static_cast<size_t>(B) * Hq * L->n_split;
   L->o_bytes = align_up(rows * d * sizeof(float), 256);
   L->lse_off = L->o_bytes;
-  L->total = L->o_bytes + align_up(rows * sizeof(float), 256);
+  L->ticket_off = L->lse_off + align_up(rows * sizeof(float), 256);   // tensor-core unit counter
+  L->total = L->ticket_off + 256;
   return true;
 }
 
@@ -262,6 +263,7 @@ fa_status launch_decode_tc_t(int dev, const void* q, const void* kc, const void*
     return FA_ERR_CUDA;
   fa::DecodeTcParams tp;
   tp.kv_lens = kv_lens;
+  tp.tickets = reinterpret_cast<unsigned*>(ws + L.ticket_off);
   tp.ws_o = reinterpret_cast<float*>(ws);
   tp.ws_lse = reinterpret_cast<float*>(ws + L.lse_off);
   tp.B = B;
@@ -278,6 +280,8 @@ fa_status launch_decode_tc_t(int dev, const void* q, const void* kc, const void*
   const long long n_units = static_cast<long long>(L.n_split) * B * Hkv * tp.n_gt;
   if (n_units >= (1LL << 31)) return FA_ERR_INVALID_ARG;
   const int grid = static_cast<int>(n_units < sm_count[dev] ? n_units : sm_count[dev]);
+  // The unit counter starts at zero on every call (stream-ordered).
+  if (cudaMemsetAsync(tp.tickets, 0, sizeof(unsigned), st) != cudaSuccess) return FA_ERR_CUDA;
   kernel<<<grid, fa::kTcThreads, fa::kTcSmemBytes, st>>>(mk, mv, mq, tp);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   return launch_combine_pdl<fa::kTcD, BF16>(cp, B, st);
@@ -511,6 +515,10 @@ FA_API int fa_debug_tc_trace(long long* host, int n) {
   if (cudaDeviceSynchronize() != cudaSuccess) return -1;
   const size_t bytes = sizeof(long long) * static_cast<size_t>(n < 8 * 1024 ? n : 8 * 1024);
   return cudaMemcpyFromSymbol(host, fa::g_fa_tc_trace, bytes) == cudaSuccess ? 0 : -1;
+}
+FA_API int fa_debug_tc_clock(long long* host) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  return cudaMemcpyFromSymbol(host, fa::g_fa_tc_clock, sizeof(long long) * 148 * 6) == cudaSuccess ? 0 : -1;
 }
 #endif
 
