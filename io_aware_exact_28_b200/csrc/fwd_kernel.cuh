@@ -438,13 +438,85 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         // registers) reads its 64-score row from TMEM twice: once for the max, once for P.
         constexpr bool kResident = (kBN == 128);
         uint32_t sr[kResident ? kBN : 32];
+        const uint64_t c2 = f2_pack(c, c);
+        // P = 2^(s*c - mref) in 32-column chunks, each stored to TMEM as 16 packed columns
+        // (P_t occupies S_t columns [0, BN/2); chunk cc only overwrites columns already
+        // read); returns the row sum of the unrounded fp32 P. With track, the row maximum
+        // of the scores is gathered in mx8 on the way. In tiles without masked scores, the
+        // pairs selected by kEmuPairs use the FMA-pipe polynomial instead of MUFU.EX2.
+        auto p_pass = [&](float mref, bool track) -> float {
+          const uint64_t nm2 = f2_pack(-mref, -mref);
+          uint64_t l2a = f2_pack(0.f, 0.f), l2b = l2a;
+#pragma unroll
+          for (int cc = 0; cc < kBN / 32; ++cc) {
+            if constexpr (!kResident) {
+              tmem_ld32x32b_x32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+              mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]), cc);
+            }
+            const uint32_t* v = kResident ? &sr[32 * cc] : &sr[0];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {               // 8 packed columns per store
+              uint32_t pk[8];
+#pragma unroll
+              for (int ii = 0; ii < 8; ++ii) {
+                const int i = 8 * hh + ii;
+                if (track)
+                  mx8[i & 7] = fmax3(mx8[i & 7], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                const uint64_t x2 =
+                    f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2);
+                uint64_t p2;
+                if (!masked_tile && ((FwdCfg<D>::kEmuPairs >> (i & 7)) & 1u)) {
+                  p2 = exp2_poly_f2(x2);
+                } else {
+                  float x0, x1;
+                  f2_unpack(x2, x0, x1);
+                  p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+                }
+                if (i & 1) l2b = f2_add(l2b, p2); else l2a = f2_add(l2a, p2);
+                float p0, p1;
+                f2_unpack(p2, p0, p1);
+                pk[ii] = pack_half2(p0, p1, BF16);
+              }
+              tmem_st32x32b_x8(tS + cc * 16 + hh * 8, pk);
+            }
+          }
+          float la, lb, lc, ld;
+          f2_unpack(l2a, la, lb);
+          f2_unpack(l2b, lc, ld);
+          return (la + lb) + (lc + ld);
+        };
+        // Raise m only when the tile max exceeds it by more than 8 (scale > 0: -inf stays
+        // -inf). Rows that already hold earlier tiles rescale O_t and l. The TMEM rescale
+        // is warp-collective: the warp runs it if any row needs it, with factor 1 elsewhere.
+        auto raise_max = [&]() -> bool {
+          const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                 fmaxf(mx8[6], mx8[7])) * c;
+          const bool grow = mx > m_used + 8.0f;
+          const bool rescale = grow && m_used != -CUDART_INF_F;
+          if (__any_sync(0xffffffffu, rescale)) {
+            const float alpha = rescale ? ex2_approx(m_used - mx) : 1.0f;
+            l *= alpha;
+            rescale_o_row<D>(tO, alpha);
+          }
+          if (grow) m_used = mx;
+          return __any_sync(0xffffffffu, grow);
+        };
         if constexpr (kResident) {
           tmem_ld32x32b_x128(tS, sr);
 #pragma unroll
-          for (int cc = 0; cc < kBN / 32; ++cc) {
-            uint32_t (&v)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]);
-            mask_chunk(v, cc);
-            max_chunk(v);
+          for (int cc = 0; cc < kBN / 32; ++cc) mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]), cc);
+          if (__all_sync(0xffffffffu, m_used != -CUDART_INF_F)) {
+            // Every row already has a running max: compute P against it while gathering the
+            // tile max; only if some row's max grew past the lazy threshold (rare after the
+            // first tiles) is P recomputed, from the scores still in registers.
+            float lsum = p_pass(m_used, true);
+            if (raise_max()) lsum = p_pass(m_used, false);
+            l += lsum;
+          } else {
+#pragma unroll
+            for (int cc = 0; cc < kBN / 32; ++cc) max_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]));
+            raise_max();
+            l += p_pass((m_used == -CUDART_INF_F) ? 0.f : m_used, false);
           }
         } else {
 #pragma unroll
@@ -453,61 +525,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]), cc);
             max_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
           }
-        }
-        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                               fmaxf(mx8[6], mx8[7])) * c;
-        // Raise m only when the tile max exceeds it by more than 8 (scale > 0: -inf stays
-        // -inf). Rows that already hold earlier tiles rescale O_t and l. The TMEM rescale
-        // is warp-collective: the warp runs it if any row needs it, with factor 1 elsewhere.
-        const bool grow = mx > m_used + 8.0f;
-        const bool rescale = grow && m_used != -CUDART_INF_F;
-        if (__any_sync(0xffffffffu, rescale)) {
-          const float alpha = rescale ? ex2_approx(m_used - mx) : 1.0f;
-          l *= alpha;
-          rescale_o_row<D>(tO, alpha);
-        }
-        if (grow) m_used = mx;
-        const float mref = (m_used == -CUDART_INF_F) ? 0.f : m_used;
-        // P = 2^(s*c - m) in 32-column chunks, each stored to TMEM as 16 packed columns
-        // (P_t occupies S_t columns [0, BN/2); chunk cc only overwrites columns already read).
-        // In tiles without masked scores, the pairs selected by kEmuPairs are evaluated
-        // with the FMA-pipe polynomial instead of MUFU.EX2. The argument s*c - m and the
-        // row sum use packed f32x2 arithmetic.
-        const uint64_t c2 = f2_pack(c, c);
-        const uint64_t nm2 = f2_pack(-mref, -mref);
-        uint64_t l2a = f2_pack(0.f, 0.f), l2b = l2a;
-#pragma unroll
-        for (int cc = 0; cc < kBN / 32; ++cc) {
-          if constexpr (!kResident) {
-            tmem_ld32x32b_x32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]), cc);
-          }
-          const uint32_t* v = kResident ? &sr[32 * cc] : &sr[0];
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint64_t x2 =
-                f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2);
-            uint64_t p2;
-            if (!masked_tile && ((FwdCfg<D>::kEmuPairs >> (i & 7)) & 1u)) {
-              p2 = exp2_poly_f2(x2);
-            } else {
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
-            }
-            if (i & 1) l2b = f2_add(l2b, p2); else l2a = f2_add(l2a, p2);
-            float p0, p1;
-            f2_unpack(p2, p0, p1);
-            pk[i] = pack_half2(p0, p1, BF16);
-          }
-          tmem_st32x32b_x16(tS + cc * 16, pk);
-        }
-        {
-          float la, lb, lc, ld;
-          f2_unpack(l2a, la, lb);
-          f2_unpack(l2b, lc, ld);
-          l += (la + lb) + (lc + ld);
+          raise_max();
+          l += p_pass((m_used == -CUDART_INF_F) ? 0.f : m_used, false);
         }
         tmem_st_wait();
         tc_fence_before();

@@ -381,6 +381,13 @@ __device__ __forceinline__ void tmem_ld32x32b_x128(uint32_t taddr, uint32_t (&r)
       : "r"(taddr) : "memory");
 }
 
+// Store N=8 consecutive 32-bit TMEM columns of this thread's lane (asynchronous; see tmem_st_wait).
+__device__ __forceinline__ void tmem_st32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n"
+      :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]) : "memory");
+}
+
 // Store N=16 consecutive 32-bit TMEM columns of this thread's lane (asynchronous; see tmem_st_wait).
 __device__ __forceinline__ void tmem_st32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
