@@ -57,6 +57,23 @@ def test_groupings_and_dims(Hq, Hkv, d, dtype):
     check(3, Hq, Hkv, 700, d, dtype, [700, 333, 1], seed=Hq + Hkv + d)
 
 
+@pytest.mark.parametrize("d,dtype", [(64, "fp16"), (128, "bf16"), (128, "fp16")])
+def test_growing_scores_force_rescales(d, dtype):
+    """Scores that grow along the cache by about 10 (log2 units) per 64 tokens: every tile
+    of every split raises the running maximum past the lazy-rescale threshold."""
+    B, Hq, Hkv, cache = 4, 8, 2, 4096
+    lens = [700, 2047, 3000, 4096]
+    kv_lens, q, kc, vc = make_decode_inputs(B, Hq, Hkv, cache, d, dtype, 1, cache, seed=d,
+                                            kv_lens=torch.tensor(lens))
+    scale = 1.0 / math.sqrt(d)
+    alpha = 10.0 / 64.0 / (scale * math.log2(math.e))
+    q[..., 0] = 1.0
+    kc[..., 0] = (torch.arange(cache, dtype=torch.float64) * alpha).to(kc.dtype)
+    o, lse = run_decode(kv_lens, q, kc, vc, scale)
+    O, L = decode_f64(q, kc, vc, kv_lens, scale)
+    assert_close(o, lse, O, L, dtype, f"decode growing scores d{d} {dtype}", strict=False)
+
+
 def test_poisoned_cache_rows_beyond_length():
     """NaN in cache rows >= kv_len must never be read."""
     B, Hq, Hkv, cache, d = 4, 16, 4, 2048, 128

@@ -51,6 +51,25 @@ def test_shapes_ragged(d, dtype, causal, N):
     check_full(1, 2, 1, N, N, d, dtype, causal, seed=N + d)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_growing_scores_force_rescales(d, dtype, causal):
+    """Scores that grow along the key axis by about 10 (log2 units) per 64 keys: the row
+    maximum exceeds the lazy-rescale threshold on nearly every key tile, so the rescale of
+    O and l, and at d = 128 the recomputation of P against the new maximum, run on almost
+    every tile instead of almost never."""
+    B, Hq, Hkv, N = 1, 2, 1, 640
+    q, k, v = make_fwd_inputs(B, Hq, Hkv, N, N, d, dtype, seed=d + N)
+    scale = 1.0 / math.sqrt(d)
+    alpha = 10.0 / 64.0 / (scale * math.log2(math.e))
+    q[..., 0] = 1.0
+    k[..., 0] = (torch.arange(N, dtype=torch.float64) * alpha).to(k.dtype)
+    o, lse = run_fwd(q, k, v, causal, scale)
+    O, L = attention_f64(q, k, v, causal, scale)
+    assert_close(o, lse, O, L, dtype, f"growing scores d{d} {dtype} c{causal}", strict=False)
+
+
 @pytest.mark.parametrize("Nq,Nk", [(128, 640), (77, 300), (300, 77), (1, 513), (256, 129),
                                    (512, 1024)])
 @pytest.mark.parametrize("causal", [False, True])
