@@ -30,6 +30,9 @@ from workloads import WORKLOADS, decode_kv_bytes, fwd_flops, make_decode_inputs,
 METRIC = "attn fwd TFLOP/s & % BF16 TC peak; decode KV-read GB/s & % HBM peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
+# ex2.approx.f32 results per clock per SM, measured on this machine's B200s with a throughput
+# probe (independent chains, 4-32 warps per SM); f16x2/bf16x2 forms give the same rate.
+MUFU_EX2_PER_CLK_SM = 16.0
 
 
 def measured_traffic(kernel: str, workload: str):
@@ -298,6 +301,20 @@ def run_ours(args):
                 "traffic_note": f"{dec_kernel} only (the combine kernel moves ~2% more)",
                 "peak_source": f"{peak_src} HBM copy bandwidth",
                 "algorithmic_bytes_per_launch": dec_bytes, "kv_bytes_per_launch": kv_bytes}
+    # The forward's other bound: one exponential (MUFU ex2) per visible score, against the
+    # measured 16.0 per clock per SM of this machine's B200s at the SM clock sampled during
+    # the timed region.
+    clocks = sampler.summary()
+    sm_mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz")
+    if sm_mhz:
+        n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+        exps = fl / (4.0 * w.d)
+        peak_exps = MUFU_EX2_PER_CLK_SM * n_sm * sm_mhz * 1e6
+        roof_fwd["exp_unit"] = {"bound": "alu", "unit": "exp2/s", "achieved": exps / fwd_avg_s,
+                                "peak": peak_exps, "frac": exps / fwd_avg_s / peak_exps,
+                                "exps_per_launch": exps,
+                                "peak_source": f"measured {MUFU_EX2_PER_CLK_SM} ex2.approx/clk/SM x "
+                                               f"{n_sm} SMs x sampled {sm_mhz} MHz"}
     dominant = roof_fwd if fwd_ms >= dec_ms else roof_dec
 
     # End to end through the public API: host (pinned) inputs in, host outputs back, every
@@ -388,7 +405,7 @@ def run_ours(args):
             "e2e": e2e, "cpu_baseline": cpu,
             "gpu_launches": K * 3,
             "gpu_launches_note": f"per step: fa_fwd_kernel + {dec_kernel} + fa_decode_combine_kernel",
-            "clocks": sampler.summary(),
+            "clocks": clocks,
             "device_status": fa.status_string(status),
         }
         print(json.dumps(line), flush=True)
