@@ -127,6 +127,21 @@ __device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
   tmem_st_wait();
 }
 
+// Multiply 16 TMEM columns of packed 16-bit P pairs (32 values of this row) by alpha.
+template <bool BF16>
+__device__ __forceinline__ void rescale_p_cols(uint32_t taddr, float alpha) {
+  uint32_t v[16];
+  tmem_ld32x32b_x16(taddr, v);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float lo, hi;
+    unpack_half2(v[i], lo, hi, BF16);
+    v[i] = pack_half2(lo * alpha, hi * alpha, BF16);
+  }
+  tmem_st32x32b_x16(taddr, v);
+  tmem_st_wait();
+}
+
 template <int D, bool BF16, bool CAUSAL>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::CTAS)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -444,46 +459,54 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         // read); returns the row sum of the unrounded fp32 P. With track, the row maximum
         // of the scores is gathered in mx8 on the way. In tiles without masked scores, the
         // pairs selected by kEmuPairs use the FMA-pipe polynomial instead of MUFU.EX2.
-        auto p_pass = [&](float mref, bool track) -> float {
+        // P of one 32-column chunk v (scores of keys 32 cc ..) against mref, stored as 16
+        // packed columns at tS + 16 cc; returns its row sum (unrounded fp32 P). With track,
+        // the scores' maximum is gathered in mx8 on the way.
+        auto chunk_p = [&](const uint32_t* v, int cc, float mref, bool track) -> float {
           const uint64_t nm2 = f2_pack(-mref, -mref);
           uint64_t l2a = f2_pack(0.f, 0.f), l2b = l2a;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {               // 8 packed columns per store
+            uint32_t pk[8];
+#pragma unroll
+            for (int ii = 0; ii < 8; ++ii) {
+              const int i = 8 * hh + ii;
+              if (track)
+                mx8[i & 7] = fmax3(mx8[i & 7], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              const uint64_t x2 =
+                  f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2);
+              uint64_t p2;
+              if (!masked_tile && ((FwdCfg<D>::kEmuPairs >> (i & 7)) & 1u)) {
+                p2 = exp2_poly_f2(x2);
+              } else {
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+                p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+              }
+              if (i & 1) l2b = f2_add(l2b, p2); else l2a = f2_add(l2a, p2);
+              float p0, p1;
+              f2_unpack(p2, p0, p1);
+              pk[ii] = pack_half2(p0, p1, BF16);
+            }
+            tmem_st32x32b_x8(tS + cc * 16 + hh * 8, pk);
+          }
+          float la, lb, lc, ld;
+          f2_unpack(l2a, la, lb);
+          f2_unpack(l2b, lc, ld);
+          return (la + lb) + (lc + ld);
+        };
+        // P of the whole row (all chunks; d = 64 loads each chunk from TMEM here).
+        auto p_pass = [&](float mref, bool track) -> float {
+          float sum = 0.f;
 #pragma unroll
           for (int cc = 0; cc < kBN / 32; ++cc) {
             if constexpr (!kResident) {
               tmem_ld32x32b_x32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
               mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]), cc);
             }
-            const uint32_t* v = kResident ? &sr[32 * cc] : &sr[0];
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {               // 8 packed columns per store
-              uint32_t pk[8];
-#pragma unroll
-              for (int ii = 0; ii < 8; ++ii) {
-                const int i = 8 * hh + ii;
-                if (track)
-                  mx8[i & 7] = fmax3(mx8[i & 7], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-                const uint64_t x2 =
-                    f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2);
-                uint64_t p2;
-                if (!masked_tile && ((FwdCfg<D>::kEmuPairs >> (i & 7)) & 1u)) {
-                  p2 = exp2_poly_f2(x2);
-                } else {
-                  float x0, x1;
-                  f2_unpack(x2, x0, x1);
-                  p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
-                }
-                if (i & 1) l2b = f2_add(l2b, p2); else l2a = f2_add(l2a, p2);
-                float p0, p1;
-                f2_unpack(p2, p0, p1);
-                pk[ii] = pack_half2(p0, p1, BF16);
-              }
-              tmem_st32x32b_x8(tS + cc * 16 + hh * 8, pk);
-            }
+            sum += chunk_p(kResident ? &sr[32 * cc] : &sr[0], cc, mref, track);
           }
-          float la, lb, lc, ld;
-          f2_unpack(l2a, la, lb);
-          f2_unpack(l2b, lc, ld);
-          return (la + lb) + (lc + ld);
+          return sum;
         };
         // Raise m only when the tile max exceeds it by more than 8 (scale > 0: -inf stays
         // -inf). Rows that already hold earlier tiles rescale O_t and l. The TMEM rescale
@@ -519,14 +542,42 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             l += p_pass((m_used == -CUDART_INF_F) ? 0.f : m_used, false);
           }
         } else {
+          // d = 64: one TMEM load per 32-column chunk. The chunk's max comes from registers;
+          // a row whose max grows past the lazy threshold (every row on its first tile,
+          // rarely later) raises m, and rows that already hold P (earlier tiles in O and l,
+          // earlier chunks in TMEM) rescale them; then P of the chunk is computed and stored.
+          uint32_t (&v)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+          float lsum = 0.f;
 #pragma unroll
           for (int cc = 0; cc < kBN / 32; ++cc) {
-            tmem_ld32x32b_x32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]), cc);
-            max_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32x32b_x32(tS + 32 * cc, v);
+            mask_chunk(v, cc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx8[i] = -CUDART_INF_F;
+            max_chunk(v);
+            const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                   fmaxf(mx8[6], mx8[7])) * c;
+            const bool grow = mx > m_used + 8.0f;
+            const bool rescale = grow && m_used != -CUDART_INF_F;
+            if (__any_sync(0xffffffffu, rescale)) {
+              const float alpha = rescale ? ex2_approx(m_used - mx) : 1.0f;
+              l *= alpha;
+              lsum *= alpha;
+              rescale_o_row<D>(tO, alpha);
+              if (cc > 0) {
+                tmem_st_wait();                            // stored P chunks, read back below
+#pragma unroll
+                for (int c0 = 0; c0 < cc; ++c0) rescale_p_cols<BF16>(tS + 16 * c0, alpha);
+              }
+              // Reload the chunk (its columns are untouched: P goes below 16 cc) instead of
+              // keeping 32 scores live across the rescale.
+              tmem_ld32x32b_x32(tS + 32 * cc, v);
+              mask_chunk(v, cc);
+            }
+            if (grow) m_used = mx;
+            lsum += chunk_p(v, cc, (m_used == -CUDART_INF_F) ? 0.f : m_used, false);
           }
-          raise_max();
-          l += p_pass((m_used == -CUDART_INF_F) ? 0.f : m_used, false);
+          l += lsum;
         }
         tmem_st_wait();
         tc_fence_before();

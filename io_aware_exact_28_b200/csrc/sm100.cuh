@@ -30,6 +30,17 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// The two 16-bit values of a packed pair (low half first) as fp32.
+__device__ __forceinline__ void unpack_half2(uint32_t v, float& lo, float& hi, bool bf16) {
+  if (bf16) {
+    lo = __uint_as_float(v << 16);
+    hi = __uint_as_float(v & 0xFFFF0000u);
+  } else {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+        : "=f"(lo), "=f"(hi) : "r"(v));
+  }
+}
+
 // max(a, b, c) in one instruction (three-operand form of max.f32, sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
