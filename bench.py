@@ -431,6 +431,22 @@ def run_single_kernel(args):
 
         def call():
             fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+    elif args.only == "chunked":
+        # Chunked prefill: the workload's sequence in --chunk-token pieces, each attending
+        # to the cache prefix up to its own end (fa_fwd_kvcache); same causal FLOPs.
+        w = WORKLOADS[args.workload]
+        q, k, v = (t.to(dev) for t in make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed))
+        o, lse = torch.empty_like(q), torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+        work = fwd_flops(w.B, w.Hq, w.N, w.N, w.d, True) / 1e12
+        unit = "TFLOP/s"
+        C = args.chunk
+        qs = [q[:, :, i:i + C].contiguous() for i in range(0, w.N, C)]
+        outs = [torch.empty_like(x) for x in qs]
+
+        def call():
+            for n, i in enumerate(range(0, w.N, C)):
+                fa.fwd_kvcache(qs[n], k, v, min(i + C, w.N), causal=True, scale=w.scale, out=outs[n],
+                               return_lse=False)
     else:
         w = WORKLOADS[args.decode_workload]
         kv_cpu, dq, kc, vc = make_decode_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.dtype, w.kv_len_lo,
@@ -459,20 +475,22 @@ def run_single_kernel(args):
         ms.append(e0.elapsed_time(e1))
     status = fa.status_string(fa.device_status())
     avg = sum(ms) / len(ms)
-    print(json.dumps({"only": args.only, "workload": w.describe(), "ms_per_launch": avg,
+    print(json.dumps({"only": args.only, "workload": w.describe(),
+                      **({"chunk": args.chunk} if args.only == "chunked" else {}), "ms_per_launch": avg,
                       "value": work / (avg * 1e-3), "unit": unit, "device_status": status}))
     return 0 if status == "FA_OK" else 1
 
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("--only", choices=["fwd", "decode"], default=None,
+    ap.add_argument("--only", choices=["fwd", "decode", "chunked"], default=None,
                     help="launch one entry point alone (profiling helper; prints its own line)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mha2k", choices=[k for k, v in WORKLOADS.items() if v.kind == "fwd"])
+    ap.add_argument("--chunk", type=int, default=1024, help="--only chunked: tokens per chunk")
     ap.add_argument("--decode-workload", default="decode")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

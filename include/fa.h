@@ -79,6 +79,27 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
                  int causal, float scale, fa_dtype dtype, void* stream);
 
 /*
+ * fa_fwd_kvcache — fa_fwd for a chunk of queries against the first Nk rows of a KV cache
+ * whose capacity per head is cache_len >= Nk (chunked prefill: the newest Nq tokens
+ * attend to the whole prefix, causally aligned to its end).
+ *
+ * Defined by: page "Flash Attention ... IO-aware exact" (fr), "Erreurs courantes et
+ * solutions" (the manual chunking example: a chunk of queries attends to every key up to
+ * the chunk's end) and "Optimisation avancée : KV Cache" (keys and values kept in a cache
+ * across calls); the result is fa_fwd's with k, v = the caches' first Nk rows.
+ *
+ *   q, o, lse           as fa_fwd, [B, Hq, Nq, d] / [B, Hq, Nq]
+ *   kcache, vcache      [B, Hkv, cache_len, d]; rows [0, Nk) of each head are used, rows
+ *                       [Nk, cache_len) are never read
+ *   causal              0 or 1; with Nq <= Nk the chunk is the cache's last Nq tokens
+ *
+ * Requirements: those of fa_fwd, plus 1 <= Nk <= cache_len. Same errors and ownership.
+ */
+FA_API fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* vcache, void* o,
+                         float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int cache_len,
+                         int d, int causal, float scale, fa_dtype dtype, void* stream);
+
+/*
  * fa_decode_workspace_bytes — bytes of scratch that fa_decode needs for these sizes.
  *
  * The split-KV decode writes, per (sequence, query head, KV split), a partial output

@@ -24,7 +24,7 @@ __all__ = ["FAError", "FALibraryError", "LIB_PATH", "lib", "fwd", "decode",
            "debug_skip_q_load", "build_info", "status_string", "EXPORTED_SYMBOLS",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_ALIGNMENT",
            "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_FP16", "FA_BF16",
-           "decode_noalloc", "DECODE_NOALLOC_SCRATCH_BYTES"]
+           "decode_noalloc", "DECODE_NOALLOC_SCRATCH_BYTES", "fwd_kvcache"]
 
 # FA_B200_LIB may name another build of the same library (e.g. a variant for timing).
 LIB_PATH = os.environ.get("FA_B200_LIB") or \
@@ -36,7 +36,7 @@ FA_FP16, FA_BF16 = 0, 1
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode", "fa_decode_workspace_bytes", "fa_status_string",
                     "fa_device_status", "fa_set_wait_timeout_ns", "fa_debug_skip_q_load",
-                    "fa_build_info", "fa_decode_noalloc")
+                    "fa_build_info", "fa_decode_noalloc", "fa_fwd_kvcache")
 
 # Size of the library's fixed decode scratch (FA_DECODE_NOALLOC_SCRATCH_BYTES in fa.h).
 DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p] + [c_int] * 7 + \
             [c_float, c_int, c_void_p]
         L.fa_fwd.restype = c_int
+        L.fa_fwd_kvcache.argtypes = [c_void_p] * 5 + [c_int] * 8 + [c_float, c_int, c_void_p]
+        L.fa_fwd_kvcache.restype = c_int
         L.fa_decode.argtypes = [c_void_p] * 6 + [c_int] * 5 + [c_float, c_int, c_void_p, c_size_t,
                                                                  c_void_p]
         L.fa_decode.restype = c_int
@@ -177,6 +179,41 @@ def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, 
                       _stream_ptr(stream))
     if st != FA_OK:
         raise FAError(st, "fa_fwd")
+    return out, lse
+
+
+def fwd_kvcache(q, kcache, vcache, nk: int, causal: bool = True, scale: Optional[float] = None,
+                out=None, lse=None, return_lse: bool = True, stream=None):
+    """Chunked prefill via ``fa_fwd_kvcache``: q [B,Hq,Nq,d] against the first ``nk`` rows of
+    kcache, vcache [B,Hkv,cache_len,d] (causal: the chunk is the prefix's last Nq tokens).
+    Returns (o [B,Hq,Nq,d], lse [B,Hq,Nq] fp32 or None).
+    """
+    import torch
+    _check(q, "q", 4, q.device)
+    _check(kcache, "kcache", 4, q.device)
+    _check(vcache, "vcache", 4, q.device)
+    if kcache.dtype != q.dtype or vcache.dtype != q.dtype:
+        raise TypeError("q, kcache, vcache must share one dtype")
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, cache_len, dk = kcache.shape
+    if tuple(vcache.shape) != tuple(kcache.shape) or Bk != B or dk != d:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} kcache{tuple(kcache.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check(out, "out", 4, q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _check(lse, "lse", 3, q.device)
+    st = lib().fa_fwd_kvcache(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), out.data_ptr(),
+                              lse.data_ptr() if lse is not None else None,
+                              B, Hq, Hkv, Nq, int(nk), cache_len, d, 1 if causal else 0,
+                              float(scale), _dtype_code(q), _stream_ptr(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_kvcache")
     return out, lse
 
 

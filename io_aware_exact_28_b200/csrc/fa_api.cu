@@ -71,14 +71,16 @@ EncodeTiledFn encode_fn() {
 
 // [heads, rows, d] 16-bit tensor, box = 64 columns (128 bytes) x box_rows rows x 1 head,
 // 128-byte swizzle; rows past `rows` read as zero and are clipped on store.
+// [heads, rows, d] 16-bit view; a head's rows start head_rows rows apart in memory
+// (head_rows >= rows; 0 = rows). Rows past `rows` read as zero.
 bool make_tile_map(CUtensorMap* m, const void* ptr, int d, int rows, long long heads, bool bf16,
-                   int box_rows) {
+                   int box_rows, long long head_rows = 0) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(heads)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                                 static_cast<cuuint64_t>(rows) * d * 2};
+                                 static_cast<cuuint64_t>(head_rows > 0 ? head_rows : rows) * d * 2};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
@@ -314,13 +316,10 @@ fa_status common_checks(int B, int Hq, int Hkv, int d, float scale, int dtype) {
   return FA_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                 int Hkv, int Nq, int Nk, int d, int causal, float scale, fa_dtype dtype,
-                 void* stream) {
+// fa_fwd and fa_fwd_kvcache: K/V heads hold kv_rows rows in memory, of which Nk are used.
+fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                   int Hkv, int Nq, int Nk, long long kv_rows, int d, int causal, float scale,
+                   fa_dtype dtype, void* stream) {
   if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
   if (Nq <= 0 || Nk <= 0 || (causal != 0 && causal != 1)) return FA_ERR_INVALID_ARG;
   fa_status s = common_checks(B, Hq, Hkv, d, scale, dtype);
@@ -340,8 +339,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   CUtensorMap mq, mk, mv;
   const int kv_box = (d == 64) ? fa::FwdCfg<64>::BN : fa::FwdCfg<128>::BN;
   if (!make_tile_map(&mq, q, d, Nq, BH, bf16, fa::kBM) ||
-      !make_tile_map(&mk, k, d, Nk, BHkv, bf16, kv_box) ||
-      !make_tile_map(&mv, v, d, Nk, BHkv, bf16, kv_box))
+      !make_tile_map(&mk, k, d, Nk, BHkv, bf16, kv_box, kv_rows) ||
+      !make_tile_map(&mv, v, d, Nk, BHkv, bf16, kv_box, kv_rows))
     return FA_ERR_CUDA;
 
   fa::FwdParams prm;
@@ -364,6 +363,23 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                 : dispatch_causal<64, false>(causal, dev, mq, mk, mv, prm, st);
   return bf16 ? dispatch_causal<128, true>(causal, dev, mq, mk, mv, prm, st)
               : dispatch_causal<128, false>(causal, dev, mq, mk, mv, prm, st);
+}
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                 int Hkv, int Nq, int Nk, int d, int causal, float scale, fa_dtype dtype,
+                 void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, Nk, d, causal, scale, dtype, stream);
+}
+
+fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* vcache, void* o,
+                         float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int cache_len,
+                         int d, int causal, float scale, fa_dtype dtype, void* stream) {
+  if (cache_len < Nk || cache_len <= 0) return FA_ERR_INVALID_ARG;
+  return fwd_impl(q, kcache, vcache, o, lse, B, Hq, Hkv, Nq, Nk, cache_len, d, causal, scale,
+                  dtype, stream);
 }
 
 size_t fa_decode_workspace_bytes(int B, int Hq, int max_kv_len, int d) {

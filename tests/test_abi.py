@@ -60,6 +60,24 @@ def test_fwd_rejects_bad_arguments_without_cuda():
     assert _fwd(L, lse=18) == fa.FA_ERR_ALIGNMENT
 
 
+def test_fwd_kvcache_rejects_bad_arguments_without_cuda():
+    L = fa.lib()
+
+    def call(Nk=128, cache_len=256, **kw):
+        a = dict(q=16, k=16, v=16, o=16, lse=None, B=1, Hq=2, Hkv=1, Nq=64, d=64, causal=1,
+                 scale=0.125, dtype=0)
+        a.update(kw)
+        return L.fa_fwd_kvcache(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"],
+                                a["Hkv"], a["Nq"], Nk, cache_len, a["d"], a["causal"], a["scale"],
+                                a["dtype"], None)
+    assert call(Nk=257, cache_len=256) == fa.FA_ERR_INVALID_ARG    # prefix longer than the cache
+    assert call(cache_len=0) == fa.FA_ERR_INVALID_ARG
+    assert call(Nk=0) == fa.FA_ERR_INVALID_ARG
+    assert call(q=None) == fa.FA_ERR_INVALID_ARG
+    assert call(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert call(k=24) == fa.FA_ERR_ALIGNMENT
+
+
 def test_decode_rejects_bad_arguments_without_cuda():
     L = fa.lib()
     need = fa.decode_workspace_bytes(2, 8, 4096, 128)
