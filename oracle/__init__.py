@@ -4,7 +4,8 @@ TEST INFRASTRUCTURE ONLY: imported by `tests/`, `__graft_entry__.smoke()` and th
 CPU-baseline leg of `bench.py`, never by the CUDA library or its Python binding.
 """
 from .attention import attention_f64, attention_rows_f64, decode_f64, visible_mask
+from .backward import attention_bwd_f64
 from .tiled import tiled_attention_f64
 
 __all__ = ["attention_f64", "attention_rows_f64", "decode_f64", "visible_mask",
-           "tiled_attention_f64"]
+           "tiled_attention_f64", "attention_bwd_f64"]
