@@ -100,6 +100,38 @@ FA_API fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* v
                          int d, int causal, float scale, fa_dtype dtype, void* stream);
 
 /*
+ * fa_bwd_workspace_bytes — bytes of scratch that fa_bwd needs for these sizes.
+ */
+FA_API size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq);
+
+/*
+ * fa_bwd — gradients of fa_fwd: dQ, dK, dV for an upstream gradient dO, recomputing the
+ * scores tile by tile from Q, K and the forward's LSE (no N x N matrix is stored).
+ *
+ * Defined by: the derivative of fa_fwd's result (page "Kotaemon FlashAttention",
+ * attention formula); the recomputation from the saved per-row statistic follows page
+ * "Flash Attention" (zh), "IO 感知的算法设计" (tiling plus recomputation) and the L output of
+ * page "Flash Attention ... IO-aware exact" (fr), tiling pseudo-code.
+ *
+ *   q, o, dout    [B, Hq,  Nq, d]  fp16/bf16; o and lse are fa_fwd's outputs for q, k, v
+ *   k, v          [B, Hkv, Nk, d]
+ *   lse           [B, Hq,  Nq]     fp32 (natural log, as fa_fwd writes it)
+ *   dq            [B, Hq,  Nq, d]  written
+ *   dk, dv        [B, Hkv, Nk, d]  written; a KV head sums the gradients of all query heads
+ *                                  that read it
+ *   causal, scale as passed to fa_fwd
+ *   workspace     device scratch of at least fa_bwd_workspace_bytes(B, Hq, Nq) bytes,
+ *                 16-byte aligned, owned by the caller, no initialisation needed
+ *
+ * Requirements: those of fa_fwd, plus every listed pointer non-NULL (lse included) and
+ * 16-byte aligned (lse 4-byte), workspace_bytes large enough (FA_ERR_WORKSPACE).
+ */
+FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
+                 const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                 int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                 fa_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fa_decode_workspace_bytes — bytes of scratch that fa_decode needs for these sizes.
  *
  * The split-KV decode writes, per (sequence, query head, KV split), a partial output

@@ -24,7 +24,8 @@ __all__ = ["FAError", "FALibraryError", "LIB_PATH", "lib", "fwd", "decode",
            "debug_skip_q_load", "build_info", "status_string", "EXPORTED_SYMBOLS",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_ALIGNMENT",
            "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_FP16", "FA_BF16",
-           "decode_noalloc", "DECODE_NOALLOC_SCRATCH_BYTES", "fwd_kvcache"]
+           "decode_noalloc", "DECODE_NOALLOC_SCRATCH_BYTES", "fwd_kvcache", "bwd",
+           "bwd_workspace_bytes"]
 
 # FA_B200_LIB may name another build of the same library (e.g. a variant for timing).
 LIB_PATH = os.environ.get("FA_B200_LIB") or \
@@ -36,7 +37,8 @@ FA_FP16, FA_BF16 = 0, 1
 
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode", "fa_decode_workspace_bytes", "fa_status_string",
                     "fa_device_status", "fa_set_wait_timeout_ns", "fa_debug_skip_q_load",
-                    "fa_build_info", "fa_decode_noalloc", "fa_fwd_kvcache")
+                    "fa_build_info", "fa_decode_noalloc", "fa_fwd_kvcache", "fa_bwd",
+                    "fa_bwd_workspace_bytes")
 
 # Size of the library's fixed decode scratch (FA_DECODE_NOALLOC_SCRATCH_BYTES in fa.h).
 DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -75,6 +77,10 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.restype = c_int
         L.fa_fwd_kvcache.argtypes = [c_void_p] * 5 + [c_int] * 8 + [c_float, c_int, c_void_p]
         L.fa_fwd_kvcache.restype = c_int
+        L.fa_bwd.argtypes = [c_void_p] * 9 + [c_int] * 7 + [c_float, c_int, c_void_p, c_size_t, c_void_p]
+        L.fa_bwd.restype = c_int
+        L.fa_bwd_workspace_bytes.argtypes = [c_int] * 3
+        L.fa_bwd_workspace_bytes.restype = c_size_t
         L.fa_decode.argtypes = [c_void_p] * 6 + [c_int] * 5 + [c_float, c_int, c_void_p, c_size_t,
                                                                  c_void_p]
         L.fa_decode.restype = c_int
@@ -215,6 +221,45 @@ def fwd_kvcache(q, kcache, vcache, nk: int, causal: bool = True, scale: Optional
     if st != FA_OK:
         raise FAError(st, "fa_fwd_kvcache")
     return out, lse
+
+
+def bwd_workspace_bytes(B: int, Hq: int, Nq: int) -> int:
+    """Scratch bytes ``fa_bwd`` needs for these sizes."""
+    return int(lib().fa_bwd_workspace_bytes(B, Hq, Nq))
+
+
+def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: Optional[float] = None, dq=None,
+        dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of ``fwd`` via ``fa_bwd``: (dq [B,Hq,Nq,d], dk, dv [B,Hkv,Nk,d]).
+
+    o and lse are ``fwd``'s outputs for q, k, v; dout is the upstream gradient of o.
+    """
+    import torch
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _check(t, name, 4, q.device)
+    _check(lse, "lse", 3, q.device)
+    if any(t.dtype != q.dtype for t in (k, v, o, dout)):
+        raise TypeError("q, k, v, o, dout must share one dtype")
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk_ = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk_ != d or tuple(o.shape) != tuple(q.shape) \
+            or tuple(dout.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_bytes(B, Hq, Nq)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq,
+                      Nk, d, 1 if causal else 0, float(scale), _dtype_code(q), workspace.data_ptr(),
+                      workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd")
+    return dq, dk, dv
 
 
 def decode(q, kcache, vcache, kv_lens, scale: Optional[float] = None, out=None, lse=None,

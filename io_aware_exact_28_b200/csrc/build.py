@@ -14,7 +14,7 @@ PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
 OUT = os.path.join(PKG, "libfa_b200.so")
 SOURCES = [os.path.join(HERE, "fa_api.cu")]
-DEPS = SOURCES + [os.path.join(HERE, f) for f in ("sm100.cuh", "fwd_kernel.cuh", "decode_kernel.cuh", "decode_tc_kernel.cuh")] \
+DEPS = SOURCES + [os.path.join(HERE, f) for f in ("sm100.cuh", "fwd_kernel.cuh", "bwd_kernel.cuh", "decode_kernel.cuh", "decode_tc_kernel.cuh")] \
     + [os.path.join(ROOT, "include", "fa.h"), os.path.abspath(__file__)]
 
 

@@ -1,0 +1,536 @@
+// bwd_kernel.cuh — gradients of exact attention (dQ, dK, dV) for sm_100a, by recomputation.
+//
+// The backward pass keeps no score matrix either: it recomputes the scores tile by tile
+// from Q, K and the forward's per-row statistic L (page "Flash Attention" (zh), "IO 感知的
+// 算法设计", tiling plus recomputation; page "Flash Attention ... IO-aware exact" (fr), the
+// pseudo-code's second output L). With P_ij = exp(scale * q_i . k_j - L_i) recomputed and
+// D_i = sum_d dO_id O_id:
+//     dV = P^T dO      dP = dO V^T      dS = P * (dP - D)
+//     dQ = scale * dS K                  dK = scale * dS^T Q
+// Three kernels:
+//   fa_bwd_preprocess_kernel  D and L * log2(e) per query row, padded to whole 128-row
+//                             tiles; rows without a visible key and rows past Nq get
+//                             +inf, so their P is exactly 0 in both kernels below.
+//   fa_bwd_dq_kernel          one CTA per 128-row query tile: per key tile j,
+//                             S = Q K_j^T and dP = dO V_j^T (tcgen05, TMEM), then the
+//                             elementwise warps form dS and dQ += dS K_j (A = dS in TMEM).
+//   fa_bwd_dkdv_kernel        one CTA per 128-row key tile of a KV head: per query tile i
+//                             of every query head of its group, S^T = K Q_i^T and
+//                             dP^T = V dO_i^T, then P^T and dS^T, and dV += P^T dO_i,
+//                             dK += dS^T Q_i (A operands in TMEM). The group's query heads
+//                             are summed in TMEM, so no atomics are needed.
+// Causal masking is bottom-right aligned as in the forward: key j is visible to query i
+// iff j <= i + (Nk - Nq).
+#pragma once
+
+#include <cuda.h>
+#include <math_constants.h>
+
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int kBwdTile = 128;          // query rows and key rows per tile
+constexpr int kBwdThreads = 192;       // warps 0-3 elementwise, 4 producer, 5 MMA
+constexpr int kBwdWarpProd = 4;
+constexpr int kBwdWarpMma = 5;
+
+struct BwdParams {
+  const float* lse2;      // [B*Hq, Nq_pad] L * log2(e), +inf where P must be 0
+  const float* dsum;      // [B*Hq, Nq_pad] D
+  void* out;              // dq [B*Hq, Nq, D] (dQ kernel) or dk [B*Hkv, Nk, D] (dK/dV kernel)
+  void* out2;             // dv [B*Hkv, Nk, D] (dK/dV kernel)
+  int Hq, Hkv, group;
+  int Nq, Nk, Nq_pad;
+  int causal_offset;      // Nk - Nq
+  float scale, scale_log2;
+  uint64_t timeout_ns;
+};
+
+// ------------------------------------------------------------------------------------
+// D_i = sum_d dO_id O_id and L_i * log2(e), padded per head to Nq_pad rows.
+// One warp per row; d = 64 or 128.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256)
+fa_bwd_preprocess_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+                         const float* __restrict__ lse, float* __restrict__ lse2,
+                         float* __restrict__ dsum, int BH, int Nq, int Nq_pad) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= BH * Nq_pad) return;
+  const int bh = warp / Nq_pad, row = warp - bh * Nq_pad;
+  float acc = 0.f;
+  if (row < Nq) {
+    const size_t base = (static_cast<size_t>(bh) * Nq + row) * D;
+#pragma unroll
+    for (int e = lane * 2; e < D; e += 64) {
+      float o0, o1, g0, g1;
+      unpack_half2(*reinterpret_cast<const uint32_t*>(o + base + e), o0, o1, BF16);
+      unpack_half2(*reinterpret_cast<const uint32_t*>(dout + base + e), g0, g1, BF16);
+      acc = fmaf(o0, g0, fmaf(o1, g1, acc));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    const float l = row < Nq ? lse[static_cast<size_t>(bh) * Nq + row] : -CUDART_INF_F;
+    lse2[static_cast<size_t>(bh) * Nq_pad + row] =
+        (l == -CUDART_INF_F) ? CUDART_INF_F : l * 1.4426950408889634f;
+    dsum[static_cast<size_t>(bh) * Nq_pad + row] = acc;
+  }
+}
+
+template <int D>
+struct BwdCfg {
+  static constexpr int NCH = D / 64;                 // 128-byte swizzle chunks along d
+  static constexpr int CHUNK = kBwdTile * 128;       // 128 rows x 128 bytes
+  static constexpr int TILE_BYTES = kBwdTile * D * 2;
+  static constexpr int NS = (D == 64) ? 8 : 4;       // ring items (one 128-row tile each)
+  static constexpr int A_OFF = 0;                    // dQ: Q, dO;  dK/dV: K, V
+  static constexpr int RING_OFF = 2 * TILE_BYTES;
+  static constexpr int VEC_OFF = RING_OFF + NS * TILE_BYTES;   // dK/dV: L and D per ring pair
+  static constexpr int BAR_OFF = VEC_OFF + (NS / 2) * 2 * kBwdTile * 4;
+  static constexpr int NBARS = 1 + 2 * NS + 4;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;         // S 128 | dP 128 | accumulators
+  static constexpr uint32_t ACC_COL = 256;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(ACC_COL + 2 * D <= TMEM_COLS, "TMEM budget");
+};
+
+// ------------------------------------------------------------------------------------
+// dQ: CTA (query tile qt, head bh). TMEM: S [0,128) (dS packed over its first 64
+// columns), dP [128,256), dQ [256, 256+D).
+template <int D, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                 const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int b = bh / p.Hq, h = bh - b * p.Hq;
+  const int bh_kv = b * p.Hkv + h / p.group;
+  const int q0 = blockIdx.x * kBwdTile;
+  const int n_kv_total = (p.Nk + kBwdTile - 1) / kBwdTile;
+  int n_kv = n_kv_total;
+  if (CAUSAL) {
+    const int kmax = min(q0 + kBwdTile - 1, p.Nq - 1) + p.causal_offset;
+    n_kv = kmax < 0 ? 0 : min(n_kv_total, kmax / kBwdTile + 1);
+  }
+
+  const uint32_t bar0 = base + C::BAR_OFF;
+  const uint32_t bar_a = bar0;                                       // Q and dO landed
+  auto bar_full = [&](int i) { return bar0 + 8u * (1 + i); };
+  auto bar_empty = [&](int i) { return bar0 + 8u * (1 + C::NS + i); };
+  const uint32_t bar_s = bar0 + 8u * (1 + 2 * C::NS);                // S and dP ready
+  const uint32_t bar_ds = bar0 + 8u * (2 + 2 * C::NS);               // dS in TMEM (128)
+  const uint32_t bar_done = bar0 + 8u * (3 + 2 * C::NS);             // every MMA done
+  const uint32_t bar_drain = bar0 + 8u * (4 + 2 * C::NS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + C::MISC_OFF + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_a, 1);
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(bar_full(i), 1);
+      mbar_init(bar_empty(i), 1);
+    }
+    mbar_init(bar_s, 1);
+    mbar_init(bar_ds, kBwdTile);
+    mbar_init(bar_done, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == kBwdWarpMma) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{abort_flag, &g_fa_status, p.timeout_ns};
+
+  if (warp == kBwdWarpProd) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_kv > 0) {
+      mbar_arrive_expect_tx(bar_a, 2 * C::TILE_BYTES);
+      for (int ch = 0; ch < C::NCH; ++ch) {
+        tma_load_3d(base + C::A_OFF + ch * C::CHUNK, &tmQ, bar_a, ch * 64, q0, bh);
+        tma_load_3d(base + C::A_OFF + C::TILE_BYTES + ch * C::CHUNK, &tmDO, bar_a, ch * 64, q0, bh);
+      }
+      int it = 0;
+      bool ok = true;
+      for (int j = 0; j < n_kv && ok; ++j) {
+        for (int kv = 0; kv < 2; ++kv) {                // K_j, then V_j
+          const int slot = it % C::NS, round = it / C::NS;
+          if (round > 0 && !mbar_wait(bar_empty(slot), (round - 1) & 1, wc)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar_full(slot), C::TILE_BYTES);
+          for (int ch = 0; ch < C::NCH; ++ch)
+            tma_load_3d(base + C::RING_OFF + slot * C::TILE_BYTES + ch * C::CHUNK, kv ? &tmV : &tmK,
+                        bar_full(slot), ch * 64, j * kBwdTile, bh_kv);
+          ++it;
+        }
+      }
+      if (!ok || *abort_flag) {
+        for (int i = max(0, it - C::NS); i < it; ++i)
+          mbar_wait_drain(bar_full(i % C::NS), (i / C::NS) & 1, kDrainNs);
+        mbar_wait_drain(bar_a, 0, kDrainNs);
+      }
+    }
+  } else if (warp == kBwdWarpMma) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_kv > 0) {
+      constexpr uint32_t IDESC_S = idesc_f16(kBwdTile, kBwdTile, BF16 ? 1u : 0u, 0u, 0u);
+      constexpr uint32_t IDESC_Q = idesc_f16(kBwdTile, D, BF16 ? 1u : 0u, 0u, 1u);
+      // X[cols col, +128) = A[128 x D] B[128 x D]^T, both K-major (d contiguous).
+      auto issue_abt = [&](uint32_t col, uint32_t a, uint32_t bt) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;
+          mma_f16_ss(tmem + col, sdesc_k_sw128(a + (kk >> 2) * C::CHUNK + koff),
+                     sdesc_k_sw128(bt + (kk >> 2) * C::CHUNK + koff), IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar_a, 0, wc);
+      bool issued = false;
+      tc_fence_after();
+      const uint32_t qa = base + C::A_OFF, doa = base + C::A_OFF + C::TILE_BYTES;
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int kit = 2 * j, kslot = kit % C::NS, vit = kit + 1, vslot = vit % C::NS;
+        if (!mbar_wait(bar_full(kslot), (kit / C::NS) & 1, wc)) { ok = false; break; }
+        if (!mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ka = base + C::RING_OFF + kslot * C::TILE_BYTES;
+        const uint32_t va = base + C::RING_OFF + vslot * C::TILE_BYTES;
+        issue_abt(0, qa, ka);                          // S = Q K_j^T
+        issue_abt(128, doa, va);                       // dP = dO V_j^T
+        issued = true;
+        mma_commit(bar_s);
+        mma_commit(bar_empty(vslot));                  // V_j no longer needed
+        if (!mbar_wait(bar_ds, j & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        // dQ += dS K_j: A = dS (packed 16-bit in TMEM columns [0, 64)), B = K_j MN-major.
+#pragma unroll
+        for (int kk = 0; kk < kBwdTile / 16; ++kk)
+          mma_f16_ts(tmem + C::ACC_COL, tmem + kk * 8, sdesc_mn_sw128(ka + kk * 2048, C::CHUNK),
+                     IDESC_Q, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar_empty(kslot));
+      }
+      if (issued) mma_commit(ok ? bar_done : bar_drain);
+      if (issued && !ok) mbar_wait_drain(bar_drain, 0, kDrainNs);
+    }
+  } else {
+    // ------------------------------------------------------------------ elementwise + epilogue
+    const int r = threadIdx.x;                              // query row of the tile
+    const int row = q0 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_base, tP = tS + 128, tQ = tS + C::ACC_COL;
+    const float lse2 = p.lse2[static_cast<size_t>(bh) * p.Nq_pad + row];
+    const float dsum = p.dsum[static_cast<size_t>(bh) * p.Nq_pad + row];
+    const int lim = CAUSAL ? min(row + p.causal_offset, p.Nk - 1) : p.Nk - 1;
+    const int lim_min = CAUSAL ? min(q0 + p.causal_offset, p.Nk - 1) : p.Nk - 1;
+    const float c = p.scale_log2;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_s, j & 1, wc))) { ok = false; break; }
+      tc_fence_after();
+      const int key0 = j * kBwdTile;
+      const bool masked = key0 + kBwdTile - 1 > lim_min;     // warp-uniform per CTA
+#pragma unroll
+      for (int cc = 0; cc < kBwdTile / 32; ++cc) {
+        uint32_t s[32], dp[32];
+        tmem_ld32x32b_x32(tS + 32 * cc, s);
+        tmem_ld32x32b_x32(tP + 32 * cc, dp);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float d2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int kk = 2 * i + e;
+            float pv = ex2_approx(__uint_as_float(s[kk]) * c - lse2);
+            if (masked && key0 + 32 * cc + kk > lim) pv = 0.f;
+            d2[e] = pv * (__uint_as_float(dp[kk]) - dsum);
+          }
+          pk[i] = pack_half2(d2[0], d2[1], BF16);
+        }
+        tmem_st32x32b_x16(tS + 16 * cc, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_ds);
+    }
+    if (ok && n_kv > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, wc));
+    if (ok) {
+      tc_fence_after();
+      // dQ = scale * (dS K), rows past Nq skipped; a tile without keys writes zeros.
+      const bool row_ok = row < p.Nq;
+      uint16_t* orow = static_cast<uint16_t*>(p.out) +
+                       (static_cast<size_t>(bh) * p.Nq + (row_ok ? row : 0)) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t a[32];
+        if (n_kv > 0) {
+          tmem_ld32x32b_x32(tQ + 32 * ch, a);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) a[i] = 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint4 w;
+          w.x = pack_half2(__uint_as_float(a[8 * u + 0]) * p.scale, __uint_as_float(a[8 * u + 1]) * p.scale, BF16);
+          w.y = pack_half2(__uint_as_float(a[8 * u + 2]) * p.scale, __uint_as_float(a[8 * u + 3]) * p.scale, BF16);
+          w.z = pack_half2(__uint_as_float(a[8 * u + 4]) * p.scale, __uint_as_float(a[8 * u + 5]) * p.scale, BF16);
+          w.w = pack_half2(__uint_as_float(a[8 * u + 6]) * p.scale, __uint_as_float(a[8 * u + 7]) * p.scale, BF16);
+          if (row_ok) *reinterpret_cast<uint4*>(orow + 32 * ch + 8 * u) = w;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// dK, dV: CTA (key tile kt, KV head bh_kv). K and V are loaded once; each step brings
+// Q_i and dO_i of one query tile of one query head of the group (a 2-item ring pair)
+// plus that tile's L * log2(e) and D vectors. TMEM: S^T [0,128) (P^T packed over its
+// first 64 columns), dP^T [128,256) (dS^T packed over its first 64), dV [256, 256+D),
+// dK [256+D, 256+2D).
+template <int D, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                   const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh_kv = blockIdx.y;
+  const int b = bh_kv / p.Hkv, hk = bh_kv - b * p.Hkv;
+  const int k0 = blockIdx.x * kBwdTile;
+  const int n_q = (p.Nq + kBwdTile - 1) / kBwdTile;
+  // Query tiles that see any key of this tile: queries i with k0 <= i + offset.
+  int q_first = 0;
+  if (CAUSAL) {
+    const int need = k0 - p.causal_offset;                  // smallest visible query row
+    q_first = need <= 0 ? 0 : min(n_q, need / kBwdTile);
+  }
+  const int per_head = n_q - q_first;
+  const int n_steps = per_head * p.group;                   // (head of the group, tile)
+  auto step_of = [&](int s, int& h, int& q0) {
+    const int g = s / max(per_head, 1);
+    h = hk * p.group + g;
+    q0 = (q_first + (s - g * per_head)) * kBwdTile;
+  };
+
+  const uint32_t bar0 = base + C::BAR_OFF;
+  const uint32_t bar_a = bar0;                                       // K and V landed
+  auto bar_full = [&](int i) { return bar0 + 8u * (1 + i); };        // pair slot i (Q, dO, vecs)
+  auto bar_empty = [&](int i) { return bar0 + 8u * (1 + C::NS + i); };
+  const uint32_t bar_s = bar0 + 8u * (1 + 2 * C::NS);                // S^T and dP^T ready
+  const uint32_t bar_ps = bar0 + 8u * (2 + 2 * C::NS);               // P^T, dS^T in TMEM (128)
+  const uint32_t bar_done = bar0 + 8u * (3 + 2 * C::NS);
+  const uint32_t bar_drain = bar0 + 8u * (4 + 2 * C::NS);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + C::MISC_OFF + 4);
+  constexpr int NP = C::NS / 2;                                      // ring pairs
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_a, 1);
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(bar_full(i), 1);
+      mbar_init(bar_empty(i), 1);
+    }
+    mbar_init(bar_s, 1);
+    mbar_init(bar_ps, kBwdTile);
+    mbar_init(bar_done, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == kBwdWarpMma) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{abort_flag, &g_fa_status, p.timeout_ns};
+  auto q_tile = [&](int slot) { return base + C::RING_OFF + (2 * slot) * C::TILE_BYTES; };
+  auto do_tile = [&](int slot) { return base + C::RING_OFF + (2 * slot + 1) * C::TILE_BYTES; };
+  auto vec = [&](int slot) { return sbase + C::VEC_OFF + slot * 2 * kBwdTile * 4; };
+
+  if (warp == kBwdWarpProd) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_steps > 0) {
+      mbar_arrive_expect_tx(bar_a, 2 * C::TILE_BYTES);
+      for (int ch = 0; ch < C::NCH; ++ch) {
+        tma_load_3d(base + C::A_OFF + ch * C::CHUNK, &tmK, bar_a, ch * 64, k0, bh_kv);
+        tma_load_3d(base + C::A_OFF + C::TILE_BYTES + ch * C::CHUNK, &tmV, bar_a, ch * 64, k0, bh_kv);
+      }
+      bool ok = true;
+      int s = 0;
+      for (; s < n_steps && ok; ++s) {
+        const int slot = s % NP, round = s / NP;
+        if (round > 0 && !mbar_wait(bar_empty(slot), (round - 1) & 1, wc)) { ok = false; break; }
+        int h, q0;
+        step_of(s, h, q0);
+        const int bhq = b * p.Hq + h;
+        mbar_arrive_expect_tx(bar_full(slot), 2 * C::TILE_BYTES + 2 * kBwdTile * 4);
+        for (int ch = 0; ch < C::NCH; ++ch) {
+          tma_load_3d(q_tile(slot) + ch * C::CHUNK, &tmQ, bar_full(slot), ch * 64, q0, bhq);
+          tma_load_3d(do_tile(slot) + ch * C::CHUNK, &tmDO, bar_full(slot), ch * 64, q0, bhq);
+        }
+        const size_t vrow = static_cast<size_t>(bhq) * p.Nq_pad + q0;
+        bulk_load(smem_u32(vec(slot)), p.lse2 + vrow, kBwdTile * 4, bar_full(slot));
+        bulk_load(smem_u32(vec(slot) + kBwdTile * 4), p.dsum + vrow, kBwdTile * 4, bar_full(slot));
+      }
+      if (!ok || *abort_flag) {
+        for (int i = max(0, s - NP); i < s; ++i)
+          mbar_wait_drain(bar_full(i % NP), (i / NP) & 1, kDrainNs);
+        mbar_wait_drain(bar_a, 0, kDrainNs);
+      }
+    }
+  } else if (warp == kBwdWarpMma) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_steps > 0) {
+      constexpr uint32_t IDESC_S = idesc_f16(kBwdTile, kBwdTile, BF16 ? 1u : 0u, 0u, 0u);
+      constexpr uint32_t IDESC_G = idesc_f16(kBwdTile, D, BF16 ? 1u : 0u, 0u, 1u);
+      auto issue_abt = [&](uint32_t col, uint32_t a, uint32_t bt) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;
+          mma_f16_ss(tmem + col, sdesc_k_sw128(a + (kk >> 2) * C::CHUNK + koff),
+                     sdesc_k_sw128(bt + (kk >> 2) * C::CHUNK + koff), IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      // X[acc] += A[128 x 128] (packed 16-bit in TMEM at col a) B[128 x D] (MN-major).
+      auto issue_tb = [&](uint32_t acc, uint32_t a, uint32_t bmn, bool acc0) {
+#pragma unroll
+        for (int kk = 0; kk < kBwdTile / 16; ++kk)
+          mma_f16_ts(tmem + acc, tmem + a + kk * 8, sdesc_mn_sw128(bmn + kk * 2048, C::CHUNK), IDESC_G,
+                     (acc0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bar_a, 0, wc);
+      bool issued = false;
+      tc_fence_after();
+      const uint32_t ka = base + C::A_OFF, va = base + C::A_OFF + C::TILE_BYTES;
+      for (int s = 0; s < n_steps && ok; ++s) {
+        const int slot = s % NP;
+        if (!mbar_wait(bar_full(slot), (s / NP) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        issue_abt(0, ka, q_tile(slot));                 // S^T = K Q_i^T
+        issue_abt(128, va, do_tile(slot));              // dP^T = V dO_i^T
+        issued = true;
+        mma_commit(bar_s);
+        if (!mbar_wait(bar_ps, s & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        issue_tb(C::ACC_COL, 0, do_tile(slot), s > 0);          // dV += P^T dO_i
+        issue_tb(C::ACC_COL + D, 128, q_tile(slot), s > 0);     // dK += dS^T Q_i
+        mma_commit(bar_empty(slot));
+      }
+      if (issued) mma_commit(ok ? bar_done : bar_drain);
+      if (issued && !ok) mbar_wait_drain(bar_drain, 0, kDrainNs);
+    }
+  } else {
+    // ------------------------------------------------------------------ elementwise + epilogue
+    const int r = threadIdx.x;                              // key row of the tile
+    const int key = k0 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_base, tP = tS + 128;
+    const uint32_t tV = tS + C::ACC_COL, tK = tS + C::ACC_COL + D;
+    const float c = p.scale_log2;
+    bool ok = true;
+    for (int s = 0; s < n_steps; ++s) {
+      const int slot = s % NP;
+      // The vectors of this step landed with its Q tile (the MMA warp waited for them too).
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_full(slot), (s / NP) & 1, wc))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_s, s & 1, wc))) { ok = false; break; }
+      tc_fence_after();
+      int h, q0;
+      step_of(s, h, q0);
+      const float* lv = reinterpret_cast<const float*>(vec(slot));
+      const float* dv = lv + kBwdTile;
+      // Key `key` is visible to query q0 + col iff key <= q0 + col + offset.
+      const int first_vis = key - p.causal_offset - q0;     // smallest visible column
+      const bool masked = CAUSAL && __any_sync(0xffffffffu, first_vis > 0);
+#pragma unroll
+      for (int cc = 0; cc < kBwdTile / 32; ++cc) {
+        uint32_t st[32], dpt[32];
+        tmem_ld32x32b_x32(tS + 32 * cc, st);
+        tmem_ld32x32b_x32(tP + 32 * cc, dpt);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = 32 * cc + 2 * i + e;
+            float x = ex2_approx(__uint_as_float(st[2 * i + e]) * c - lv[col]);
+            if (masked && col < first_vis) x = 0.f;
+            pv[e] = x;
+            dsv[e] = x * (__uint_as_float(dpt[2 * i + e]) - dv[col]);
+          }
+          pk[i] = pack_half2(pv[0], pv[1], BF16);
+          dk[i] = pack_half2(dsv[0], dsv[1], BF16);
+        }
+        tmem_st32x32b_x16(tS + 16 * cc, pk);
+        tmem_st32x32b_x16(tP + 16 * cc, dk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_ps);
+    }
+    if (ok && n_steps > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, wc));
+    if (ok) {
+      tc_fence_after();
+      const bool row_ok = key < p.Nk;
+      const size_t orow = (static_cast<size_t>(bh_kv) * p.Nk + (row_ok ? key : 0)) * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {             // dV, then dK (times scale)
+        uint16_t* dst = static_cast<uint16_t*>(which ? p.out : p.out2) + orow;
+        const float f = which ? p.scale : 1.0f;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t a[32];
+          if (n_steps > 0) {
+            tmem_ld32x32b_x32((which ? tK : tV) + 32 * ch, a);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) a[i] = 0u;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 w;
+            w.x = pack_half2(__uint_as_float(a[8 * u + 0]) * f, __uint_as_float(a[8 * u + 1]) * f, BF16);
+            w.y = pack_half2(__uint_as_float(a[8 * u + 2]) * f, __uint_as_float(a[8 * u + 3]) * f, BF16);
+            w.z = pack_half2(__uint_as_float(a[8 * u + 4]) * f, __uint_as_float(a[8 * u + 5]) * f, BF16);
+            w.w = pack_half2(__uint_as_float(a[8 * u + 6]) * f, __uint_as_float(a[8 * u + 7]) * f, BF16);
+            if (row_ok) *reinterpret_cast<uint4*>(dst + 32 * ch + 8 * u) = w;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

@@ -62,13 +62,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
-// Bulk (non-tensor) TMA copy global -> shared, completing on an mbarrier.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar) : "memory");
-}
-
 // A pair of fp32 values: one packed f32x2 register pair (FA_DEC_F32X2 = 1, default) or
 // two scalar floats.
 #ifndef FA_DEC_F32X2

@@ -13,6 +13,7 @@
 #include "decode_kernel.cuh"
 #include "decode_tc_kernel.cuh"
 #include "fwd_kernel.cuh"
+#include "bwd_kernel.cuh"
 
 namespace {
 
@@ -87,6 +88,53 @@ bool make_tile_map(CUtensorMap* m, const void* ptr, int d, int rows, long long h
              const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------------------
+// Backward launch: D and L * log2(e), then dQ, then dK / dV (stream-ordered).
+// ---------------------------------------------------------------------------------------
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+         cudaSuccess;
+}
+
+template <int D, bool BF16>
+fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const CUtensorMap& mdo, const void* o, const void* dout, const float* lse,
+                     void* dq, void* dk, void* dv, fa::BwdParams prm, long long BH, long long BHkv,
+                     int n_q, int n_k, int causal, cudaStream_t st) {
+  using C = fa::BwdCfg<D>;
+  auto dq_c = fa::fa_bwd_dq_kernel<D, BF16, true>;
+  auto dq_n = fa::fa_bwd_dq_kernel<D, BF16, false>;
+  auto kv_c = fa::fa_bwd_dkdv_kernel<D, BF16, true>;
+  auto kv_n = fa::fa_bwd_dkdv_kernel<D, BF16, false>;
+  static int ready[kMaxDevices];
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!ready[dev]) {
+      if (!set_smem(dq_c, C::SMEM_BYTES) || !set_smem(dq_n, C::SMEM_BYTES) ||
+          !set_smem(kv_c, C::SMEM_BYTES) || !set_smem(kv_n, C::SMEM_BYTES))
+        return FA_ERR_CUDA;
+      ready[dev] = 1;
+    }
+  }
+  const long long warps = BH * prm.Nq_pad;
+  fa::fa_bwd_preprocess_kernel<D, BF16><<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(
+      static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse,
+      const_cast<float*>(prm.lse2), const_cast<float*>(prm.dsum), static_cast<int>(BH), prm.Nq,
+      prm.Nq_pad);
+  prm.out = dq;
+  prm.out2 = nullptr;
+  const dim3 gq(n_q, static_cast<unsigned>(BH));
+  if (causal) dq_c<<<gq, fa::kBwdThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, prm);
+  else dq_n<<<gq, fa::kBwdThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, prm);
+  prm.out = dk;
+  prm.out2 = dv;
+  const dim3 gk(n_k, static_cast<unsigned>(BHkv));
+  if (causal) kv_c<<<gk, fa::kBwdThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, prm);
+  else kv_n<<<gk, fa::kBwdThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -374,12 +422,74 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, Nk, d, causal, scale, dtype, stream);
 }
 
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+                 int Nk, int d, int causal, float scale, fa_dtype dtype, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (Nq <= 0 || Nk <= 0 || (causal != 0 && causal != 1)) return FA_ERR_INVALID_ARG;
+  fa_status s = common_checks(B, Hq, Hkv, d, scale, dtype);
+  if (s != FA_OK) return s;
+  const long long BH = static_cast<long long>(B) * Hq;
+  const long long BHkv = static_cast<long long>(B) * Hkv;
+  const int n_q = (Nq + fa::kBwdTile - 1) / fa::kBwdTile;
+  const int n_k = (Nk + fa::kBwdTile - 1) / fa::kBwdTile;
+  if (BH >= 65536 || BHkv >= 65536 || BH * n_q * fa::kBwdTile * 32 >= (1LL << 31))
+    return FA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv)})
+    if (!aligned16(ptr)) return FA_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < fa_bwd_workspace_bytes(B, Hq, Nq)) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_ALIGNMENT;
+  int dev = 0;
+  s = check_device(&dev);
+  if (s != FA_OK) return s;
+
+  const bool bf16 = dtype == FA_BF16;
+  const int nq_pad = n_q * fa::kBwdTile;
+  float* lse2 = static_cast<float*>(workspace);
+  float* dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                         fa_bwd_workspace_bytes(B, Hq, Nq) / 2);
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_tile_map(&mq, q, d, Nq, BH, bf16, fa::kBwdTile) ||
+      !make_tile_map(&mdo, dout, d, Nq, BH, bf16, fa::kBwdTile) ||
+      !make_tile_map(&mk, k, d, Nk, BHkv, bf16, fa::kBwdTile) ||
+      !make_tile_map(&mv, v, d, Nk, BHkv, bf16, fa::kBwdTile))
+    return FA_ERR_CUDA;
+  fa::BwdParams prm;
+  prm.lse2 = lse2;
+  prm.dsum = dsum;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.Nq_pad = nq_pad;
+  prm.causal_offset = Nk - Nq;
+  prm.scale = scale;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.timeout_ns = g_timeout_ns;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return bf16 ? launch_bwd<64, true>(dev, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st)
+                : launch_bwd<64, false>(dev, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st);
+  return bf16 ? launch_bwd<128, true>(dev, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st)
+              : launch_bwd<128, false>(dev, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st);
+}
+
 fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* vcache, void* o,
                          float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int cache_len,
                          int d, int causal, float scale, fa_dtype dtype, void* stream) {
   if (cache_len < Nk || cache_len <= 0) return FA_ERR_INVALID_ARG;
   return fwd_impl(q, kcache, vcache, o, lse, B, Hq, Hkv, Nq, Nk, cache_len, d, causal, scale,
                   dtype, stream);
+}
+
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq) {
+  if (B <= 0 || Hq <= 0 || Nq <= 0) return 0;
+  const size_t nq_pad = static_cast<size_t>((Nq + fa::kBwdTile - 1) / fa::kBwdTile) * fa::kBwdTile;
+  return 2 * align_up(static_cast<size_t>(B) * Hq * nq_pad * sizeof(float), 256);
 }
 
 size_t fa_decode_workspace_bytes(int B, int Hq, int max_kv_len, int d) {

@@ -242,6 +242,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint
 
 // L2 prefetch of a contiguous global range (a hint: no completion). 16-byte aligned
 // address, size a multiple of 16.
+// Bulk (non-tensor) TMA copy global -> shared, completing on an mbarrier. Both addresses
+// 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
                :: "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes) : "memory");

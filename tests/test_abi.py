@@ -78,6 +78,29 @@ def test_fwd_kvcache_rejects_bad_arguments_without_cuda():
     assert call(k=24) == fa.FA_ERR_ALIGNMENT
 
 
+def test_bwd_rejects_bad_arguments_without_cuda():
+    L = fa.lib()
+    ws_need = L.fa_bwd_workspace_bytes(1, 2, 200)
+    assert ws_need == 2 * 2 * 256 * 4          # L*log2(e) and D, each [B*Hq, Nq padded to 256]
+    assert L.fa_bwd_workspace_bytes(0, 2, 200) == 0
+
+    def call(**kw):
+        a = dict(q=16, k=16, v=16, o=16, lse=16, do=16, dq=16, dk=16, dv=16, B=1, Hq=2, Hkv=1,
+                 Nq=200, Nk=200, d=64, causal=1, scale=0.125, dtype=0, ws=16, ws_bytes=ws_need)
+        a.update(kw)
+        return L.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["do"], a["dq"], a["dk"], a["dv"],
+                        a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"], a["d"], a["causal"], a["scale"],
+                        a["dtype"], a["ws"], a["ws_bytes"], None)
+    assert call(lse=None) == fa.FA_ERR_INVALID_ARG
+    assert call(dv=None) == fa.FA_ERR_INVALID_ARG
+    assert call(Nk=0) == fa.FA_ERR_INVALID_ARG
+    assert call(Hq=3, Hkv=2) == fa.FA_ERR_INVALID_ARG
+    assert call(d=80) == fa.FA_ERR_UNSUPPORTED
+    assert call(dk=8) == fa.FA_ERR_ALIGNMENT
+    assert call(ws_bytes=ws_need - 1) == fa.FA_ERR_WORKSPACE
+    assert call(ws=None) == fa.FA_ERR_WORKSPACE
+
+
 def test_decode_rejects_bad_arguments_without_cuda():
     L = fa.lib()
     need = fa.decode_workspace_bytes(2, 8, 4096, 128)
