@@ -431,6 +431,22 @@ def run_single_kernel(args):
 
         def call():
             fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+    elif args.only == "bwd":
+        # Backward pass (fa_bwd) of the workload, with fa_fwd's O and LSE as its inputs.
+        # Algorithmic FLOPs: 2.5x the forward's (five N^2 d products instead of two).
+        w = WORKLOADS[args.workload]
+        q, k, v = (t.to(dev) for t in make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed))
+        gen = torch.Generator(device=dev).manual_seed(w.seed + 1)
+        dout = torch.randn(q.shape, generator=gen, device=dev, dtype=torch.float32).to(q.dtype)
+        o, lse = fa.fwd(q, k, v, causal=w.causal, scale=w.scale)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(fa.bwd_workspace_bytes(w.B, w.Hq, w.N), dtype=torch.uint8, device=dev)
+        work = 2.5 * fwd_flops(w.B, w.Hq, w.N, w.N, w.d, w.causal) / 1e12
+        unit = "TFLOP/s"
+
+        def call():
+            fa.bwd(q, k, v, o, lse, dout, causal=w.causal, scale=w.scale, dq=dq, dk=dk, dv=dv,
+                   workspace=ws)
     elif args.only == "chunked":
         # Chunked prefill: the workload's sequence in --chunk-token pieces, each attending
         # to the cache prefix up to its own end (fa_fwd_kvcache); same causal FLOPs.
@@ -483,7 +499,7 @@ def run_single_kernel(args):
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("--only", choices=["fwd", "decode", "chunked"], default=None,
+    ap.add_argument("--only", choices=["fwd", "decode", "chunked", "bwd"], default=None,
                     help="launch one entry point alone (profiling helper; prints its own line)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)

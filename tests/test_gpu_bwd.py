@@ -64,3 +64,28 @@ def test_grouped_query_heads(Hq, Hkv, causal):
 def test_rectangular(Nq, Nk, causal):
     """Nq != Nk with bottom-right causal alignment; Nq > Nk has rows without keys."""
     check_bwd(1, 4, 2, Nq, Nk, 64, "fp16", causal, seed=Nq + 3 * Nk)
+
+
+def test_mha2k_workload_sampled_heads():
+    """The full causal B=8 H=12 N=2048 d=64 fp16 backward pass; two (batch, head) problems
+    checked element by element against the oracle (each head is independent here)."""
+    from workloads import WORKLOADS
+    w = WORKLOADS["mha2k"]
+    q, k, v = make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed)
+    g = torch.Generator().manual_seed(w.seed + 1)
+    dout = torch.randn(q.shape, generator=g).to(q.dtype)
+    qd, kd, vd, dod = q.to(DEV), k.to(DEV), v.to(DEV), dout.to(DEV)
+    o, lse = fa.fwd(qd, kd, vd, causal=True, scale=w.scale)
+    dq, dk, dv = fa.bwd(qd, kd, vd, o, lse, dod, causal=True, scale=w.scale)
+    torch.cuda.synchronize()
+    assert fa.device_status() == fa.FA_OK
+    rms_tol, max_tol = TOL[w.dtype]
+    for b, h in ((0, 0), (w.B - 1, w.Hq - 1)):
+        sl = slice(b, b + 1), slice(h, h + 1)
+        ref = attention_bwd_f64(q[sl], k[sl], v[sl], dout[sl], True, w.scale)
+        for name, got, want in zip(("dq", "dk", "dv"), (dq[sl], dk[sl], dv[sl]), ref):
+            got = to_f64(got.cpu())
+            err = got - want
+            rel_rms = math.sqrt(float(np.mean(err ** 2))) / math.sqrt(float(np.mean(want ** 2)))
+            rel_max = float(np.max(np.abs(err))) / float(np.max(np.abs(want)))
+            assert rel_rms <= rms_tol and rel_max <= max_tol, f"{name} b{b} h{h}: {rel_rms:.2e} {rel_max:.2e}"
