@@ -5,7 +5,9 @@ CPU-baseline leg of `bench.py`, never by the CUDA library or its Python binding.
 """
 from .attention import attention_f64, attention_rows_f64, decode_f64, visible_mask
 from .backward import attention_bwd_f64
+from .paged import attention_paged_rows_f64, decode_paged_f64, gather_pages
 from .tiled import tiled_attention_f64
 
 __all__ = ["attention_f64", "attention_rows_f64", "decode_f64", "visible_mask",
-           "tiled_attention_f64", "attention_bwd_f64"]
+           "tiled_attention_f64", "attention_bwd_f64", "decode_paged_f64",
+           "attention_paged_rows_f64", "gather_pages"]

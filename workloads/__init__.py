@@ -27,7 +27,7 @@ from typing import Optional
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "make_fwd_inputs", "make_decode_inputs",
-           "fwd_flops", "decode_kv_bytes", "torch_dtype"]
+           "make_page_table", "paginate", "fwd_flops", "decode_kv_bytes", "torch_dtype"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -104,6 +104,48 @@ def make_decode_inputs(B: int, Hq: int, Hkv: int, cache_len: int, d: int, dtype:
     kc = _randn16(gen, (B, Hkv, cache_len, d), dt)
     vc = _randn16(gen, (B, Hkv, cache_len, d), dt)
     return kv_lens, q, kc, vc
+
+
+def make_page_table(lens, page_size: int, max_pages: int, spare_pages: int = 3, seed: int = 0,
+                    fill: int = -1):
+    """Random page assignment for a paged KV cache.
+
+    Sequence b receives ceil(lens[b] / page_size) pages, taken in order from one seeded
+    random permutation of the pool (``torch.randperm``), so pages of different sequences
+    never coincide and consecutive tokens land in scattered pages. The pool has
+    ``spare_pages`` pages more than the sequences use; table entries past a sequence's
+    last page hold ``fill``. Returns (table int32 [B, max_pages], num_pages).
+    """
+    lens = [int(x) for x in torch.as_tensor(lens).tolist()]
+    need = [(n + page_size - 1) // page_size for n in lens]
+    if max(need, default=0) > max_pages:
+        raise ValueError("a sequence needs more pages than max_pages")
+    num_pages = sum(need) + spare_pages
+    gen = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(num_pages, generator=gen).to(torch.int32)
+    table = torch.full((len(lens), max_pages), fill, dtype=torch.int32)
+    at = 0
+    for b, n in enumerate(need):
+        table[b, :n] = perm[at:at + n]
+        at += n
+    return table, num_pages
+
+
+def paginate(cache: torch.Tensor, table: torch.Tensor, lens, page_size: int, num_pages: int,
+             fill_value: float = float("nan")) -> torch.Tensor:
+    """Copy tokens [0, lens[b]) of a contiguous cache [B, Hkv, L, d] into a page pool
+    [num_pages, Hkv, page_size, d] laid out by `table` (token t of sequence b goes to
+    page table[b, t // page_size], row t % page_size). Pool rows no token maps to hold
+    `fill_value` (NaN by default, so a kernel that reads them shows it)."""
+    B, Hkv, _, d = cache.shape
+    pool = torch.full((num_pages, Hkv, page_size, d), fill_value, dtype=cache.dtype)
+    lens = [int(x) for x in torch.as_tensor(lens).tolist()]
+    for b in range(B):
+        for j in range((lens[b] + page_size - 1) // page_size):
+            t0 = j * page_size
+            t1 = min(lens[b], t0 + page_size)
+            pool[int(table[b, j]), :, : t1 - t0] = cache[b, :, t0:t1]
+    return pool
 
 
 def workload_inputs(w: Workload):
