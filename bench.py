@@ -25,7 +25,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from workloads import WORKLOADS, decode_kv_bytes, fwd_flops, make_decode_inputs, make_fwd_inputs  # noqa: E402
+from workloads import (WORKLOADS, decode_kv_bytes, fwd_flops, make_decode_inputs,  # noqa: E402
+                       make_fwd_inputs, make_page_table, paginate)
 
 METRIC = "attn fwd TFLOP/s & % BF16 TC peak; decode KV-read GB/s & % HBM peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -463,6 +464,39 @@ def run_single_kernel(args):
             for n, i in enumerate(range(0, w.N, C)):
                 fa.fwd_kvcache(qs[n], k, v, min(i + C, w.N), causal=True, scale=w.scale, out=outs[n],
                                return_lse=False)
+    elif args.only == "fwd_paged":
+        # Prefill of the workload with K and V in a page pool (fa_fwd_paged), pages drawn by
+        # a seeded random table; same causal FLOPs as --only fwd.
+        w = WORKLOADS[args.workload]
+        q, k, v = make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed)
+        ps = args.page_size
+        lens = torch.full((w.B,), w.N)
+        table, n_pages = make_page_table(lens, ps, (w.N + ps - 1) // ps, seed=w.seed)
+        kp, vp = paginate(k, table, lens, ps, n_pages), paginate(v, table, lens, ps, n_pages)
+        q, kp, vp, table = q.to(dev), kp.to(dev), vp.to(dev), table.to(dev)
+        o, lse = torch.empty_like(q), torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+        work = fwd_flops(w.B, w.Hq, w.N, w.N, w.d, w.causal) / 1e12
+        unit = "TFLOP/s"
+
+        def call():
+            fa.fwd_paged(q, kp, vp, table, w.N, causal=w.causal, scale=w.scale, out=o, lse=lse)
+    elif args.only == "decode_paged":
+        # The decode workload with its cache in a page pool (fa_decode_paged).
+        w = WORKLOADS[args.decode_workload]
+        kv_cpu, dq, kc, vc = make_decode_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.dtype, w.kv_len_lo,
+                                                w.kv_len_hi, w.seed)
+        ps = args.page_size
+        table, n_pages = make_page_table(kv_cpu, ps, w.N // ps, seed=w.seed)
+        kp, vp = paginate(kc, table, kv_cpu, ps, n_pages), paginate(vc, table, kv_cpu, ps, n_pages)
+        del kc, vc
+        kv_lens, dq, kp, vp, table = kv_cpu.to(dev), dq.to(dev), kp.to(dev), vp.to(dev), table.to(dev)
+        do, dlse = torch.empty_like(dq), torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+        ws = torch.empty(fa.decode_workspace_bytes(w.B, w.Hq, w.N, w.d), dtype=torch.uint8, device=dev)
+        work = (decode_kv_bytes(kv_cpu, w.Hkv, w.d) + 4 * dq.numel() + 4 * dlse.numel()) / 1e9
+        unit = "GB/s"
+
+        def call():
+            fa.decode_paged(dq, kp, vp, table, kv_lens, scale=w.scale, out=do, lse=dlse, workspace=ws)
     else:
         w = WORKLOADS[args.decode_workload]
         kv_cpu, dq, kc, vc = make_decode_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.dtype, w.kv_len_lo,
@@ -492,14 +526,16 @@ def run_single_kernel(args):
     status = fa.status_string(fa.device_status())
     avg = sum(ms) / len(ms)
     print(json.dumps({"only": args.only, "workload": w.describe(),
-                      **({"chunk": args.chunk} if args.only == "chunked" else {}), "ms_per_launch": avg,
+                      **({"chunk": args.chunk} if args.only == "chunked" else {}),
+                      **({"page_size": args.page_size} if "paged" in args.only else {}), "ms_per_launch": avg,
                       "value": work / (avg * 1e-3), "unit": unit, "device_status": status}))
     return 0 if status == "FA_OK" else 1
 
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("--only", choices=["fwd", "decode", "chunked", "bwd"], default=None,
+    ap.add_argument("--only", choices=["fwd", "decode", "chunked", "bwd", "fwd_paged", "decode_paged"],
+                    default=None,
                     help="launch one entry point alone (profiling helper; prints its own line)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -507,6 +543,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mha2k", choices=[k for k, v in WORKLOADS.items() if v.kind == "fwd"])
     ap.add_argument("--chunk", type=int, default=1024, help="--only chunked: tokens per chunk")
+    ap.add_argument("--page-size", type=int, default=64, help="--only *_paged: tokens per page")
     ap.add_argument("--decode-workload", default="decode")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

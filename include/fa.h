@@ -100,6 +100,47 @@ FA_API fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* v
                          int d, int causal, float scale, fa_dtype dtype, void* stream);
 
 /*
+ * Paged KV cache (fa_fwd_paged, fa_decode_paged).
+ *
+ * Defined by: page "Flash Attention ... IO-aware exact" (fr), "Optimisation avancée : KV
+ * Cache et persistent attention": keys and values are cached per session, extended as
+ * tokens arrive and released per session. Here the cache is one pool of fixed-size pages
+ * shared by all sequences: a sequence owns a list of pages (its block-table row), so a
+ * sequence is grown or released without moving any other sequence's data. The result is
+ * the one fa_fwd / fa_decode give on the sequence's tokens gathered in order.
+ *
+ *   kpool, vpool  [num_pages, Hkv, page_size, d] fp16/bf16, 16-byte aligned: page p of KV
+ *                 head h holds page_size consecutive tokens of one sequence
+ *   block_table   [B, max_pages_per_seq] int32, device memory, 4-byte aligned: token t of
+ *                 sequence b sits in page block_table[b][t / page_size], row
+ *                 t % page_size. Only the entries that cover the sequence's tokens are
+ *                 read (the others may hold anything, e.g. -1).
+ *   page_size     a power of two >= 16 (FA_ERR_UNSUPPORTED otherwise)
+ *   num_pages     pool size; num_pages * Hkv < 2^31 - 1, max_pages_per_seq * page_size < 2^31
+ *
+ * Pool rows that hold no token of the sequence (a page's rows past the sequence's end,
+ * pages of other sequences, unused pages) never affect the result, whatever they hold.
+ * A table entry that is read and lies outside [0, num_pages) is never dereferenced: the
+ * kernel records FA_ERR_INVALID_ARG in the device status word (fa_device_status) and the
+ * result of that sequence is unspecified.
+ */
+
+/*
+ * fa_fwd_paged — fa_fwd_kvcache with the keys and values in a paged pool: each of the B
+ * sequences attends to its first Nk tokens, found through its block-table row.
+ *
+ *   q, o, lse   as fa_fwd, [B, Hq, Nq, d] / [B, Hq, Nq]
+ *   causal      0 or 1, bottom-right aligned (the chunk is the last Nq of the Nk tokens)
+ *
+ * Requirements: those of fa_fwd and of the paged cache above, plus
+ * Nk <= max_pages_per_seq * page_size.
+ */
+FA_API fa_status fa_fwd_paged(const void* q, const void* kpool, const void* vpool,
+                       const int* block_table, void* o, float* lse, int B, int Hq, int Hkv,
+                       int Nq, int Nk, int num_pages, int page_size, int max_pages_per_seq,
+                       int d, int causal, float scale, fa_dtype dtype, void* stream);
+
+/*
  * fa_bwd_workspace_bytes — bytes of scratch that fa_bwd needs for these sizes.
  */
 FA_API size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq);
@@ -175,6 +216,23 @@ FA_API fa_status fa_decode(const void* q, const void* kcache, const void* vcache
                     void* stream);
 
 /*
+ * fa_decode_paged — fa_decode over a paged pool (see "Paged KV cache" above): sequence b
+ * attends to its first kv_lens[b] tokens, found through its block-table row.
+ *
+ *   q, o, lse, kv_lens   as fa_decode; kv_lens are clamped to
+ *                        [0, max_pages_per_seq * page_size]
+ *   workspace            at least fa_decode_workspace_bytes(B, Hq,
+ *                        max_pages_per_seq * page_size, d) bytes, as for fa_decode
+ *
+ * Requirements: those of fa_decode and of the paged cache.
+ */
+FA_API fa_status fa_decode_paged(const void* q, const void* kpool, const void* vpool,
+                          const int* block_table, const int* kv_lens, void* o, float* lse,
+                          int B, int Hq, int Hkv, int num_pages, int page_size,
+                          int max_pages_per_seq, int d, float scale, fa_dtype dtype,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fa_decode_noalloc — fa_decode for callers that cannot allocate device memory.
  *
  * Not from the pages (they have no counterpart): a convenience form of fa_decode whose
@@ -211,7 +269,8 @@ FA_API const char* fa_status_string(fa_status s);
 
 /*
  * fa_device_status — synchronises the current device, then returns FA_OK or the first
- * error a kernel of this library recorded on it (FA_ERR_DEVICE_TIMEOUT). If `clear` is
+ * error a kernel of this library recorded on it (FA_ERR_DEVICE_TIMEOUT, or
+ * FA_ERR_INVALID_ARG for a paged-cache table entry outside the pool). If `clear` is
  * non-zero the recorded error is reset afterwards. FA_ERR_CUDA if the synchronisation
  * itself fails.
  */

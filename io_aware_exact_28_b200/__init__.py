@@ -9,6 +9,7 @@ Functions mirror the C ABI in ``include/fa.h``:
 * ``fwd(q, k, v, causal, scale)`` -> ``(o, lse)``   (``fa_fwd``)
 * ``decode(q, kcache, vcache, kv_lens, scale)`` -> ``(o, lse)``   (``fa_decode``)
 * ``decode_workspace_bytes(B, Hq, max_kv_len, d)``   (``fa_decode_workspace_bytes``)
+* ``fwd_kvcache``, ``fwd_paged``, ``decode_paged``, ``decode_noalloc``, ``bwd``
 * ``device_status``, ``set_wait_timeout_ns``, ``debug_skip_q_load``, ``build_info``
 """
 from __future__ import annotations
@@ -25,7 +26,7 @@ __all__ = ["FAError", "FALibraryError", "LIB_PATH", "lib", "fwd", "decode",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_ALIGNMENT",
            "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_FP16", "FA_BF16",
            "decode_noalloc", "DECODE_NOALLOC_SCRATCH_BYTES", "fwd_kvcache", "bwd",
-           "bwd_workspace_bytes"]
+           "bwd_workspace_bytes", "fwd_paged", "decode_paged"]
 
 # FA_B200_LIB may name another build of the same library (e.g. a variant for timing).
 LIB_PATH = os.environ.get("FA_B200_LIB") or \
@@ -38,7 +39,7 @@ FA_FP16, FA_BF16 = 0, 1
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode", "fa_decode_workspace_bytes", "fa_status_string",
                     "fa_device_status", "fa_set_wait_timeout_ns", "fa_debug_skip_q_load",
                     "fa_build_info", "fa_decode_noalloc", "fa_fwd_kvcache", "fa_bwd",
-                    "fa_bwd_workspace_bytes")
+                    "fa_bwd_workspace_bytes", "fa_fwd_paged", "fa_decode_paged")
 
 # Size of the library's fixed decode scratch (FA_DECODE_NOALLOC_SCRATCH_BYTES in fa.h).
 DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -98,6 +99,11 @@ def lib() -> ctypes.CDLL:
         L.fa_build_info.restype = ctypes.c_char_p
         L.fa_decode_noalloc.argtypes = [c_void_p] * 6 + [c_int] * 5 + [c_float, c_int, c_void_p]
         L.fa_decode_noalloc.restype = c_int
+        L.fa_fwd_paged.argtypes = [c_void_p] * 6 + [c_int] * 10 + [c_float, c_int, c_void_p]
+        L.fa_fwd_paged.restype = c_int
+        L.fa_decode_paged.argtypes = [c_void_p] * 7 + [c_int] * 7 + [c_float, c_int, c_void_p,
+                                                                     c_size_t, c_void_p]
+        L.fa_decode_paged.restype = c_int
         _lib = L
         return L
 
@@ -220,6 +226,87 @@ def fwd_kvcache(q, kcache, vcache, nk: int, causal: bool = True, scale: Optional
                               float(scale), _dtype_code(q), _stream_ptr(stream))
     if st != FA_OK:
         raise FAError(st, "fa_fwd_kvcache")
+    return out, lse
+
+
+def _check_pool(q, kpool, vpool, block_table):
+    import torch
+    _check(kpool, "kpool", 4, q.device)
+    _check(vpool, "vpool", 4, q.device)
+    _check(block_table, "block_table", 2, q.device)
+    if block_table.dtype != torch.int32:
+        raise TypeError("block_table must be int32")
+    if kpool.dtype != q.dtype or vpool.dtype != q.dtype:
+        raise TypeError("q and the page pools must share one dtype")
+    if tuple(vpool.shape) != tuple(kpool.shape) or kpool.shape[3] != q.shape[-1]:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} kpool{tuple(kpool.shape)}")
+    if block_table.shape[0] != q.shape[0]:
+        raise ValueError("block_table needs one row per sequence")
+
+
+def fwd_paged(q, kpool, vpool, block_table, nk: int, causal: bool = True,
+              scale: Optional[float] = None, out=None, lse=None, return_lse: bool = True,
+              stream=None):
+    """Prefill against a paged KV cache via ``fa_fwd_paged``: q [B,Hq,Nq,d] attends to the
+    first ``nk`` tokens of each sequence, kept in pools [num_pages,Hkv,page_size,d] at the
+    pages listed by block_table int32 [B, max_pages] (causal: the chunk is the last Nq of
+    the nk tokens). Returns (o [B,Hq,Nq,d], lse [B,Hq,Nq] fp32 or None).
+    """
+    import torch
+    _check(q, "q", 4, q.device)
+    _check_pool(q, kpool, vpool, block_table)
+    B, Hq, Nq, d = q.shape
+    num_pages, Hkv, page_size, _ = kpool.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    _check(out, "out", 4, q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _check(lse, "lse", 3, q.device)
+    st = lib().fa_fwd_paged(q.data_ptr(), kpool.data_ptr(), vpool.data_ptr(),
+                            block_table.data_ptr(), out.data_ptr(),
+                            lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, int(nk),
+                            num_pages, page_size, block_table.shape[1], d, 1 if causal else 0,
+                            float(scale), _dtype_code(q), _stream_ptr(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_paged")
+    return out, lse
+
+
+def decode_paged(q, kpool, vpool, block_table, kv_lens, scale: Optional[float] = None, out=None,
+                 lse=None, workspace=None, return_lse: bool = True, stream=None):
+    """Single-token decode over a paged KV cache via ``fa_decode_paged``.
+
+    q [B,Hq,d]; kpool, vpool [num_pages,Hkv,page_size,d]; block_table int32 [B, max_pages];
+    kv_lens int32 [B]; all on the device. Returns (o [B,Hq,d], lse [B,Hq] fp32 or None).
+    """
+    import torch
+    _check(q, "q", 3, q.device)
+    _check_pool(q, kpool, vpool, block_table)
+    _check(kv_lens, "kv_lens", 1, q.device)
+    if kv_lens.dtype != torch.int32 or kv_lens.shape[0] != q.shape[0]:
+        raise TypeError("kv_lens must be int32 [B]")
+    B, Hq, d = q.shape
+    num_pages, Hkv, page_size, _ = kpool.shape
+    max_pages = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_bytes(B, Hq, max_pages * page_size, d),
+                                dtype=torch.uint8, device=q.device)
+    st = lib().fa_decode_paged(q.data_ptr(), kpool.data_ptr(), vpool.data_ptr(),
+                               block_table.data_ptr(), kv_lens.data_ptr(), out.data_ptr(),
+                               lse.data_ptr() if lse is not None else None, B, Hq, Hkv, num_pages,
+                               page_size, max_pages, d, float(scale), _dtype_code(q),
+                               workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                               _stream_ptr(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_decode_paged")
     return out, lse
 
 

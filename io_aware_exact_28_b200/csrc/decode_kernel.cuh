@@ -18,6 +18,11 @@
 // The four warps merge through shared memory and the CTA writes, per query head, a
 // normalised partial O row and its log2-domain logsumexp.
 //
+// PAGED = true reads the rows from a page pool (PagedKV in sm100.cuh). Pages hold a power
+// of two >= 16 tokens and stages start at multiples of 32, so a stage is one copy per
+// tensor from one page, or two from two 16-token pages. A table entry outside the pool is
+// recorded in the status word and its rows are not copied.
+//
 // Combine kernel: grid (sequence x query head), D threads, launched as a programmatic
 // dependent of the split kernel. It merges the valid splits with weights 2^(lse_s - max)
 // (the online-softmax rescaling identity, page "Kotaemon FlashAttention", running max and
@@ -48,6 +53,7 @@ struct DecodeParams {
   int max_len, split_tokens, n_split;
   float scale_log2;
   uint64_t timeout_ns;
+  PagedKV pk;             // PAGED kernels only (kc, vc are then the page pools)
 };
 
 __device__ __forceinline__ int clamp_len(int n, int max_len) {
@@ -111,7 +117,7 @@ struct DecCfg {
   static_assert(GROUPS >= 1 && TPW % TPI == 0, "stage split");
 };
 
-template <int D, int GT, bool BF16>
+template <int D, int GT, bool BF16, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, DecCfg<D, GT>::MIN_BLOCKS)
 fa_decode_split_kernel(const DecodeParams p) {
   using C = DecCfg<D, GT>;
@@ -161,13 +167,41 @@ fa_decode_split_kernel(const DecodeParams p) {
 
   auto issue = [&](int st) {               // thread 0: fill ring slot st % kDecStages
     const int slot = st % kDecStages;
-    const int n = min(kDecStageTok, t1 - (t0 + st * kDecStageTok));
-    const uint32_t bytes = static_cast<uint32_t>(n) * C::ROW;
-    mbar_arrive_expect_tx(bar_full + 8 * slot, 2 * bytes);
-    bulk_load(sK + slot * C::STAGE_BYTES, kg + static_cast<size_t>(st) * kDecStageTok * D, bytes,
-              bar_full + 8 * slot);
-    bulk_load(sV + slot * C::STAGE_BYTES, vg + static_cast<size_t>(st) * kDecStageTok * D, bytes,
-              bar_full + 8 * slot);
+    const int tok0 = t0 + st * kDecStageTok;
+    const int n = min(kDecStageTok, t1 - tok0);
+    if constexpr (PAGED) {
+      // Tokens [tok0, tok0 + n0) from one page, [tok0 + n0, tok0 + n) from the next.
+      const int ps = 1 << p.pk.page_shift;
+      const int n0 = min(n, ps - (tok0 & (ps - 1)));
+      const int n1 = n - n0;
+      const int e0 = paged_entry(p.pk, b, tok0);
+      const int e1 = n1 > 0 ? paged_entry(p.pk, b, tok0 + n0) : 0;
+      const bool ok0 = static_cast<unsigned>(e0) < static_cast<unsigned>(p.pk.num_pages);
+      const bool ok1 = n1 > 0 && static_cast<unsigned>(e1) < static_cast<unsigned>(p.pk.num_pages);
+      if (!ok0 || (n1 > 0 && !ok1)) atomicCAS(&g_fa_status, 0, kStatusBadPage);
+      const uint32_t b0 = ok0 ? static_cast<uint32_t>(n0) * C::ROW : 0u;
+      const uint32_t b1 = ok1 ? static_cast<uint32_t>(n1) * C::ROW : 0u;
+      mbar_arrive_expect_tx(bar_full + 8 * slot, 2 * (b0 + b1));
+      const size_t page_elems = static_cast<size_t>(ps) * D;
+      if (ok0) {
+        const size_t off = (static_cast<size_t>(e0) * p.Hkv + kvh) * page_elems +
+                           static_cast<size_t>(tok0 & (ps - 1)) * D;
+        bulk_load(sK + slot * C::STAGE_BYTES, p.kc + off, b0, bar_full + 8 * slot);
+        bulk_load(sV + slot * C::STAGE_BYTES, p.vc + off, b0, bar_full + 8 * slot);
+      }
+      if (ok1) {
+        const size_t off = (static_cast<size_t>(e1) * p.Hkv + kvh) * page_elems;
+        bulk_load(sK + slot * C::STAGE_BYTES + n0 * C::ROW, p.kc + off, b1, bar_full + 8 * slot);
+        bulk_load(sV + slot * C::STAGE_BYTES + n0 * C::ROW, p.vc + off, b1, bar_full + 8 * slot);
+      }
+    } else {
+      const uint32_t bytes = static_cast<uint32_t>(n) * C::ROW;
+      mbar_arrive_expect_tx(bar_full + 8 * slot, 2 * bytes);
+      bulk_load(sK + slot * C::STAGE_BYTES, kg + static_cast<size_t>(st) * kDecStageTok * D, bytes,
+                bar_full + 8 * slot);
+      bulk_load(sV + slot * C::STAGE_BYTES, vg + static_cast<size_t>(st) * kDecStageTok * D, bytes,
+                bar_full + 8 * slot);
+    }
   };
   int issued = 0;
   if (threadIdx.x == 0) {

@@ -33,6 +33,12 @@
 // done, a tile before the V slot frees. Tokens of a tile past the split's end are masked
 // to -inf and their V rows zeroed in shared memory (rows of the cache past kv_len are never
 // used, whatever they hold).
+//
+// PAGED = true reads the cache from a page pool (PagedKV in sm100.cuh): a 128-token tile
+// is one box of a page of >= 128 tokens, or 128 / page_size boxes of smaller pages, each
+// landing at its row offset of the swizzled tile (page_size >= 16 keeps every box on a
+// 1 KB swizzle-atom boundary). A box wholly past the split's end is aimed past the pool
+// and reads zeros, so table entries beyond the sequence are never read.
 #pragma once
 
 #include <cuda.h>
@@ -96,6 +102,7 @@ struct DecodeTcParams {
   int max_len, split_tokens, n_split;
   float scale_log2;
   uint64_t timeout_ns;
+  PagedKV pk;             // PAGED kernels only
 };
 
 struct TcUnit {
@@ -179,7 +186,7 @@ __device__ __forceinline__ void tc_unit_from(const DecodeTcParams& p, const TcDe
   w.t1 = min(tc_seq_len(p, d.b), w.t0 + p.split_tokens);
 }
 
-template <bool BF16, int GT>
+template <bool BF16, int GT, bool PAGED>
 __global__ void __launch_bounds__(kTcThreads, 1)
 fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmQ, const DecodeTcParams p) {
@@ -336,6 +343,19 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           const int stg = jg % kTcStages;
           const uint32_t empty = is_k ? bar_kempty(stg) : bar_vempty(stg);
           const uint32_t full = is_k ? bar_kfull(stg) : bar_vfull(stg);
+          // Paged: the tile's table entries, read before the slot wait so that their
+          // latency hides behind it. Box i holds tokens [t + i*rows, t + (i+1)*rows).
+          constexpr int kMaxBoxes = kTcTile / 16;
+          int pg[kMaxBoxes];
+          int rows = kTcTile;
+          if constexpr (PAGED) {
+            rows = min(kTcTile, 1 << p.pk.page_shift);
+#pragma unroll
+            for (int i = 0; i < kMaxBoxes; ++i) {
+              const int tok = t + i * rows;
+              pg[i] = (i * rows < kTcTile && tok < w.t1) ? paged_entry(p.pk, w.b, tok) : 0;
+            }
+          }
           if (jg >= kTcStages && !mbar_wait(empty, ((jg / kTcStages) - 1) & 1, wc)) {
             ok = false;
             break;
@@ -343,7 +363,18 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           if (is_k) FA_TC_EVENT(0, jg); else FA_TC_EVENT(6, jg);
           mbar_arrive_expect_tx(full, kTcTileBytes);
           const uint32_t dst = base + stg * kTcStageBytes + (is_k ? 0 : kTcTileBytes);
-          for (int ch = 0; ch < 2; ++ch) tma_load_3d(dst + ch * kTcChunk, tm, full, ch * 64, t, bhkv);
+          if constexpr (PAGED) {
+            const int y = t & ((1 << p.pk.page_shift) - 1) & ~(kTcTile - 1);   // 0 for small pages
+#pragma unroll
+            for (int i = 0; i < kMaxBoxes; ++i) {
+              if (i * rows >= kTcTile) break;
+              const int z = (t + i * rows < w.t1) ? paged_z(p.pk, pg[i], w.kvh) : paged_z_oob(p.pk);
+              for (int ch = 0; ch < 2; ++ch)
+                tma_load_3d(dst + ch * kTcChunk + i * rows * 128, tm, full, ch * 64, y, z);
+            }
+          } else {
+            for (int ch = 0; ch < 2; ++ch) tma_load_3d(dst + ch * kTcChunk, tm, full, ch * 64, t, bhkv);
+          }
         }
         if (is_k) ticket = static_cast<long long>(gridDim.x) + next_ticket;
       }

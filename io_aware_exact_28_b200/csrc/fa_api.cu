@@ -140,11 +140,16 @@ fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
 // ---------------------------------------------------------------------------------------
 // Forward launch
 // ---------------------------------------------------------------------------------------
-template <int D, bool BF16, bool CAUSAL>
-fa_status launch_fwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const fa::FwdParams& prm, cudaStream_t stream) {
+// K/V maps of one call: the whole cache, and (paged) the last page's used rows.
+struct KVMaps {
+  CUtensorMap k, v, kt, vt;
+};
+
+template <int D, bool BF16, bool CAUSAL, bool PAGED>
+fa_status launch_fwd(int dev, const CUtensorMap& mq, const KVMaps& kv, const fa::FwdParams& prm,
+                     cudaStream_t stream) {
   using C = fa::FwdCfg<D>;
-  auto kernel = fa::fa_fwd_kernel<D, BF16, CAUSAL>;
+  auto kernel = fa::fa_fwd_kernel<D, BF16, CAUSAL, PAGED>;
   static int attr_state[kMaxDevices];   // 0 unknown, 1 ready, 2 unusable build
   {
     std::lock_guard<std::mutex> lock(g_mu);
@@ -166,15 +171,18 @@ fa_status launch_fwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
   // One CTA per work unit (query block of a (batch, head)); running CTAs take over the
   // ones that have not started, so the grid size only bounds the work, not the residency.
   const unsigned n_units = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_qb);
-  kernel<<<n_units, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+  kernel<<<n_units, C::THREADS, C::SMEM_BYTES, stream>>>(mq, kv.k, kv.v, kv.kt, kv.vt, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 template <int D, bool BF16>
-fa_status dispatch_causal(int causal, int dev, const CUtensorMap& mq, const CUtensorMap& mk,
-                          const CUtensorMap& mv, const fa::FwdParams& prm, cudaStream_t st) {
-  return causal ? launch_fwd<D, BF16, true>(dev, mq, mk, mv, prm, st)
-                : launch_fwd<D, BF16, false>(dev, mq, mk, mv, prm, st);
+fa_status dispatch_causal(int causal, bool paged, int dev, const CUtensorMap& mq, const KVMaps& kv,
+                          const fa::FwdParams& prm, cudaStream_t st) {
+  if (paged)
+    return causal ? launch_fwd<D, BF16, true, true>(dev, mq, kv, prm, st)
+                  : launch_fwd<D, BF16, false, true>(dev, mq, kv, prm, st);
+  return causal ? launch_fwd<D, BF16, true, false>(dev, mq, kv, prm, st)
+                : launch_fwd<D, BF16, false, false>(dev, mq, kv, prm, st);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -255,11 +263,11 @@ fa_status launch_combine_pdl(const fa::CombineParams& cp, int B, cudaStream_t st
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D, int GT, bool BF16>
+template <int D, int GT, bool BF16, bool PAGED>
 fa_status launch_decode_t(int dev, const fa::DecodeParams& dp, const fa::CombineParams& cp,
                           int B, int Hkv, int G, cudaStream_t st) {
   using C = fa::DecCfg<D, GT>;
-  auto split_kernel = fa::fa_decode_split_kernel<D, GT, BF16>;
+  auto split_kernel = fa::fa_decode_split_kernel<D, GT, BF16, PAGED>;
   static bool attr_set[kMaxDevices];
   {
     std::lock_guard<std::mutex> lock(g_mu);
@@ -277,21 +285,48 @@ fa_status launch_decode_t(int dev, const fa::DecodeParams& dp, const fa::Combine
   return launch_combine_pdl<D, BF16>(cp, B, st);
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool PAGED>
 fa_status launch_decode_g(int dev, const fa::DecodeParams& dp, const fa::CombineParams& cp,
                           int B, int Hkv, int G, cudaStream_t st) {
-  if (G <= 1) return launch_decode_t<D, 1, BF16>(dev, dp, cp, B, Hkv, G, st);
-  if (G <= 2) return launch_decode_t<D, 2, BF16>(dev, dp, cp, B, Hkv, G, st);
-  if (G <= 4) return launch_decode_t<D, 4, BF16>(dev, dp, cp, B, Hkv, G, st);
-  return launch_decode_t<D, 8, BF16>(dev, dp, cp, B, Hkv, G, st);
+  if (G <= 1) return launch_decode_t<D, 1, BF16, PAGED>(dev, dp, cp, B, Hkv, G, st);
+  if (G <= 2) return launch_decode_t<D, 2, BF16, PAGED>(dev, dp, cp, B, Hkv, G, st);
+  if (G <= 4) return launch_decode_t<D, 4, BF16, PAGED>(dev, dp, cp, B, Hkv, G, st);
+  return launch_decode_t<D, 8, BF16, PAGED>(dev, dp, cp, B, Hkv, G, st);
 }
 
-template <bool BF16, int GT>
+// Paged-cache arguments of one call (host side); see include/fa.h.
+struct PagedArgs {
+  const int* table;
+  int num_pages, page_size, max_pages;
+  fa::PagedKV device(int Hkv) const {
+    fa::PagedKV pk;
+    pk.table = table;
+    pk.max_pages = max_pages;
+    pk.page_shift = 0;
+    while ((1 << pk.page_shift) < page_size) ++pk.page_shift;
+    pk.num_pages = num_pages;
+    pk.Hkv = Hkv;
+    return pk;
+  }
+};
+
+fa_status check_paged(const PagedArgs& pg, int Hkv) {
+  if (!pg.table || pg.num_pages <= 0 || pg.max_pages <= 0 || pg.page_size <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (pg.page_size < 16 || (pg.page_size & (pg.page_size - 1)) != 0) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(pg.max_pages) * pg.page_size >= (1LL << 31) ||
+      static_cast<long long>(pg.num_pages) * Hkv >= (1LL << 31) - 1)
+    return FA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(pg.table) & 3u) return FA_ERR_ALIGNMENT;
+  return FA_OK;
+}
+
+template <bool BF16, int GT, bool PAGED>
 fa_status launch_decode_tc_t(int dev, const void* q, const void* kc, const void* vc,
                            const int* kv_lens, uint8_t* ws, const DecodeLayout& L, int B, int Hq,
                            int Hkv, int max_len, float scale, const fa::CombineParams& cp,
-                           cudaStream_t st) {
-  auto kernel = fa::fa_decode_tc_kernel<BF16, GT>;
+                           const PagedArgs* pg, cudaStream_t st) {
+  auto kernel = fa::fa_decode_tc_kernel<BF16, GT, PAGED>;
   static int sm_count[kMaxDevices];
   {
     std::lock_guard<std::mutex> lock(g_mu);
@@ -307,10 +342,18 @@ fa_status launch_decode_tc_t(int dev, const void* q, const void* kc, const void*
   CUtensorMap mk, mv, mq;
   const long long BHkv = static_cast<long long>(B) * Hkv;
   // q as [1, B*Hq, 128]: 16-row boxes, one per work unit (rows past B*Hq read as zero).
-  if (!make_tile_map(&mk, kc, fa::kTcD, max_len, BHkv, BF16, fa::kTcTile) ||
-      !make_tile_map(&mv, vc, fa::kTcD, max_len, BHkv, BF16, fa::kTcTile) ||
-      !make_tile_map(&mq, q, fa::kTcD, B * Hq, 1, BF16, fa::kTcN))
+  // Paged pools as [num_pages*Hkv, page_size, 128] with boxes of min(page_size, 128) rows.
+  if (PAGED) {
+    const long long heads = static_cast<long long>(pg->num_pages) * Hkv;
+    const int box = pg->page_size < fa::kTcTile ? pg->page_size : fa::kTcTile;
+    if (!make_tile_map(&mk, kc, fa::kTcD, pg->page_size, heads, BF16, box) ||
+        !make_tile_map(&mv, vc, fa::kTcD, pg->page_size, heads, BF16, box))
+      return FA_ERR_CUDA;
+  } else if (!make_tile_map(&mk, kc, fa::kTcD, max_len, BHkv, BF16, fa::kTcTile) ||
+             !make_tile_map(&mv, vc, fa::kTcD, max_len, BHkv, BF16, fa::kTcTile)) {
     return FA_ERR_CUDA;
+  }
+  if (!make_tile_map(&mq, q, fa::kTcD, B * Hq, 1, BF16, fa::kTcN)) return FA_ERR_CUDA;
   fa::DecodeTcParams tp;
   tp.kv_lens = kv_lens;
   tp.tickets = reinterpret_cast<unsigned*>(ws + L.ticket_off);
@@ -327,6 +370,7 @@ fa_status launch_decode_tc_t(int dev, const void* q, const void* kc, const void*
   tp.n_split = L.n_split;
   tp.scale_log2 = scale * 1.4426950408889634f;
   tp.timeout_ns = g_timeout_ns;
+  tp.pk = PAGED ? pg->device(Hkv) : fa::PagedKV{};
   const long long n_units = static_cast<long long>(L.n_split) * B * Hkv * tp.n_gt;
   if (n_units >= (1LL << 31)) return FA_ERR_INVALID_ARG;
   const int grid = static_cast<int>(n_units < sm_count[dev] ? n_units : sm_count[dev]);
@@ -338,15 +382,15 @@ fa_status launch_decode_tc_t(int dev, const void* q, const void* kc, const void*
 }
 
 // Head tile = the smallest of 1, 2, 4, 8, 16 that holds G (16 tiles larger groups).
-template <bool BF16>
+template <bool BF16, bool PAGED>
 fa_status launch_decode_tc(int dev, const void* q, const void* kc, const void* vc,
                            const int* kv_lens, uint8_t* ws, const DecodeLayout& L, int B, int Hq,
                            int Hkv, int max_len, float scale, const fa::CombineParams& cp,
-                           cudaStream_t st) {
+                           const PagedArgs* pg, cudaStream_t st) {
   const int G = Hq / Hkv;
-#define FA_TC_CASE(GT_)                                                                    \
-  return launch_decode_tc_t<BF16, GT_>(dev, q, kc, vc, kv_lens, ws, L, B, Hq, Hkv, max_len, \
-                                       scale, cp, st)
+#define FA_TC_CASE(GT_)                                                                           \
+  return launch_decode_tc_t<BF16, GT_, PAGED>(dev, q, kc, vc, kv_lens, ws, L, B, Hq, Hkv, max_len, \
+                                              scale, cp, pg, st)
   if (G <= 1) FA_TC_CASE(1);
   if (G <= 2) FA_TC_CASE(2);
   if (G <= 4) FA_TC_CASE(4);
@@ -364,14 +408,20 @@ fa_status common_checks(int B, int Hq, int Hkv, int d, float scale, int dtype) {
   return FA_OK;
 }
 
-// fa_fwd and fa_fwd_kvcache: K/V heads hold kv_rows rows in memory, of which Nk are used.
+// fa_fwd, fa_fwd_kvcache and fa_fwd_paged: K/V heads hold kv_rows rows in memory, of which
+// Nk are used; pg != nullptr reads them from a page pool instead.
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                    int Hkv, int Nq, int Nk, long long kv_rows, int d, int causal, float scale,
-                   fa_dtype dtype, void* stream) {
+                   fa_dtype dtype, const PagedArgs* pg, void* stream) {
   if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
   if (Nq <= 0 || Nk <= 0 || (causal != 0 && causal != 1)) return FA_ERR_INVALID_ARG;
   fa_status s = common_checks(B, Hq, Hkv, d, scale, dtype);
   if (s != FA_OK) return s;
+  if (pg) {
+    s = check_paged(*pg, Hkv);
+    if (s != FA_OK) return s;
+    if (static_cast<long long>(pg->max_pages) * pg->page_size < Nk) return FA_ERR_INVALID_ARG;
+  }
   const long long BH = static_cast<long long>(B) * Hq;
   const long long BHkv = static_cast<long long>(B) * Hkv;
   if (BH >= (1LL << 31)) return FA_ERR_INVALID_ARG;
@@ -384,12 +434,27 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   if (s != FA_OK) return s;
 
   const bool bf16 = dtype == FA_BF16;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq;
+  KVMaps kv;
   const int kv_box = (d == 64) ? fa::FwdCfg<64>::BN : fa::FwdCfg<128>::BN;
-  if (!make_tile_map(&mq, q, d, Nq, BH, bf16, fa::kBM) ||
-      !make_tile_map(&mk, k, d, Nk, BHkv, bf16, kv_box, kv_rows) ||
-      !make_tile_map(&mv, v, d, Nk, BHkv, bf16, kv_box, kv_rows))
-    return FA_ERR_CUDA;
+  if (!make_tile_map(&mq, q, d, Nq, BH, bf16, fa::kBM)) return FA_ERR_CUDA;
+  if (pg) {
+    // [num_pages*Hkv, page_size, d] views; the tail maps end at the last page's used rows.
+    const long long heads = static_cast<long long>(pg->num_pages) * Hkv;
+    const int box = pg->page_size < kv_box ? pg->page_size : kv_box;
+    const int tail_rows = Nk - ((Nk - 1) / pg->page_size) * pg->page_size;
+    if (!make_tile_map(&kv.k, k, d, pg->page_size, heads, bf16, box) ||
+        !make_tile_map(&kv.v, v, d, pg->page_size, heads, bf16, box) ||
+        !make_tile_map(&kv.kt, k, d, tail_rows, heads, bf16, box, pg->page_size) ||
+        !make_tile_map(&kv.vt, v, d, tail_rows, heads, bf16, box, pg->page_size))
+      return FA_ERR_CUDA;
+  } else {
+    if (!make_tile_map(&kv.k, k, d, Nk, BHkv, bf16, kv_box, kv_rows) ||
+        !make_tile_map(&kv.v, v, d, Nk, BHkv, bf16, kv_box, kv_rows))
+      return FA_ERR_CUDA;
+    kv.kt = kv.k;
+    kv.vt = kv.v;
+  }
 
   fa::FwdParams prm;
   prm.o = o;
@@ -405,12 +470,15 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.timeout_ns = g_timeout_ns;
   prm.skip_q_load = g_skip_q_load;
+  prm.pk = pg ? pg->device(Hkv) : fa::PagedKV{};
+  prm.last_page = pg ? (Nk - 1) / pg->page_size : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool paged = pg != nullptr;
   if (d == 64)
-    return bf16 ? dispatch_causal<64, true>(causal, dev, mq, mk, mv, prm, st)
-                : dispatch_causal<64, false>(causal, dev, mq, mk, mv, prm, st);
-  return bf16 ? dispatch_causal<128, true>(causal, dev, mq, mk, mv, prm, st)
-              : dispatch_causal<128, false>(causal, dev, mq, mk, mv, prm, st);
+    return bf16 ? dispatch_causal<64, true>(causal, paged, dev, mq, kv, prm, st)
+                : dispatch_causal<64, false>(causal, paged, dev, mq, kv, prm, st);
+  return bf16 ? dispatch_causal<128, true>(causal, paged, dev, mq, kv, prm, st)
+              : dispatch_causal<128, false>(causal, paged, dev, mq, kv, prm, st);
 }
 }  // namespace
 
@@ -419,7 +487,7 @@ extern "C" {
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                  int Hkv, int Nq, int Nk, int d, int causal, float scale, fa_dtype dtype,
                  void* stream) {
-  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, Nk, d, causal, scale, dtype, stream);
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, Nk, d, causal, scale, dtype, nullptr, stream);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -483,7 +551,16 @@ fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* vcache, 
                          int d, int causal, float scale, fa_dtype dtype, void* stream) {
   if (cache_len < Nk || cache_len <= 0) return FA_ERR_INVALID_ARG;
   return fwd_impl(q, kcache, vcache, o, lse, B, Hq, Hkv, Nq, Nk, cache_len, d, causal, scale,
-                  dtype, stream);
+                  dtype, nullptr, stream);
+}
+
+fa_status fa_fwd_paged(const void* q, const void* kpool, const void* vpool, const int* block_table,
+                       void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int num_pages,
+                       int page_size, int max_pages_per_seq, int d, int causal, float scale,
+                       fa_dtype dtype, void* stream) {
+  const PagedArgs pg{block_table, num_pages, page_size, max_pages_per_seq};
+  return fwd_impl(q, kpool, vpool, o, lse, B, Hq, Hkv, Nq, Nk, 0, d, causal, scale, dtype, &pg,
+                  stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq) {
@@ -498,14 +575,23 @@ size_t fa_decode_workspace_bytes(int B, int Hq, int max_kv_len, int d) {
   return L.total;
 }
 
-fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const int* kv_lens,
-                    void* o, float* lse, int B, int Hq, int Hkv, int max_kv_len, int d,
-                    float scale, fa_dtype dtype, void* workspace, size_t workspace_bytes,
-                    void* stream) {
+}  // extern "C"
+
+namespace {
+// fa_decode and fa_decode_paged; pg != nullptr reads the cache from a page pool, whose
+// sequences hold at most max_kv_len = max_pages * page_size tokens.
+fa_status decode_impl(const void* q, const void* kcache, const void* vcache, const int* kv_lens,
+                      void* o, float* lse, int B, int Hq, int Hkv, int max_kv_len, int d,
+                      float scale, fa_dtype dtype, void* workspace, size_t workspace_bytes,
+                      const PagedArgs* pg, void* stream) {
   if (!q || !kcache || !vcache || !kv_lens || !o) return FA_ERR_INVALID_ARG;
   if (max_kv_len <= 0) return FA_ERR_INVALID_ARG;
   fa_status s = common_checks(B, Hq, Hkv, d, scale, dtype);
   if (s != FA_OK) return s;
+  if (pg) {
+    s = check_paged(*pg, Hkv);
+    if (s != FA_OK) return s;
+  }
   if (B > 65535 || static_cast<long long>(B) * Hq >= (1LL << 31)) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o))
     return FA_ERR_ALIGNMENT;
@@ -534,11 +620,17 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
   cp.max_len = max_kv_len;
   cp.split_tokens = L.split_tokens;
   cp.n_split = L.n_split;
-  if (use_tc_decode(d))
-    return bf16 ? launch_decode_tc<true>(dev, q, kcache, vcache, kv_lens, ws, L, B, Hq, Hkv,
-                                         max_kv_len, scale, cp, st)
-                : launch_decode_tc<false>(dev, q, kcache, vcache, kv_lens, ws, L, B, Hq, Hkv,
-                                          max_kv_len, scale, cp, st);
+  if (use_tc_decode(d)) {
+    if (pg)
+      return bf16 ? launch_decode_tc<true, true>(dev, q, kcache, vcache, kv_lens, ws, L, B, Hq, Hkv,
+                                                 max_kv_len, scale, cp, pg, st)
+                  : launch_decode_tc<false, true>(dev, q, kcache, vcache, kv_lens, ws, L, B, Hq,
+                                                  Hkv, max_kv_len, scale, cp, pg, st);
+    return bf16 ? launch_decode_tc<true, false>(dev, q, kcache, vcache, kv_lens, ws, L, B, Hq, Hkv,
+                                                max_kv_len, scale, cp, nullptr, st)
+                : launch_decode_tc<false, false>(dev, q, kcache, vcache, kv_lens, ws, L, B, Hq, Hkv,
+                                                 max_kv_len, scale, cp, nullptr, st);
+  }
   fa::DecodeParams dp;
   dp.q = static_cast<const uint16_t*>(q);
   dp.kc = static_cast<const uint16_t*>(kcache);
@@ -554,11 +646,40 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
   dp.n_split = L.n_split;
   dp.scale_log2 = scale * 1.4426950408889634f;
   dp.timeout_ns = g_timeout_ns;
-  if (d == 64)
-    return bf16 ? launch_decode_g<64, true>(dev, dp, cp, B, Hkv, G, st)
-                : launch_decode_g<64, false>(dev, dp, cp, B, Hkv, G, st);
-  return bf16 ? launch_decode_g<128, true>(dev, dp, cp, B, Hkv, G, st)
-              : launch_decode_g<128, false>(dev, dp, cp, B, Hkv, G, st);
+  dp.pk = pg ? pg->device(Hkv) : fa::PagedKV{};
+#define FA_DEC_CASE(D_, BF_)                                                         \
+  return pg ? launch_decode_g<D_, BF_, true>(dev, dp, cp, B, Hkv, G, st)             \
+            : launch_decode_g<D_, BF_, false>(dev, dp, cp, B, Hkv, G, st)
+  if (d == 64) {
+    if (bf16) FA_DEC_CASE(64, true);
+    FA_DEC_CASE(64, false);
+  }
+  if (bf16) FA_DEC_CASE(128, true);
+  FA_DEC_CASE(128, false);
+#undef FA_DEC_CASE
+}
+}  // namespace
+
+extern "C" {
+
+fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const int* kv_lens,
+                    void* o, float* lse, int B, int Hq, int Hkv, int max_kv_len, int d,
+                    float scale, fa_dtype dtype, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  return decode_impl(q, kcache, vcache, kv_lens, o, lse, B, Hq, Hkv, max_kv_len, d, scale, dtype,
+                     workspace, workspace_bytes, nullptr, stream);
+}
+
+fa_status fa_decode_paged(const void* q, const void* kpool, const void* vpool,
+                          const int* block_table, const int* kv_lens, void* o, float* lse, int B,
+                          int Hq, int Hkv, int num_pages, int page_size, int max_pages_per_seq,
+                          int d, float scale, fa_dtype dtype, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  const PagedArgs pg{block_table, num_pages, page_size, max_pages_per_seq};
+  const long long max_len = static_cast<long long>(max_pages_per_seq) * page_size;
+  if (max_pages_per_seq <= 0 || page_size <= 0 || max_len >= (1LL << 31)) return FA_ERR_INVALID_ARG;
+  return decode_impl(q, kpool, vpool, kv_lens, o, lse, B, Hq, Hkv, static_cast<int>(max_len), d,
+                     scale, dtype, workspace, workspace_bytes, &pg, stream);
 }
 
 }  // extern "C"

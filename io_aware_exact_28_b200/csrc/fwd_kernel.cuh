@@ -24,6 +24,13 @@
 // overwrites the first BN/2 of those columns as packed 16-bit pairs; O_t at
 // [2*BN + t*D, 2*BN + (t+1)*D).
 //
+// PAGED = true reads K and V from a page pool (PagedKV in sm100.cuh) through two map
+// pairs over [num_pages * Hkv, rows, d]: tmK/tmV with rows = page_size, and tmKt/tmVt
+// with rows = the used rows of the sequence's last page, so that pool rows past Nk read
+// as zero exactly as the rows past Nk of a contiguous map do. A key tile is one box of a
+// page of >= BN tokens or BN / page_size boxes of smaller pages; a box wholly past Nk is
+// aimed past the pool (zeros) and its table entry is never read.
+//
 // Lazy rescaling: the running maximum m used in the exponent is only raised when a new
 // tile maximum exceeds it by more than 8 (log2 units). O and l are both accumulated
 // against the same m, so the final O/l and LSE = (m + log2 l) ln 2 are exact in real
@@ -112,6 +119,8 @@ struct FwdParams {
   float scale_log2;     // scale * log2(e)
   uint64_t timeout_ns;
   int skip_q_load;      // test hook
+  PagedKV pk;           // PAGED kernels only
+  int last_page;        // PAGED: page index (t / page_size) of key Nk - 1
 };
 
 template <int D>
@@ -142,10 +151,11 @@ __device__ __forceinline__ void rescale_p_cols(uint32_t taddr, float alpha) {
   tmem_st_wait();
 }
 
-template <int D, bool BF16, bool CAUSAL>
+template <int D, bool BF16, bool CAUSAL, bool PAGED>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::CTAS)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
+              const __grid_constant__ CUtensorMap tmVt, const FwdParams p) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -230,6 +240,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    if (PAGED) {
+      prefetch_tmap(&tmKt);
+      prefetch_tmap(&tmVt);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -267,6 +281,28 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           ++q_loads;
         }
         for (int j = 0; j < w.n_kv && ok; ++j) {
+          // Paged: box i of key tile j holds keys [j*BN + i*rows, j*BN + (i+1)*rows); its
+          // page's table entry is read once for K and V, before the slot waits.
+          constexpr int kMaxBoxes = kBN / 16;
+          int z[kMaxBoxes];
+          int rows = kBN, y = 0;
+          if constexpr (PAGED) {
+            const int ps = 1 << p.pk.page_shift;
+            rows = min(kBN, ps);
+            y = (j * kBN) & (ps - 1) & ~(kBN - 1);   // row of the tile in a large page
+            const int b = w.bh_kv / p.Hkv, kvh = w.bh_kv - b * p.Hkv;
+#pragma unroll
+            for (int i = 0; i < kMaxBoxes; ++i) {
+              const int tok = j * kBN + i * rows;
+              z[i] = (i * rows < kBN && tok < p.Nk) ? paged_entry(p.pk, b, tok) : -1;
+            }
+#pragma unroll
+            for (int i = 0; i < kMaxBoxes; ++i) {
+              const int tok = j * kBN + i * rows;
+              if (i * rows < kBN)
+                z[i] = tok < p.Nk ? paged_z(p.pk, z[i], kvh) : paged_z_oob(p.pk);
+            }
+          }
           for (int kv = 0; kv < 2; ++kv) {
             const int slot = it % C::NS;
             const int round = it / C::NS;
@@ -275,10 +311,22 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               break;
             }
             mbar_arrive_expect_tx(bar_full(slot), C::KV_TILE_BYTES);
-            const CUtensorMap* tm = kv ? &tmV : &tmK;
-            for (int ch = 0; ch < C::NCH; ++ch)
-              tma_load_3d(base + C::KV_OFF + slot * C::KV_TILE_BYTES + ch * C::KV_CHUNK, tm,
-                          bar_full(slot), ch * 64, j * kBN, w.bh_kv);
+            const uint32_t dst = base + C::KV_OFF + slot * C::KV_TILE_BYTES;
+            if constexpr (PAGED) {
+#pragma unroll
+              for (int i = 0; i < kMaxBoxes; ++i) {
+                if (i * rows >= kBN) break;
+                const bool tail = ((j * kBN + i * rows) >> p.pk.page_shift) == p.last_page;
+                const CUtensorMap* tm = kv ? (tail ? &tmVt : &tmV) : (tail ? &tmKt : &tmK);
+                for (int ch = 0; ch < C::NCH; ++ch)
+                  tma_load_3d(dst + ch * C::KV_CHUNK + i * rows * 128, tm, bar_full(slot), ch * 64, y,
+                              z[i]);
+              }
+            } else {
+              const CUtensorMap* tm = kv ? &tmV : &tmK;
+              for (int ch = 0; ch < C::NCH; ++ch)
+                tma_load_3d(dst + ch * C::KV_CHUNK, tm, bar_full(slot), ch * 64, j * kBN, w.bh_kv);
+            }
             ++it;
           }
         }

@@ -219,6 +219,41 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
 
 constexpr uint64_t kDrainNs = 200000000ull;   // 0.2 s limit for abort-path drains
 
+// ---------------------------------------------------------------------------------------
+// Paged KV cache: a pool [num_pages, Hkv, page_size, d] shared by all sequences; token t
+// of sequence b sits in page table[b * max_pages + t / page_size] at row t % page_size.
+// Viewed as [num_pages * Hkv, page_size, d], the (page, KV head) slab is head index
+// page * Hkv + kvh of a TMA map. page_size is a power of two >= 16.
+// ---------------------------------------------------------------------------------------
+struct PagedKV {
+  const int* table;     // [B, max_pages], device
+  int max_pages;        // row stride of the table
+  int page_shift;       // log2(page_size)
+  int num_pages;
+  int Hkv;
+};
+
+constexpr int kStatusBadPage = 1;   // == FA_ERR_INVALID_ARG
+
+// Table entry of the page that holds token `tok` of sequence b (tok below the sequence's
+// length, so the entry is one the caller filled in).
+__device__ __forceinline__ int paged_entry(const PagedKV& pk, int b, int tok) {
+  return __ldg(pk.table + static_cast<size_t>(b) * pk.max_pages + (tok >> pk.page_shift));
+}
+
+// Head index past the pool: a TMA load there reads zeros.
+__device__ __forceinline__ int paged_z_oob(const PagedKV& pk) { return pk.num_pages * pk.Hkv; }
+
+// TMA head index of KV head kvh in pool page `page`. An entry outside the pool is never
+// dereferenced: it maps past the pool (zeros) and is recorded in the status word.
+__device__ __forceinline__ int paged_z(const PagedKV& pk, int page, int kvh) {
+  if (static_cast<unsigned>(page) >= static_cast<unsigned>(pk.num_pages)) {
+    atomicCAS(&g_fa_status, 0, kStatusBadPage);
+    return paged_z_oob(pk);
+  }
+  return page * pk.Hkv + kvh;
+}
+
 // Drain wait used on the abort path: ignores the abort flag, fixed limit.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();

@@ -125,3 +125,31 @@ def test_workspace_size_covers_every_split():
         assert n >= B * Hq * (d + 1) * 4
         assert n % 256 == 0
     assert fa.decode_workspace_bytes(0, 8, 128, 64) == 0
+
+
+def test_paged_entry_points_reject_bad_arguments_without_cuda():
+    L = fa.lib()
+    need = fa.decode_workspace_bytes(2, 8, 16 * 64, 128)
+
+    def dec(q=16, kp=16, vp=16, table=16, lens=16, o=16, B=2, Hq=8, Hkv=2, num_pages=40,
+            page_size=64, max_pages=16, d=128, ws=32, ws_bytes=need):
+        return L.fa_decode_paged(q, kp, vp, table, lens, o, None, B, Hq, Hkv, num_pages, page_size,
+                                 max_pages, d, 0.088, 1, ws, ws_bytes, None)
+
+    def fwd(q=16, kp=16, vp=16, table=16, o=16, Nq=64, Nk=300, num_pages=40, page_size=32,
+            max_pages=10, d=64):
+        return L.fa_fwd_paged(q, kp, vp, table, o, None, 1, 2, 1, Nq, Nk, num_pages, page_size,
+                              max_pages, d, 1, 0.125, 0, None)
+    for call in (dec, fwd):
+        assert call(table=None) == fa.FA_ERR_INVALID_ARG
+        assert call(num_pages=0) == fa.FA_ERR_INVALID_ARG
+        assert call(max_pages=0) == fa.FA_ERR_INVALID_ARG
+        assert call(page_size=48) == fa.FA_ERR_UNSUPPORTED     # not a power of two
+        assert call(page_size=8) == fa.FA_ERR_UNSUPPORTED      # below 16 rows
+        assert call(table=18) == fa.FA_ERR_ALIGNMENT
+        assert call(kp=24) == fa.FA_ERR_ALIGNMENT
+        assert call(num_pages=2**31 - 1) == fa.FA_ERR_INVALID_ARG   # past-the-pool index overflows
+        assert call(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert fwd(Nk=321) == fa.FA_ERR_INVALID_ARG                 # more tokens than the table covers
+    assert dec(ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE
+    assert dec(max_pages=1 << 26) == fa.FA_ERR_INVALID_ARG      # max_pages * page_size >= 2^31
