@@ -37,8 +37,9 @@
 // PAGED = true reads the cache from a page pool (PagedKV in sm100.cuh): a 128-token tile
 // is one box of a page of >= 128 tokens, or 128 / page_size boxes of smaller pages, each
 // landing at its row offset of the swizzled tile (page_size >= 16 keeps every box on a
-// 1 KB swizzle-atom boundary). A box wholly past the split's end is aimed past the pool
-// and reads zeros, so table entries beyond the sequence are never read.
+// 1 KB swizzle-atom boundary). Each producer then runs as a whole warp, lane i handling
+// page i of a tile. A box wholly past the split's end is aimed past the pool and reads
+// zeros, so table entries beyond the sequence are never read.
 #pragma once
 
 #include <cuda.h>
@@ -290,6 +291,7 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 
   if (warp == kTcWarpKProd || warp == kTcWarpVProd) {
     // ---------------------------------------------------------------- TMA producers
+    if constexpr (!PAGED) {
     if (lane == 0) {
       const bool is_k = warp == kTcWarpKProd;
       const CUtensorMap* tm = is_k ? &tmK : &tmV;
@@ -343,19 +345,6 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           const int stg = jg % kTcStages;
           const uint32_t empty = is_k ? bar_kempty(stg) : bar_vempty(stg);
           const uint32_t full = is_k ? bar_kfull(stg) : bar_vfull(stg);
-          // Paged: the tile's table entries, read before the slot wait so that their
-          // latency hides behind it. Box i holds tokens [t + i*rows, t + (i+1)*rows).
-          constexpr int kMaxBoxes = kTcTile / 16;
-          int pg[kMaxBoxes];
-          int rows = kTcTile;
-          if constexpr (PAGED) {
-            rows = min(kTcTile, 1 << p.pk.page_shift);
-#pragma unroll
-            for (int i = 0; i < kMaxBoxes; ++i) {
-              const int tok = t + i * rows;
-              pg[i] = (i * rows < kTcTile && tok < w.t1) ? paged_entry(p.pk, w.b, tok) : 0;
-            }
-          }
           if (jg >= kTcStages && !mbar_wait(empty, ((jg / kTcStages) - 1) & 1, wc)) {
             ok = false;
             break;
@@ -363,18 +352,7 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           if (is_k) FA_TC_EVENT(0, jg); else FA_TC_EVENT(6, jg);
           mbar_arrive_expect_tx(full, kTcTileBytes);
           const uint32_t dst = base + stg * kTcStageBytes + (is_k ? 0 : kTcTileBytes);
-          if constexpr (PAGED) {
-            const int y = t & ((1 << p.pk.page_shift) - 1) & ~(kTcTile - 1);   // 0 for small pages
-#pragma unroll
-            for (int i = 0; i < kMaxBoxes; ++i) {
-              if (i * rows >= kTcTile) break;
-              const int z = (t + i * rows < w.t1) ? paged_z(p.pk, pg[i], w.kvh) : paged_z_oob(p.pk);
-              for (int ch = 0; ch < 2; ++ch)
-                tma_load_3d(dst + ch * kTcChunk + i * rows * 128, tm, full, ch * 64, y, z);
-            }
-          } else {
-            for (int ch = 0; ch < 2; ++ch) tma_load_3d(dst + ch * kTcChunk, tm, full, ch * 64, t, bhkv);
-          }
+          for (int ch = 0; ch < 2; ++ch) tma_load_3d(dst + ch * kTcChunk, tm, full, ch * 64, t, bhkv);
         }
         if (is_k) ticket = static_cast<long long>(gridDim.x) + next_ticket;
       }
@@ -394,6 +372,116 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         if (is_k)
           for (int k = max(0, uc - 2); k < uc; ++k) mbar_wait_drain(bar_qfull(k & 1), (k >> 1) & 1, kDrainNs);
       }
+    }
+    } else {
+    // Paged pool: the whole warp walks the units. Lane 0 does what the contiguous path's
+    // producer does (unit ring, tickets, Q, ring barriers); lane i reads the table entry of
+    // page i of each tile and issues that page's two boxes.
+    const bool leader = lane == 0;
+    const bool is_k = warp == kTcWarpKProd;
+    const CUtensorMap* tm = is_k ? &tmK : &tmV;
+    const int ps = 1 << p.pk.page_shift;
+    const int rows = min(kTcTile, ps);
+    const bool mine = lane * rows < kTcTile;
+    int jg = 0, uc = 0, n = 0;
+    bool ok = true;
+    const TcStart st = *start0;
+    TcCursor cursor = st.cur;
+    long long ticket = blockIdx.x;                   // unit of the CTA's first ticket
+    while (ok) {
+      TcUnit w;
+      if (is_k) {
+        // Publish unit n (or the end) to the other roles.
+        const bool have = ticket < st.total;
+        if (have) cursor.locate(p, ticket, w);
+        if (leader) {
+          if (n >= kTcUnitRing && !mbar_wait(bar_uempty(n), (n / kTcUnitRing - 1) & 1, wc)) {
+            ok = false;
+          } else {
+            ring[n & (kTcUnitRing - 1)] =
+                have ? make_int4(w.b, w.kvh, w.g0, w.split) : make_int4(-1, 0, 0, 0);
+            mbar_arrive(bar_ufull(n));
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        ++n;
+        if (!have) break;
+        // Query rows of the unit (as in the contiguous path), Q buffer uc % 2.
+        const int qb = uc & 1;
+        if (leader) {
+          if (uc >= 2 && !mbar_wait(bar_qempty(qb), ((uc >> 1) - 1) & 1, wc)) {
+            ok = false;
+          } else {
+            mbar_arrive_expect_tx(bar_qfull(qb), kTcQBytes);
+            const int row0 = w.b * p.Hq + w.kvh * p.G + w.g0;
+            for (int ch = 0; ch < 2; ++ch)
+              tma_load_3d(base + kTcOffQ + qb * kTcQBytes + ch * kTcSmallChunk, &tmQ, bar_qfull(qb),
+                          ch * 64, row0, 0);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        ++uc;
+      } else {
+        TcDesc d{0, 0, 0, 0};
+        int got = 1;
+        if (leader) {
+          got = ring_read(n, d) ? 1 : 0;
+          if (got) mbar_arrive(bar_uempty(n));
+        }
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) { ok = false; break; }
+        d.b = __shfl_sync(0xffffffffu, d.b, 0);
+        d.kvh = __shfl_sync(0xffffffffu, d.kvh, 0);
+        d.g0 = __shfl_sync(0xffffffffu, d.g0, 0);
+        d.split = __shfl_sync(0xffffffffu, d.split, 0);
+        ++n;
+        if (d.b < 0) break;
+        tc_unit_from(p, d, w);
+      }
+      unsigned next_ticket = 0;
+      bool asked = false;
+      for (int t = w.t0; t < w.t1; t += kTcTile, ++jg) {
+        // The next ticket is drawn two tiles before this unit's loads end.
+        if (is_k && !asked && t + 2 * kTcTile >= w.t1) {
+          if (leader) next_ticket = atomicAdd(p.tickets, 1u);
+          asked = true;
+        }
+        const int stg = jg % kTcStages;
+        const uint32_t empty = is_k ? bar_kempty(stg) : bar_vempty(stg);
+        const uint32_t full = is_k ? bar_kfull(stg) : bar_vfull(stg);
+        // This lane's page: read before the slot wait so that its latency hides behind it.
+        // A page wholly past the split's end is aimed past the pool (zeros).
+        const int tok = t + lane * rows;
+        const bool used = mine && tok < w.t1;
+        const int entry = used ? paged_entry(p.pk, w.b, tok) : 0;
+        if (leader) {
+          if (jg >= kTcStages && !mbar_wait(empty, ((jg / kTcStages) - 1) & 1, wc))
+            ok = false;
+          else
+            mbar_arrive_expect_tx(full, kTcTileBytes);
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        if (mine) {
+          const uint32_t dst = base + stg * kTcStageBytes + (is_k ? 0 : kTcTileBytes);
+          const int z = used ? paged_z(p.pk, entry, w.kvh) : paged_z_oob(p.pk);
+          const int y = t & (ps - 1) & ~(kTcTile - 1);   // 0 for pages of <= 128 tokens
+          for (int ch = 0; ch < 2; ++ch)
+            tma_load_3d(dst + ch * kTcChunk + lane * rows * 128, tm, full, ch * 64, y, z);
+        }
+      }
+      if (is_k) ticket = static_cast<long long>(gridDim.x) + __shfl_sync(0xffffffffu, next_ticket, 0);
+    }
+    if (leader && (!ok || *abort_flag)) {
+      // Loads still in flight must land before the CTA exits.
+      for (int k = max(0, jg - kTcStages); k < jg; ++k)
+        mbar_wait_drain(is_k ? bar_kfull(k % kTcStages) : bar_vfull(k % kTcStages),
+                        (k / kTcStages) & 1, kDrainNs);
+      if (is_k)
+        for (int k = max(0, uc - 2); k < uc; ++k) mbar_wait_drain(bar_qfull(k & 1), (k >> 1) & 1, kDrainNs);
+    }
     }
   } else if (warp == kTcWarpMma) {
     // ---------------------------------------------------------------- MMA issuer

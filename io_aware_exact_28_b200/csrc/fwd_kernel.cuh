@@ -258,6 +258,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if constexpr (C::REGSPLIT) setmaxnreg_dec<C::REGS_OTHER>();
     if (warp == kWarpProducer) {
     // ------------------------------------------------------------------ TMA producer
+    // Contiguous K/V: lane 0 alone issues every copy (one box per 64 columns of a tile).
+    if constexpr (!PAGED) {
     if (lane == 0) {
       int unit = blockIdx.x, k = 0, it = 0, q_loads = 0;
       bool ok = true, clc_pending = false;
@@ -281,28 +283,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           ++q_loads;
         }
         for (int j = 0; j < w.n_kv && ok; ++j) {
-          // Paged: box i of key tile j holds keys [j*BN + i*rows, j*BN + (i+1)*rows); its
-          // page's table entry is read once for K and V, before the slot waits.
-          constexpr int kMaxBoxes = kBN / 16;
-          int z[kMaxBoxes];
-          int rows = kBN, y = 0;
-          if constexpr (PAGED) {
-            const int ps = 1 << p.pk.page_shift;
-            rows = min(kBN, ps);
-            y = (j * kBN) & (ps - 1) & ~(kBN - 1);   // row of the tile in a large page
-            const int b = w.bh_kv / p.Hkv, kvh = w.bh_kv - b * p.Hkv;
-#pragma unroll
-            for (int i = 0; i < kMaxBoxes; ++i) {
-              const int tok = j * kBN + i * rows;
-              z[i] = (i * rows < kBN && tok < p.Nk) ? paged_entry(p.pk, b, tok) : -1;
-            }
-#pragma unroll
-            for (int i = 0; i < kMaxBoxes; ++i) {
-              const int tok = j * kBN + i * rows;
-              if (i * rows < kBN)
-                z[i] = tok < p.Nk ? paged_z(p.pk, z[i], kvh) : paged_z_oob(p.pk);
-            }
-          }
           for (int kv = 0; kv < 2; ++kv) {
             const int slot = it % C::NS;
             const int round = it / C::NS;
@@ -311,22 +291,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               break;
             }
             mbar_arrive_expect_tx(bar_full(slot), C::KV_TILE_BYTES);
-            const uint32_t dst = base + C::KV_OFF + slot * C::KV_TILE_BYTES;
-            if constexpr (PAGED) {
-#pragma unroll
-              for (int i = 0; i < kMaxBoxes; ++i) {
-                if (i * rows >= kBN) break;
-                const bool tail = ((j * kBN + i * rows) >> p.pk.page_shift) == p.last_page;
-                const CUtensorMap* tm = kv ? (tail ? &tmVt : &tmV) : (tail ? &tmKt : &tmK);
-                for (int ch = 0; ch < C::NCH; ++ch)
-                  tma_load_3d(dst + ch * C::KV_CHUNK + i * rows * 128, tm, bar_full(slot), ch * 64, y,
-                              z[i]);
-              }
-            } else {
-              const CUtensorMap* tm = kv ? &tmV : &tmK;
-              for (int ch = 0; ch < C::NCH; ++ch)
-                tma_load_3d(dst + ch * C::KV_CHUNK, tm, bar_full(slot), ch * 64, j * kBN, w.bh_kv);
-            }
+            const CUtensorMap* tm = kv ? &tmV : &tmK;
+            for (int ch = 0; ch < C::NCH; ++ch)
+              tma_load_3d(base + C::KV_OFF + slot * C::KV_TILE_BYTES + ch * C::KV_CHUNK, tm,
+                          bar_full(slot), ch * 64, j * kBN, w.bh_kv);
             ++it;
           }
         }
@@ -352,6 +320,124 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         if (q_loads > 0) mbar_wait_drain(bar_q(), (q_loads - 1) & 1, kDrainNs);
         if (clc_pending) mbar_wait_drain(bar_clc_full(k & 1), (k >> 1) & 1, kDrainNs);
       }
+    }
+    } else {
+    // The whole warp walks the units. Lane 0 waits on the ring, arms the barriers, loads Q
+    // and takes over CTAs; its decisions reach the other lanes through shuffles. Paged:
+    // lane i reads the table entry of page i of a key tile and issues that page's boxes,
+    // so a tile of small pages costs one table read and NCH boxes per lane.
+    const bool leader = lane == 0;
+    int unit = blockIdx.x, k = 0, it = 0, q_loads = 0;
+    bool ok = true, clc_pending = false;
+    while (true) {
+      const Unit w = decode_unit(unit);
+      // A query tile with no visible key writes zeros and needs no Q.
+      if (!p.skip_q_load && w.n_kv > 0) {
+        if (leader) {
+          // Q is reloaded once the previous unit's S products have all read it.
+          if (q_loads > 0 && !mbar_wait(bar_qempty, (q_loads - 1) & 1, wc)) {
+            ok = false;
+          } else {
+            int q_tiles = 0;
+#pragma unroll
+            for (int t = 0; t < kQTiles; ++t) q_tiles += w.n_t[t] > 0 ? 1 : 0;
+            mbar_arrive_expect_tx(bar_q(), q_tiles * C::Q_TILE_BYTES);
+#pragma unroll
+            for (int t = 0; t < kQTiles; ++t) {
+              if (w.n_t[t] == 0) continue;
+              for (int ch = 0; ch < C::NCH; ++ch)
+                tma_load_3d(base + C::Q_OFF + t * C::Q_TILE_BYTES + ch * C::Q_CHUNK, &tmQ, bar_q(),
+                            ch * 64, w.q0 + t * kBM, w.bh);
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        ++q_loads;
+      }
+      for (int j = 0; j < w.n_kv && ok; ++j) {
+        // Paged: box `lane` of key tile j holds keys [j*BN + lane*rows, +rows). The table
+        // entry is read here and checked after the slot wait, so its latency hides there.
+        int rows = kBN, y = 0, entry = 0, z = 0;
+        bool have = false;
+        if constexpr (PAGED) {
+          const int ps = 1 << p.pk.page_shift;
+          rows = min(kBN, ps);
+          y = (j * kBN) & (ps - 1) & ~(kBN - 1);   // row of the tile in a large page
+          const int b = w.bh_kv / p.Hkv;
+          const int tok = j * kBN + lane * rows;
+          have = lane * rows < kBN && tok < p.Nk;
+          if (have) entry = paged_entry(p.pk, b, tok);
+        }
+        for (int kv = 0; kv < 2; ++kv) {
+          const int slot = it % C::NS;
+          const int round = it / C::NS;
+          if (leader) {
+            if (round > 0 && !mbar_wait(bar_empty(slot), (round - 1) & 1, wc))
+              ok = false;
+            else
+              mbar_arrive_expect_tx(bar_full(slot), C::KV_TILE_BYTES);
+          }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          const uint32_t dst = base + C::KV_OFF + slot * C::KV_TILE_BYTES;
+          if constexpr (PAGED) {
+            if (lane * rows < kBN) {
+              const int tok = j * kBN + lane * rows;
+              if (kv == 0) {   // the page's head index, shared by the K and V boxes
+                const int kvh = w.bh_kv - (w.bh_kv / p.Hkv) * p.Hkv;
+                z = have ? paged_z(p.pk, entry, kvh) : paged_z_oob(p.pk);
+              }
+              const bool tail = have && (tok >> p.pk.page_shift) == p.last_page;
+              const CUtensorMap* tm = kv ? (tail ? &tmVt : &tmV) : (tail ? &tmKt : &tmK);
+              for (int ch = 0; ch < C::NCH; ++ch)
+                tma_load_3d(dst + ch * C::KV_CHUNK + lane * rows * 128, tm, bar_full(slot), ch * 64,
+                            y, z);
+            }
+          } else if (leader) {
+            const CUtensorMap* tm = kv ? &tmV : &tmK;
+            for (int ch = 0; ch < C::NCH; ++ch)
+              tma_load_3d(dst + ch * C::KV_CHUNK, tm, bar_full(slot), ch * 64, j * kBN, w.bh_kv);
+          }
+          ++it;
+        }
+      }
+      if (!ok) break;
+      // All loads of this unit are issued: take over the next CTA that has not started.
+      const int sl = k & 1;
+      int more = 0;
+      uint32_t next = 0;
+      if (leader) {
+        if (k >= 2 && !mbar_wait(bar_clc_empty(sl), ((k >> 1) - 1) & 1, wc)) {
+          ok = false;
+        } else {
+          mbar_arrive_expect_tx(bar_clc_full(sl), 16);
+          clc_try_cancel(clc_resp(sl), bar_clc_full(sl));
+          clc_pending = true;
+          if (!mbar_wait(bar_clc_full(sl), (k >> 1) & 1, wc)) {
+            ok = false;
+          } else {
+            clc_pending = false;
+            more = clc_query(clc_resp(sl), next) ? 1 : 0;
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      more = __shfl_sync(0xffffffffu, more, 0);
+      next = __shfl_sync(0xffffffffu, next, 0);
+      if (!ok) break;
+      ++k;
+      if (!more) break;
+      unit = static_cast<int>(next);
+    }
+    if (leader && (!ok || *abort_flag)) {
+      // Copies still in flight must land before the CTA exits (copies issued by any lane
+      // complete on the same ring barriers).
+      for (int i = max(0, it - C::NS); i < it; ++i)
+        mbar_wait_drain(bar_full(i % C::NS), (i / C::NS) & 1, kDrainNs);
+      if (q_loads > 0) mbar_wait_drain(bar_q(), (q_loads - 1) & 1, kDrainNs);
+      if (clc_pending) mbar_wait_drain(bar_clc_full(k & 1), (k >> 1) & 1, kDrainNs);
+    }
     }
     } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
