@@ -27,7 +27,8 @@ from typing import Optional
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "make_fwd_inputs", "make_decode_inputs",
-           "make_page_table", "paginate", "fwd_flops", "decode_kv_bytes", "torch_dtype"]
+           "make_page_table", "paginate", "make_fp8_inputs", "fwd_flops", "decode_kv_bytes",
+           "torch_dtype"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -104,6 +105,27 @@ def make_decode_inputs(B: int, Hq: int, Hkv: int, cache_len: int, d: int, dtype:
     kc = _randn16(gen, (B, Hkv, cache_len, d), dt)
     vc = _randn16(gen, (B, Hkv, cache_len, d), dt)
     return kv_lens, q, kc, vc
+
+
+def make_fp8_inputs(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, seed: int = 0):
+    """E4M3 Q [B,Hq,Nq,d], K and V [B,Hkv,Nk,d] as uint8 codes, and their descales.
+
+    Q, K, V are drawn as in `make_fwd_inputs` (N(0,1) float32, in that order, chunked along
+    the batch axis), then each tensor is divided by descale = amax / 448 (its largest
+    magnitude lands on the largest finite E4M3 value) and rounded to E4M3 (round to
+    nearest even) by torch's float8_e4m3fn conversion. Returns
+    (q8, k8, v8, q_descale, k_descale, v_descale), CPU tensors and Python floats.
+    """
+    gen = torch.Generator().manual_seed(seed)
+    out = []
+    for shape in ((B, Hq, Nq, d), (B, Hkv, Nk, d), (B, Hkv, Nk, d)):
+        x = torch.empty(shape, dtype=torch.float32)
+        for i in range(shape[0]):
+            x[i] = torch.randn(shape[1:], generator=gen, dtype=torch.float32)
+        descale = float(x.abs().max()) / 448.0
+        out.append(((x / descale).to(torch.float8_e4m3fn).view(torch.uint8), descale))
+    (q8, dq), (k8, dk), (v8, dv) = out
+    return q8, k8, v8, dq, dk, dv
 
 
 def make_page_table(lens, page_size: int, max_pages: int, spare_pages: int = 3, seed: int = 0,
