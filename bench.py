@@ -26,7 +26,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from workloads import (WORKLOADS, decode_kv_bytes, fwd_flops, make_decode_inputs,  # noqa: E402
-                       make_fwd_inputs, make_page_table, paginate)
+                       make_fp8_inputs, make_fwd_inputs, make_page_table, paginate)
 
 METRIC = "attn fwd TFLOP/s & % BF16 TC peak; decode KV-read GB/s & % HBM peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -464,6 +464,18 @@ def run_single_kernel(args):
             for n, i in enumerate(range(0, w.N, C)):
                 fa.fwd_kvcache(qs[n], k, v, min(i + C, w.N), causal=True, scale=w.scale, out=outs[n],
                                return_lse=False)
+    elif args.only == "fwd_fp8":
+        # The workload's shape with E4M3 Q, K, V (fa_fwd_fp8, bf16 output); same causal FLOPs.
+        w = WORKLOADS[args.workload]
+        q8, k8, v8, dq_, dk_, dv_ = make_fp8_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.seed)
+        q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)
+        o = torch.empty(q8.shape, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+        work = fwd_flops(w.B, w.Hq, w.N, w.N, w.d, w.causal) / 1e12
+        unit = "TFLOP/s"
+
+        def call():
+            fa.fwd_fp8(q8, k8, v8, dq_, dk_, dv_, causal=w.causal, scale=w.scale, out=o, lse=lse)
     elif args.only == "fwd_paged":
         # Prefill of the workload with K and V in a page pool (fa_fwd_paged), pages drawn by
         # a seeded random table; same causal FLOPs as --only fwd.
@@ -534,7 +546,8 @@ def run_single_kernel(args):
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("--only", choices=["fwd", "decode", "chunked", "bwd", "fwd_paged", "decode_paged"],
+    ap.add_argument("--only", choices=["fwd", "decode", "chunked", "bwd", "fwd_paged", "decode_paged",
+                                       "fwd_fp8"],
                     default=None,
                     help="launch one entry point alone (profiling helper; prints its own line)")
     ap.add_argument("--gpus", type=int, default=1)

@@ -141,6 +141,28 @@ FA_API fa_status fa_fwd_paged(const void* q, const void* kpool, const void* vpoo
                        int d, int causal, float scale, fa_dtype dtype, void* stream);
 
 /*
+ * fa_fwd_fp8 — fa_fwd with 8-bit (E4M3) Q, K and V and per-tensor descale factors: the
+ * attention of the real-valued tensors q_descale*Q, k_descale*K, v_descale*V.
+ *
+ * Not on the pages as a kernel: the pages discuss lowering precision by quantisation
+ * (page "Empreinte mémoire et calcul des couches Transformer", quantisation bullet: 16 to
+ * 8 bits halves the memory; page "Kotaemon FlashAttention", engineering notes on
+ * quantisation); this applies it to the attention inputs. The method is fa_fwd's, with both products on the 8-bit tensor-core
+ * path and P rounded to E4M3 before P.V (its row sum is taken before rounding).
+ *
+ *   q    [B, Hq,  Nq, d]  E4M3 bytes (OCP FP8 E4M3: bias 7, no infinities, max 448)
+ *   k, v [B, Hkv, Nk, d]  E4M3 bytes
+ *   o    [B, Hq,  Nq, d]  bf16 (written)
+ *   lse  [B, Hq,  Nq]     fp32, natural log, of the descaled scores; may be NULL
+ *   scale, causal         as fa_fwd; q_descale, k_descale, v_descale finite and > 0
+ *
+ * Requirements: those of fa_fwd, with d = 128 only (FA_ERR_UNSUPPORTED otherwise).
+ */
+FA_API fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                     float q_descale, float k_descale, float v_descale, void* stream);
+
+/*
  * fa_bwd_workspace_bytes — bytes of scratch that fa_bwd needs for these sizes.
  */
 FA_API size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq);

@@ -9,7 +9,7 @@ Functions mirror the C ABI in ``include/fa.h``:
 * ``fwd(q, k, v, causal, scale)`` -> ``(o, lse)``   (``fa_fwd``)
 * ``decode(q, kcache, vcache, kv_lens, scale)`` -> ``(o, lse)``   (``fa_decode``)
 * ``decode_workspace_bytes(B, Hq, max_kv_len, d)``   (``fa_decode_workspace_bytes``)
-* ``fwd_kvcache``, ``fwd_paged``, ``decode_paged``, ``decode_noalloc``, ``bwd``
+* ``fwd_kvcache``, ``fwd_paged``, ``decode_paged``, ``decode_noalloc``, ``bwd``, ``fwd_fp8``
 * ``device_status``, ``set_wait_timeout_ns``, ``debug_skip_q_load``, ``build_info``
 """
 from __future__ import annotations
@@ -26,7 +26,7 @@ __all__ = ["FAError", "FALibraryError", "LIB_PATH", "lib", "fwd", "decode",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_ALIGNMENT",
            "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT", "FA_ERR_WORKSPACE", "FA_FP16", "FA_BF16",
            "decode_noalloc", "DECODE_NOALLOC_SCRATCH_BYTES", "fwd_kvcache", "bwd",
-           "bwd_workspace_bytes", "fwd_paged", "decode_paged"]
+           "bwd_workspace_bytes", "fwd_paged", "decode_paged", "fwd_fp8"]
 
 # FA_B200_LIB may name another build of the same library (e.g. a variant for timing).
 LIB_PATH = os.environ.get("FA_B200_LIB") or \
@@ -39,7 +39,7 @@ FA_FP16, FA_BF16 = 0, 1
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_decode", "fa_decode_workspace_bytes", "fa_status_string",
                     "fa_device_status", "fa_set_wait_timeout_ns", "fa_debug_skip_q_load",
                     "fa_build_info", "fa_decode_noalloc", "fa_fwd_kvcache", "fa_bwd",
-                    "fa_bwd_workspace_bytes", "fa_fwd_paged", "fa_decode_paged")
+                    "fa_bwd_workspace_bytes", "fa_fwd_paged", "fa_decode_paged", "fa_fwd_fp8")
 
 # Size of the library's fixed decode scratch (FA_DECODE_NOALLOC_SCRATCH_BYTES in fa.h).
 DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -104,6 +104,8 @@ def lib() -> ctypes.CDLL:
         L.fa_decode_paged.argtypes = [c_void_p] * 7 + [c_int] * 7 + [c_float, c_int, c_void_p,
                                                                      c_size_t, c_void_p]
         L.fa_decode_paged.restype = c_int
+        L.fa_fwd_fp8.argtypes = [c_void_p] * 5 + [c_int] * 7 + [c_float] * 4 + [c_void_p]
+        L.fa_fwd_fp8.restype = c_int
         _lib = L
         return L
 
@@ -307,6 +309,39 @@ def decode_paged(q, kpool, vpool, block_table, kv_lens, scale: Optional[float] =
                                _stream_ptr(stream))
     if st != FA_OK:
         raise FAError(st, "fa_decode_paged")
+    return out, lse
+
+
+def fwd_fp8(q8, k8, v8, q_descale: float, k_descale: float, v_descale: float,
+            causal: bool = False, scale: Optional[float] = None, out=None, lse=None,
+            return_lse: bool = True, stream=None):
+    """Attention of E4M3 inputs via ``fa_fwd_fp8``: q8 [B,Hq,Nq,128], k8, v8 [B,Hkv,Nk,128]
+    as uint8 codes or float8_e4m3fn tensors; the inputs are code x descale per tensor.
+    Returns (o [B,Hq,Nq,128] bf16, lse [B,Hq,Nq] fp32 or None)."""
+    import torch
+    for t, name in ((q8, "q8"), (k8, "k8"), (v8, "v8")):
+        _check(t, name, 4, q8.device)
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+            raise TypeError(f"{name} must hold E4M3 codes (uint8 or float8_e4m3fn)")
+    B, Hq, Nq, d = q8.shape
+    Bk, Hkv, Nk, dk = k8.shape
+    if tuple(v8.shape) != tuple(k8.shape) or Bk != B or dk != d:
+        raise ValueError(f"shape mismatch q{tuple(q8.shape)} k{tuple(k8.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=q8.device)
+    _check(out, "out", 4, q8.device)
+    if out.dtype != torch.bfloat16:
+        raise TypeError("out must be bfloat16")
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q8.device)
+    st = lib().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
+                          lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d,
+                          1 if causal else 0, float(scale), float(q_descale), float(k_descale),
+                          float(v_descale), _stream_ptr(stream))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_fp8")
     return out, lse
 
 

@@ -90,6 +90,23 @@ bool make_tile_map(CUtensorMap* m, const void* ptr, int d, int rows, long long h
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [heads, rows, d] 8-bit (E4M3) view: box = 128 columns (128 bytes) x box_rows rows x 1
+// head, 128-byte swizzle; rows past `rows` read as zero.
+bool make_tile_map8(CUtensorMap* m, const void* ptr, int d, int rows, long long heads,
+                    int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d),
+                                 static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(d)};
+  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------------------
 // Backward launch: D and L * log2(e), then dQ, then dK / dV (stream-ordered).
 // ---------------------------------------------------------------------------------------
@@ -145,11 +162,11 @@ struct KVMaps {
   CUtensorMap k, v, kt, vt;
 };
 
-template <int D, bool BF16, bool CAUSAL, bool PAGED>
+template <int D, bool BF16, bool CAUSAL, bool PAGED, bool FP8 = false>
 fa_status launch_fwd(int dev, const CUtensorMap& mq, const KVMaps& kv, const fa::FwdParams& prm,
                      cudaStream_t stream) {
-  using C = fa::FwdCfg<D>;
-  auto kernel = fa::fa_fwd_kernel<D, BF16, CAUSAL, PAGED>;
+  using C = fa::FwdCfg<D, FP8>;
+  auto kernel = fa::fa_fwd_kernel<D, BF16, CAUSAL, PAGED, FP8>;
   static int attr_state[kMaxDevices];   // 0 unknown, 1 ready, 2 unusable build
   {
     std::lock_guard<std::mutex> lock(g_mu);
@@ -470,6 +487,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.timeout_ns = g_timeout_ns;
   prm.skip_q_load = g_skip_q_load;
+  prm.o_scale = 1.f;
   prm.pk = pg ? pg->device(Hkv) : fa::PagedKV{};
   prm.last_page = pg ? (Nk - 1) / pg->page_size : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -552,6 +570,59 @@ fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* vcache, 
   if (cache_len < Nk || cache_len <= 0) return FA_ERR_INVALID_ARG;
   return fwd_impl(q, kcache, vcache, o, lse, B, Hq, Hkv, Nq, Nk, cache_len, d, causal, scale,
                   dtype, nullptr, stream);
+}
+
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                     float q_descale, float k_descale, float v_descale, void* stream) {
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (Nq <= 0 || Nk <= 0 || (causal != 0 && causal != 1)) return FA_ERR_INVALID_ARG;
+  fa_status s = common_checks(B, Hq, Hkv, d, scale, FA_BF16);
+  if (s != FA_OK) return s;
+  for (float x : {q_descale, k_descale, v_descale})
+    if (!std::isfinite(x) || !(x > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(B) * Hq;
+  const long long BHkv = static_cast<long long>(B) * Hkv;
+  if (BH >= (1LL << 31)) return FA_ERR_INVALID_ARG;
+  const long long n_qb = (Nq + fa::kQTiles * fa::kBM - 1) / (fa::kQTiles * fa::kBM);
+  if (BH * n_qb >= (1LL << 31)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGNMENT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_ALIGNMENT;
+  int dev = 0;
+  s = check_device(&dev);
+  if (s != FA_OK) return s;
+
+  using C8 = fa::FwdCfg<128, true>;
+  CUtensorMap mq;
+  KVMaps kv;
+  if (!make_tile_map8(&mq, q, d, Nq, BH, fa::kBM) ||
+      !make_tile_map8(&kv.k, k, d, Nk, BHkv, C8::BN) ||
+      !make_tile_map8(&kv.v, v, d, Nk, BHkv, C8::BN))
+    return FA_ERR_CUDA;
+  kv.kt = kv.k;
+  kv.vt = kv.v;
+  fa::FwdParams prm;
+  prm.o = o;
+  prm.lse = lse;
+  prm.BH = static_cast<int>(BH);
+  prm.n_qb = static_cast<int>(n_qb);
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.group = Hq / Hkv;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.causal_offset = Nk - Nq;
+  // Scores of the stored values carry the Q and K descales; O carries V's.
+  prm.scale_log2 = scale * q_descale * k_descale * 1.4426950408889634f;
+  prm.timeout_ns = g_timeout_ns;
+  prm.skip_q_load = g_skip_q_load;
+  prm.pk = fa::PagedKV{};
+  prm.last_page = 0;
+  prm.o_scale = v_descale;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return causal ? launch_fwd<128, true, true, false, true>(dev, mq, kv, prm, st)
+                : launch_fwd<128, true, false, false, true>(dev, mq, kv, prm, st);
 }
 
 fa_status fa_fwd_paged(const void* q, const void* kpool, const void* vpool, const int* block_table,

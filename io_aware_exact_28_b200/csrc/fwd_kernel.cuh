@@ -67,20 +67,34 @@ constexpr int kWarpMma = 9;
 //           four Q tiles are in flight per SM and one CTA's prologue/epilogue overlaps the
 //           other's main loop: at d = 64 the per-tile softmax <-> MMA round trip, not any
 //           one pipe, is the limit.
-template <int D>
+//  FP8 (d = 128 only): E4M3 Q, K, V; a row is 128 bytes, so the shared-memory tiles have
+//           the d = 64 geometry (one 128-byte swizzle chunk) and the ring is 8 stages deep;
+//           TMEM, threads and registers are those of d = 128.
+template <int D, bool FP8 = false>
 struct FwdCfg {
+  static constexpr int ELEM = FP8 ? 1 : 2;            // bytes per Q/K/V element
+  static constexpr int ROWB = D * ELEM;               // bytes per Q/K/V row
   static constexpr int BN = (D == 64) ? 64 : 128;     // keys per K/V tile
   static constexpr int CTAS = (D == 64) ? 2 : 1;      // resident CTAs per SM
   // d = 128: 3 warpgroups (warps 10-11 idle) so the register re-split below can apply;
   // d = 64: 10 warps, two CTAs per SM share the register file (96 registers per thread).
   static constexpr int THREADS = (D == 64) ? 320 : 384;
   static constexpr bool REGSPLIT = (D == 128) && FA_REGSPLIT;
-  static constexpr int NCH = D / 64;                  // 128-byte swizzle chunks along d
+  static constexpr int NCH = ROWB / 128;              // 128-byte swizzle chunks along d
+  static constexpr int OCH = D / 64;                  // 64-column chunks of an O row
   static constexpr int Q_CHUNK = kBM * 128;           // 128 rows x 128 bytes
   static constexpr int KV_CHUNK = BN * 128;
-  static constexpr int Q_TILE_BYTES = kBM * D * 2;    // one 128-row tile of Q or O
-  static constexpr int KV_TILE_BYTES = BN * D * 2;
-  static constexpr int NS = (D == 64) ? 8 : 4;        // K/V ring stages
+  static constexpr int Q_TILE_BYTES = kBM * ROWB;     // one 128-row tile of Q
+  static constexpr int KV_TILE_BYTES = BN * ROWB;
+  static constexpr int NS = (D == 64 || FP8) ? 8 : 4; // K/V ring stages
+  // Keys per P.V instruction (32 bytes of K) and TMEM columns of P per 32 scores.
+  static constexpr int KPI = 32 / ELEM;
+  static constexpr int P_COLS32 = 8 * ELEM;
+  // Lazy-rescale threshold (log2 units) and exponent offset: P = 2^(s*c - m + OFF) stays
+  // in (0, 2^(TAU+OFF)]. FP8 keeps P in [2^-6, 2^8] (normal E4M3) for every score within
+  // 10 of the running max, and the offset cancels in O / l.
+  static constexpr float TAU = FP8 ? 4.f : 8.f;
+  static constexpr float OFF = FP8 ? 4.f : 0.f;
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = kQTiles * Q_TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NS * KV_TILE_BYTES;
@@ -103,7 +117,7 @@ struct FwdCfg {
                 "register split");
   static_assert(THREADS * REGS_LAUNCH * CTAS <= 65536, "register file");
   // Which of every 8 consecutive P column pairs use the polynomial exp2 (bit i = pair i).
-  static constexpr uint32_t kEmuPairs = (D == 64) ? FA_EMU_PAIRS_D64 : FA_EMU_PAIRS_D128;
+  static constexpr uint32_t kEmuPairs = FP8 ? 0u : (D == 64) ? FA_EMU_PAIRS_D64 : FA_EMU_PAIRS_D128;
   static_assert(O_COL + kQTiles * D <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES * CTAS <= 227 * 1024, "shared memory budget");
 };
@@ -121,6 +135,7 @@ struct FwdParams {
   int skip_q_load;      // test hook
   PagedKV pk;           // PAGED kernels only
   int last_page;        // PAGED: page index (t / page_size) of key Nk - 1
+  float o_scale;        // FP8 kernels: multiplies O (the descale of V)
 };
 
 template <int D>
@@ -151,12 +166,13 @@ __device__ __forceinline__ void rescale_p_cols(uint32_t taddr, float alpha) {
   tmem_st_wait();
 }
 
-template <int D, bool BF16, bool CAUSAL, bool PAGED>
-__global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::CTAS)
+template <int D, bool BF16, bool CAUSAL, bool PAGED, bool FP8 = false>
+__global__ void __launch_bounds__(FwdCfg<D, FP8>::THREADS, FwdCfg<D, FP8>::CTAS)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
               const __grid_constant__ CUtensorMap tmVt, const FwdParams p) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, FP8>;
+  static_assert(!FP8 || (D == 128 && !PAGED), "FP8: d = 128, contiguous K/V");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -442,26 +458,35 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     } else if (warp == kWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_f16(kBM, kBN, BF16 ? 1u : 0u, 0u, 0u);
-      constexpr uint32_t IDESC_O = idesc_f16(kBM, D, BF16 ? 1u : 0u, 0u, 1u);
+      // Format code: fp16 0 / bf16 1 under kind::f16; E4M3 is code 0 under kind::f8f6f4.
+      constexpr uint32_t FMT = (!FP8 && BF16) ? 1u : 0u;
+      constexpr uint32_t IDESC_S = idesc_f16(kBM, kBN, FMT, 0u, 0u);
+      constexpr uint32_t IDESC_O = idesc_f16(kBM, D, FMT, 0u, 1u);
+      // 32 bytes of K per instruction: d/16 (16-bit) or d/32 (E4M3) instructions per S.
       auto issue_s = [&](int t, int kslot) {
         const uint32_t qa = base + C::Q_OFF + t * C::Q_TILE_BYTES;
         const uint32_t ka = base + C::KV_OFF + kslot * C::KV_TILE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < C::ROWB / 32; ++kk) {
           const uint32_t koff = (kk & 3) * 32;
-          mma_f16_ss(tmem + C::S_COL + t * kBN, sdesc_k_sw128(qa + (kk >> 2) * C::Q_CHUNK + koff),
-                     sdesc_k_sw128(ka + (kk >> 2) * C::KV_CHUNK + koff),
-                     IDESC_S, kk > 0 ? 1u : 0u);
+          const uint64_t da = sdesc_k_sw128(qa + (kk >> 2) * C::Q_CHUNK + koff);
+          const uint64_t db = sdesc_k_sw128(ka + (kk >> 2) * C::KV_CHUNK + koff);
+          if constexpr (FP8) mma_f8_ss(tmem + C::S_COL + t * kBN, da, db, IDESC_S, kk > 0 ? 1u : 0u);
+          else mma_f16_ss(tmem + C::S_COL + t * kBN, da, db, IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
+      // P from TMEM (8 columns = KPI keys per instruction), V rows MN-major from SMEM.
       auto issue_pv = [&](int t, int vslot, bool acc0) {
         const uint32_t va = base + C::KV_OFF + vslot * C::KV_TILE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_f16_ts(tmem + C::O_COL + t * D, tmem + C::S_COL + t * kBN + kk * 8,
-                     sdesc_mn_sw128(va + kk * 2048, C::KV_CHUNK), IDESC_O,
-                     (acc0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kBN / C::KPI; ++kk) {
+          const uint64_t db = sdesc_mn_sw128(va + kk * C::KPI * 128, C::KV_CHUNK);
+          if constexpr (FP8)
+            mma_f8_ts(tmem + C::O_COL + t * D, tmem + C::S_COL + t * kBN + kk * 8, db, IDESC_O,
+                      (acc0 || kk > 0) ? 1u : 0u);
+          else
+            mma_f16_ts(tmem + C::O_COL + t * D, tmem + C::S_COL + t * kBN + kk * 8, db, IDESC_O,
+                       (acc0 || kk > 0) ? 1u : 0u);
         }
       };
       int unit = blockIdx.x, k = 0, it = 0, q_uses = 0;
@@ -597,8 +622,34 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         // packed columns at tS + 16 cc; returns its row sum (unrounded fp32 P). With track,
         // the scores' maximum is gathered in mx8 on the way.
         auto chunk_p = [&](const uint32_t* v, int cc, float mref, bool track) -> float {
-          const uint64_t nm2 = f2_pack(-mref, -mref);
+          const float nm = FP8 ? C::OFF - mref : -mref;
+          const uint64_t nm2 = f2_pack(nm, nm);
           uint64_t l2a = f2_pack(0.f, 0.f), l2b = l2a;
+          if constexpr (FP8) {
+            // 32 scores -> 8 columns of four E4M3 values, one store.
+            uint32_t pk[8];
+            float pp[2];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if (track)
+                mx8[i & 7] = fmax3(mx8[i & 7], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              const uint64_t x2 =
+                  f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2);
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              const uint64_t p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+              if (i & 1) l2b = f2_add(l2b, p2); else l2a = f2_add(l2a, p2);
+              float p0, p1;
+              f2_unpack(p2, p0, p1);
+              if (i & 1) pk[i >> 1] = pack_e4m3x4(pp[0], pp[1], p0, p1);
+              else { pp[0] = p0; pp[1] = p1; }
+            }
+            tmem_st32x32b_x8(tS + cc * C::P_COLS32, pk);
+            float la, lb, lc, ld;
+            f2_unpack(l2a, la, lb);
+            f2_unpack(l2b, lc, ld);
+            return (la + lb) + (lc + ld);
+          }
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {               // 8 packed columns per store
             uint32_t pk[8];
@@ -610,7 +661,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               const uint64_t x2 =
                   f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2);
               uint64_t p2;
-              if (!masked_tile && ((FwdCfg<D>::kEmuPairs >> (i & 7)) & 1u)) {
+              if (!masked_tile && ((C::kEmuPairs >> (i & 7)) & 1u)) {
                 p2 = exp2_poly_f2(x2);
               } else {
                 float x0, x1;
@@ -648,7 +699,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         auto raise_max = [&]() -> bool {
           const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
                                  fmaxf(mx8[6], mx8[7])) * c;
-          const bool grow = mx > m_used + 8.0f;
+          const bool grow = mx > m_used + C::TAU;
           const bool rescale = grow && m_used != -CUDART_INF_F;
           if (__any_sync(0xffffffffu, rescale)) {
             const float alpha = rescale ? ex2_approx(m_used - mx) : 1.0f;
@@ -691,7 +742,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             max_chunk(v);
             const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
                                    fmaxf(mx8[6], mx8[7])) * c;
-            const bool grow = mx > m_used + 8.0f;
+            const bool grow = mx > m_used + C::TAU;
             const bool rescale = grow && m_used != -CUDART_INF_F;
             if (__any_sync(0xffffffffu, rescale)) {
               const float alpha = rescale ? ex2_approx(m_used - mx) : 1.0f;
@@ -730,9 +781,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const bool row_ok = row < p.Nq;
         uint16_t* orow = static_cast<uint16_t*>(p.o) +
                          (static_cast<size_t>(w.bh) * p.Nq + (row_ok ? row : 0)) * D;
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        if constexpr (FP8) inv_l *= p.o_scale;
 #pragma unroll
-        for (int ch = 0; ch < C::NCH; ++ch) {
+        for (int ch = 0; ch < C::OCH; ++ch) {
           uint32_t o[64];
           if (n_t > 0) {
             uint32_t (&o_lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&o[0]);
@@ -755,7 +807,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
         if (row_ok && p.lse != nullptr) {
           p.lse[static_cast<size_t>(w.bh) * p.Nq + row] =
-              (l > 0.f) ? (m_used + __log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
+              (l > 0.f) ? (m_used - C::OFF + __log2f(l)) * 0.69314718055994530942f : -CUDART_INF_F;
         }
       }
       // The next unit: every lane reads the response, then one arrival per warp.

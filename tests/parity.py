@@ -8,6 +8,8 @@ O = 0 and LSE = -inf exactly.
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 MAX_ABS = {"fp16": 4e-3, "bf16": 1.6e-2}
@@ -78,3 +80,52 @@ def sample_rows(N: int, n_random: int, seed: int) -> np.ndarray:
     r = np.random.default_rng(seed).choice(N, size=min(n_random, N), replace=False)
     rows = np.unique(np.concatenate([[x for x in fixed if 0 <= x < N], r]))
     return rows.astype(np.int64)
+
+
+# E4M3 attention (fa_fwd_fp8). The kernel rounds P to E4M3 before P.V; a normal E4M3
+# value carries a relative rounding error of at most 2^-4 (3 mantissa bits, round to
+# nearest), and the kernel keeps P in the normal range for every score within 10 (log2
+# units) of the running maximum. Modelling each rounding error as uniform on
+# [-2^-4, 2^-4] relative and independent, the output error of row i, column c has
+# standard deviation sigma_ic = 2^-4 / sqrt(3) * sqrt(sum_j pi_ij^2 V_jc^2), with pi the
+# exact softmax row. The bound is 6 sigma, plus bf16 output rounding (2^-8 relative) and
+# 2^-12 absolute for the P values below the normal range.
+E4M3_REL = 2.0 ** -4
+FP8_SIGMAS = 6.0
+
+
+def fp8_sigma(Q, K, V, causal: bool, scale: float, rows, Nq: int) -> np.ndarray:
+    """sigma_ic of the rounding model for query rows `rows` of one head (float64 arrays:
+    Q [len(rows), d], K and V [Nk, d])."""
+    from oracle import visible_mask
+    S = scale * (Q @ K.T)
+    vis = visible_mask(np.asarray(rows), Nq, K.shape[0], causal)
+    S = np.where(vis, S, -np.inf)
+    m = S.max(axis=1)
+    has = np.isfinite(m)
+    E = np.zeros_like(S)
+    E[has] = np.exp(S[has] - m[has, None])
+    pi = np.zeros_like(S)
+    pi[has] = E[has] / E[has].sum(axis=1, keepdims=True)
+    return E4M3_REL / math.sqrt(3.0) * np.sqrt((pi ** 2) @ (V ** 2))
+
+
+def assert_close_fp8(o_gpu, lse_gpu, O_ref, L_ref, sigma, what: str = ""):
+    o = to_f64(o_gpu)
+    err = np.abs(o - O_ref)
+    bound = FP8_SIGMAS * sigma + 2.0 ** -8 * np.abs(O_ref) + 2.0 ** -12
+    ratio = float((err / np.maximum(sigma, 1e-30)).max()) if err.size else 0.0
+    assert np.isfinite(o).all(), f"{what}: non-finite output"
+    assert (err <= bound).all(), \
+        f"{what}: {int((err > bound).sum())} outputs past the bound; max err/sigma {ratio:.2f}"
+    if lse_gpu is not None:
+        lg = to_f64(lse_gpu)
+        fin = np.isfinite(L_ref)
+        assert np.array_equal(np.isfinite(lg), fin), f"{what}: -inf pattern of LSE differs"
+        if fin.any():
+            rel = np.abs(lg[fin] - L_ref[fin]) / np.maximum(np.abs(L_ref[fin]), 1.0)
+            assert rel.max() <= LSE_REL, f"{what}: LSE rel {rel.max():.3e}"
+        assert not np.any(np.abs(o[~fin]) > 0), f"{what}: rows without keys must be 0"
+    return {"max_err_over_sigma": ratio, "max_abs": float(err.max()) if err.size else 0.0,
+            "rms": float(np.sqrt(np.mean(err ** 2))) if err.size else 0.0,
+            "rms_sigma": float(np.sqrt(np.mean(sigma ** 2))) if sigma.size else 0.0}

@@ -153,3 +153,19 @@ def test_paged_entry_points_reject_bad_arguments_without_cuda():
     assert fwd(Nk=321) == fa.FA_ERR_INVALID_ARG                 # more tokens than the table covers
     assert dec(ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE
     assert dec(max_pages=1 << 26) == fa.FA_ERR_INVALID_ARG      # max_pages * page_size >= 2^31
+
+
+def test_fwd_fp8_rejects_bad_arguments_without_cuda():
+    L = fa.lib()
+
+    def call(q=16, k=16, v=16, o=16, lse=None, B=1, Hq=2, Hkv=1, Nq=128, Nk=128, d=128, causal=1,
+             scale=0.088, dq=0.01, dk=0.01, dv=0.01):
+        return L.fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, dq, dk, dv, None)
+    assert call(q=None) == fa.FA_ERR_INVALID_ARG
+    assert call(Nk=0) == fa.FA_ERR_INVALID_ARG
+    assert call(Hq=3, Hkv=2) == fa.FA_ERR_INVALID_ARG
+    assert call(dq=0.0) == fa.FA_ERR_INVALID_ARG
+    assert call(dv=float("nan")) == fa.FA_ERR_INVALID_ARG
+    assert call(dk=-1.0) == fa.FA_ERR_INVALID_ARG
+    assert call(d=64) == fa.FA_ERR_UNSUPPORTED        # d = 128 only
+    assert call(v=40) == fa.FA_ERR_ALIGNMENT
