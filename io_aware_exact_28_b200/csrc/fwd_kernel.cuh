@@ -681,6 +681,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           return (la + lb) + (lc + ld);
         };
         // P of the whole row (all chunks; d = 64 loads each chunk from TMEM here).
+        // d = 64: a 32-key chunk past every row limit of the warp (causal diagonal) has
+        // P = 0, stored without loading its scores or evaluating its exponentials
+        // (warp-uniform test). The resident d = 128 path keeps its straight-line chunk
+        // loop: the branch cost it more than the skipped exponentials saved.
+        auto dead_chunk = [&](int cc) -> bool {
+          return masked_tile && __all_sync(0xffffffffu, key0 + 32 * cc > lim);
+        };
+        auto store_zero_p = [&](int cc) {
+          const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int hh = 0; hh < C::P_COLS32 / 8; ++hh) tmem_st32x32b_x8(tS + cc * C::P_COLS32 + hh * 8, z);
+        };
         auto p_pass = [&](float mref, bool track) -> float {
           float sum = 0.f;
 #pragma unroll
@@ -735,6 +747,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           float lsum = 0.f;
 #pragma unroll
           for (int cc = 0; cc < kBN / 32; ++cc) {
+            if (dead_chunk(cc)) {
+              store_zero_p(cc);
+              continue;
+            }
             tmem_ld32x32b_x32(tS + 32 * cc, v);
             mask_chunk(v, cc);
 #pragma unroll
