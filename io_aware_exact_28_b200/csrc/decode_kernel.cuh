@@ -418,20 +418,40 @@ struct CombineParams {
 template <int D, bool BF16>
 __global__ void __launch_bounds__(D)
 fa_decode_combine_kernel(const CombineParams p) {
-  // Launched as a programmatic dependent of the split kernel: wait until it has finished
-  // and its writes are visible.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int bh = blockIdx.x;
   const int b = bh / p.Hq;
   const int e = threadIdx.x;
+  // kv_lens is an input, not a result of the split kernel: read it before the wait.
   const int len = clamp_len(p.kv_lens[b], p.max_len);
   const int ns = (len + p.split_tokens - 1) / p.split_tokens;
   const float* lse_s = p.ws_lse + static_cast<size_t>(bh) * p.n_split;
   const float* o_s = p.ws_o + static_cast<size_t>(bh) * p.n_split * D;
+  // Launched as a programmatic dependent of the split kernel: wait until it has finished
+  // and its writes are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The first kU splits' LSE and partial rows are all requested before any is used (one
+  // round trip); longer split lists continue in a loop.
+  constexpr int kU = 8;
+  float ls[kU], ov[kU];
+#pragma unroll
+  for (int s = 0; s < kU; ++s) {
+    ls[s] = s < ns ? lse_s[s] : -CUDART_INF_F;
+    ov[s] = s < ns ? o_s[static_cast<size_t>(s) * D + e] : 0.f;
+  }
   float M = -CUDART_INF_F;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, lse_s[s]);
+#pragma unroll
+  for (int s = 0; s < kU; ++s) M = fmaxf(M, ls[s]);
+  for (int s = kU; s < ns; ++s) M = fmaxf(M, lse_s[s]);
   float L = 0.f, O = 0.f;
-  for (int s = 0; s < ns; ++s) {
+#pragma unroll
+  for (int s = 0; s < kU; ++s) {
+    if (s < ns) {
+      const float w = ex2_approx(ls[s] - M);
+      L += w;
+      O = fmaf(w, ov[s], O);
+    }
+  }
+  for (int s = kU; s < ns; ++s) {
     const float w = ex2_approx(lse_s[s] - M);
     L += w;
     O = fmaf(w, o_s[static_cast<size_t>(s) * D + e], O);

@@ -15,8 +15,10 @@
 // Persistent CTAs (one per SM), scheduled dynamically. A work unit is one split (up to
 // split_tokens tokens) of one (sequence, KV-head tile); the units that exist (splits
 // before kv_len) are numbered in (sequence, head tile, split) order. CTA c starts with
-// unit c; each further unit is a ticket from an atomic counter in the workspace (zeroed
-// before the launch), so a CTA that streams slower simply takes fewer units. The K
+// unit c; each further unit is a ticket from an atomic counter in the workspace, so a
+// CTA that streams slower simply takes fewer units. The counter is zeroed by a one-thread
+// kernel that this one depends on programmatically: the CTAs start at once, and the
+// ticket taker waits (griddepcontrol.wait) for the zeroing only before its first ticket. The K
 // producer takes the tickets and hands each unit to the other roles through a 4-deep
 // shared-memory ring of unit descriptors. Warps:
 //   0-3  softmax: thread t owns token t of the tile (TMEM lane t of S^T) and row d = t
@@ -187,6 +189,14 @@ __device__ __forceinline__ void tc_unit_from(const DecodeTcParams& p, const TcDe
   w.t1 = min(tc_seq_len(p, d.b), w.t0 + p.split_tokens);
 }
 
+// Zeroes the unit counter of one decode call. The split kernel is its programmatic
+// dependent: it may start once this has begun and waits for the store only before its
+// first ticket.
+__global__ void __launch_bounds__(32) fa_decode_ticket_reset_kernel(unsigned* tickets) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (threadIdx.x == 0) *tickets = 0u;
+}
+
 template <bool BF16, int GT, bool PAGED>
 __global__ void __launch_bounds__(kTcThreads, 1)
 fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -296,7 +306,7 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       const bool is_k = warp == kTcWarpKProd;
       const CUtensorMap* tm = is_k ? &tmK : &tmV;
       int jg = 0, uc = 0, n = 0;
-      bool ok = true;
+      bool ok = true, counter_ready = false;
       const TcStart st = *start0;
       TcCursor cursor = st.cur;
       long long ticket = blockIdx.x;                 // unit of the CTA's first ticket
@@ -339,6 +349,10 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           // The next ticket is drawn two tiles before this unit's loads end: late enough to
           // balance, early enough that its latency hides behind these loads.
           if (is_k && !asked && t + 2 * kTcTile >= w.t1) {
+            if (!counter_ready) {   // the counter is zeroed by the launch this one depends on
+              asm volatile("griddepcontrol.wait;" ::: "memory");
+              counter_ready = true;
+            }
             next_ticket = atomicAdd(p.tickets, 1u);
             asked = true;
           }
@@ -384,7 +398,7 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     const int rows = min(kTcTile, ps);
     const bool mine = lane * rows < kTcTile;
     int jg = 0, uc = 0, n = 0;
-    bool ok = true;
+    bool ok = true, counter_ready = false;
     const TcStart st = *start0;
     TcCursor cursor = st.cur;
     long long ticket = blockIdx.x;                   // unit of the CTA's first ticket
@@ -445,7 +459,13 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       for (int t = w.t0; t < w.t1; t += kTcTile, ++jg) {
         // The next ticket is drawn two tiles before this unit's loads end.
         if (is_k && !asked && t + 2 * kTcTile >= w.t1) {
-          if (leader) next_ticket = atomicAdd(p.tickets, 1u);
+          if (leader) {
+            if (!counter_ready) {   // the counter is zeroed by the launch this one depends on
+              asm volatile("griddepcontrol.wait;" ::: "memory");
+              counter_ready = true;
+            }
+            next_ticket = atomicAdd(p.tickets, 1u);
+          }
           asked = true;
         }
         const int stg = jg % kTcStages;

@@ -391,9 +391,21 @@ fa_status launch_decode_tc_t(int dev, const void* q, const void* kc, const void*
   const long long n_units = static_cast<long long>(L.n_split) * B * Hkv * tp.n_gt;
   if (n_units >= (1LL << 31)) return FA_ERR_INVALID_ARG;
   const int grid = static_cast<int>(n_units < sm_count[dev] ? n_units : sm_count[dev]);
-  // The unit counter starts at zero on every call (stream-ordered).
-  if (cudaMemsetAsync(tp.tickets, 0, sizeof(unsigned), st) != cudaSuccess) return FA_ERR_CUDA;
-  kernel<<<grid, fa::kTcThreads, fa::kTcSmemBytes, st>>>(mk, mv, mq, tp);
+  // The unit counter starts at zero on every call: a one-thread kernel stores the zero,
+  // and the split kernel, its programmatic dependent, overlaps its own start with it.
+  fa::fa_decode_ticket_reset_kernel<<<1, 32, 0, st>>>(tp.tickets);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(fa::kTcThreads, 1, 1);
+  cfg.dynamicSmemBytes = fa::kTcSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, mk, mv, mq, tp) != cudaSuccess) return FA_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   return launch_combine_pdl<fa::kTcD, BF16>(cp, B, st);
 }
