@@ -80,30 +80,41 @@ fa_bwd_preprocess_kernel(const uint16_t* __restrict__ o, const uint16_t* __restr
   }
 }
 
+// Per head-dimension configuration. Each CTA keeps one 128-row tile resident (Q and dO
+// in the dQ kernel, K and V in the dK/dV kernel) and streams the other side in tiles of
+// TN rows. d = 64 streams 64-row tiles, so that TMEM (S | dP | accumulators) fits in 256
+// columns and shared memory in half an SM: two CTAs per SM then overlap one's elementwise
+// step with the other's products (each CTA on its own is serial: products, elementwise,
+// products). d = 128 streams 128-row tiles, one CTA per SM.
 template <int D>
 struct BwdCfg {
+  static constexpr int TN = (D == 64) ? 64 : 128;    // rows of a streamed tile
+  static constexpr int CTAS = (D == 64) ? 2 : 1;     // resident CTAs per SM
   static constexpr int NCH = D / 64;                 // 128-byte swizzle chunks along d
-  static constexpr int CHUNK = kBwdTile * 128;       // 128 rows x 128 bytes
+  static constexpr int CHUNK = kBwdTile * 128;       // resident tile: 128 rows x 128 bytes
+  static constexpr int SCHUNK = TN * 128;            // streamed tile: TN rows x 128 bytes
   static constexpr int TILE_BYTES = kBwdTile * D * 2;
-  static constexpr int NS = (D == 64) ? 8 : 4;       // ring items (one 128-row tile each)
+  static constexpr int STILE_BYTES = TN * D * 2;
+  static constexpr int NS = (D == 64) ? 8 : 4;       // ring items (one streamed tile each)
   static constexpr int A_OFF = 0;                    // dQ: Q, dO;  dK/dV: K, V
   static constexpr int RING_OFF = 2 * TILE_BYTES;
-  static constexpr int VEC_OFF = RING_OFF + NS * TILE_BYTES;   // dK/dV: L and D per ring pair
-  static constexpr int BAR_OFF = VEC_OFF + (NS / 2) * 2 * kBwdTile * 4;
+  static constexpr int VEC_OFF = RING_OFF + NS * STILE_BYTES;  // dK/dV: L and D per ring pair
+  static constexpr int BAR_OFF = VEC_OFF + (NS / 2) * 2 * TN * 4;
   static constexpr int NBARS = 1 + 2 * NS + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
-  static constexpr uint32_t TMEM_COLS = 512;         // S 128 | dP 128 | accumulators
-  static constexpr uint32_t ACC_COL = 256;
-  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static constexpr uint32_t TMEM_COLS = (D == 64) ? 256 : 512;
+  static constexpr uint32_t P_COL = TN;              // dP (dQ kernel) / dP^T (dK/dV kernel)
+  static constexpr uint32_t ACC_COL = 2 * TN;        // dQ, or dV then dK
+  static_assert(SMEM_BYTES * CTAS <= 227 * 1024, "shared memory budget");
   static_assert(ACC_COL + 2 * D <= TMEM_COLS, "TMEM budget");
 };
 
 // ------------------------------------------------------------------------------------
-// dQ: CTA (query tile qt, head bh). TMEM: S [0,128) (dS packed over its first 64
-// columns), dP [128,256), dQ [256, 256+D).
+// dQ: CTA (query tile qt, head bh), key tiles of TN rows. TMEM: S [0,TN) (dS packed
+// over its first TN/2 columns), dP [TN,2TN), dQ [2TN, 2TN+D).
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::CTAS)
 fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                  const BwdParams p) {
@@ -116,12 +127,13 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const int bh = blockIdx.y;
   const int b = bh / p.Hq, h = bh - b * p.Hq;
   const int bh_kv = b * p.Hkv + h / p.group;
+  constexpr int TN = C::TN;
   const int q0 = blockIdx.x * kBwdTile;
-  const int n_kv_total = (p.Nk + kBwdTile - 1) / kBwdTile;
+  const int n_kv_total = (p.Nk + TN - 1) / TN;
   int n_kv = n_kv_total;
   if (CAUSAL) {
     const int kmax = min(q0 + kBwdTile - 1, p.Nq - 1) + p.causal_offset;
-    n_kv = kmax < 0 ? 0 : min(n_kv_total, kmax / kBwdTile + 1);
+    n_kv = kmax < 0 ? 0 : min(n_kv_total, kmax / TN + 1);
   }
 
   const uint32_t bar0 = base + C::BAR_OFF;
@@ -129,7 +141,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   auto bar_full = [&](int i) { return bar0 + 8u * (1 + i); };
   auto bar_empty = [&](int i) { return bar0 + 8u * (1 + C::NS + i); };
   const uint32_t bar_s = bar0 + 8u * (1 + 2 * C::NS);                // S and dP ready
-  const uint32_t bar_ds = bar0 + 8u * (2 + 2 * C::NS);               // dS in TMEM (128)
+  const uint32_t bar_ds = bar0 + 8u * (2 + 2 * C::NS);               // dS in TMEM (128 rows)
   const uint32_t bar_done = bar0 + 8u * (3 + 2 * C::NS);             // every MMA done
   const uint32_t bar_drain = bar0 + 8u * (4 + 2 * C::NS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + C::MISC_OFF);
@@ -169,10 +181,10 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         for (int kv = 0; kv < 2; ++kv) {                // K_j, then V_j
           const int slot = it % C::NS, round = it / C::NS;
           if (round > 0 && !mbar_wait(bar_empty(slot), (round - 1) & 1, wc)) { ok = false; break; }
-          mbar_arrive_expect_tx(bar_full(slot), C::TILE_BYTES);
+          mbar_arrive_expect_tx(bar_full(slot), C::STILE_BYTES);
           for (int ch = 0; ch < C::NCH; ++ch)
-            tma_load_3d(base + C::RING_OFF + slot * C::TILE_BYTES + ch * C::CHUNK, kv ? &tmV : &tmK,
-                        bar_full(slot), ch * 64, j * kBwdTile, bh_kv);
+            tma_load_3d(base + C::RING_OFF + slot * C::STILE_BYTES + ch * C::SCHUNK, kv ? &tmV : &tmK,
+                        bar_full(slot), ch * 64, j * TN, bh_kv);
           ++it;
         }
       }
@@ -185,15 +197,15 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   } else if (warp == kBwdWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_kv > 0) {
-      constexpr uint32_t IDESC_S = idesc_f16(kBwdTile, kBwdTile, BF16 ? 1u : 0u, 0u, 0u);
+      constexpr uint32_t IDESC_S = idesc_f16(kBwdTile, TN, BF16 ? 1u : 0u, 0u, 0u);
       constexpr uint32_t IDESC_Q = idesc_f16(kBwdTile, D, BF16 ? 1u : 0u, 0u, 1u);
-      // X[cols col, +128) = A[128 x D] B[128 x D]^T, both K-major (d contiguous).
+      // X[cols col, +TN) = A[128 x D] B[TN x D]^T, both K-major (d contiguous).
       auto issue_abt = [&](uint32_t col, uint32_t a, uint32_t bt) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk & 3) * 32;
           mma_f16_ss(tmem + col, sdesc_k_sw128(a + (kk >> 2) * C::CHUNK + koff),
-                     sdesc_k_sw128(bt + (kk >> 2) * C::CHUNK + koff), IDESC_S, kk > 0 ? 1u : 0u);
+                     sdesc_k_sw128(bt + (kk >> 2) * C::SCHUNK + koff), IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(bar_a, 0, wc);
@@ -205,19 +217,19 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (!mbar_wait(bar_full(kslot), (kit / C::NS) & 1, wc)) { ok = false; break; }
         if (!mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t ka = base + C::RING_OFF + kslot * C::TILE_BYTES;
-        const uint32_t va = base + C::RING_OFF + vslot * C::TILE_BYTES;
+        const uint32_t ka = base + C::RING_OFF + kslot * C::STILE_BYTES;
+        const uint32_t va = base + C::RING_OFF + vslot * C::STILE_BYTES;
         issue_abt(0, qa, ka);                          // S = Q K_j^T
-        issue_abt(128, doa, va);                       // dP = dO V_j^T
+        issue_abt(C::P_COL, doa, va);                  // dP = dO V_j^T
         issued = true;
         mma_commit(bar_s);
         mma_commit(bar_empty(vslot));                  // V_j no longer needed
         if (!mbar_wait(bar_ds, j & 1, wc)) { ok = false; break; }
         tc_fence_after();
-        // dQ += dS K_j: A = dS (packed 16-bit in TMEM columns [0, 64)), B = K_j MN-major.
+        // dQ += dS K_j: A = dS (packed 16-bit in TMEM columns [0, TN/2)), B = K_j MN-major.
 #pragma unroll
-        for (int kk = 0; kk < kBwdTile / 16; ++kk)
-          mma_f16_ts(tmem + C::ACC_COL, tmem + kk * 8, sdesc_mn_sw128(ka + kk * 2048, C::CHUNK),
+        for (int kk = 0; kk < TN / 16; ++kk)
+          mma_f16_ts(tmem + C::ACC_COL, tmem + kk * 8, sdesc_mn_sw128(ka + kk * 2048, C::SCHUNK),
                      IDESC_Q, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar_empty(kslot));
       }
@@ -229,7 +241,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int r = threadIdx.x;                              // query row of the tile
     const int row = q0 + r;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base, tP = tS + 128, tQ = tS + C::ACC_COL;
+    const uint32_t tS = tmem + lane_base, tP = tS + C::P_COL, tQ = tS + C::ACC_COL;
     const float lse2 = p.lse2[static_cast<size_t>(bh) * p.Nq_pad + row];
     const float dsum = p.dsum[static_cast<size_t>(bh) * p.Nq_pad + row];
     const int lim = CAUSAL ? min(row + p.causal_offset, p.Nk - 1) : p.Nk - 1;
@@ -239,10 +251,10 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     for (int j = 0; j < n_kv; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(bar_s, j & 1, wc))) { ok = false; break; }
       tc_fence_after();
-      const int key0 = j * kBwdTile;
-      const bool masked = key0 + kBwdTile - 1 > lim_min;     // warp-uniform per CTA
+      const int key0 = j * TN;
+      const bool masked = key0 + TN - 1 > lim_min;           // warp-uniform per CTA
 #pragma unroll
-      for (int cc = 0; cc < kBwdTile / 32; ++cc) {
+      for (int cc = 0; cc < TN / 32; ++cc) {
         uint32_t s[32], dp[32];
         tmem_ld32x32b_x32(tS + 32 * cc, s);
         tmem_ld32x32b_x32(tP + 32 * cc, dp);
@@ -304,12 +316,12 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
 // ------------------------------------------------------------------------------------
 // dK, dV: CTA (key tile kt, KV head bh_kv). K and V are loaded once; each step brings
-// Q_i and dO_i of one query tile of one query head of the group (a 2-item ring pair)
-// plus that tile's L * log2(e) and D vectors. TMEM: S^T [0,128) (P^T packed over its
-// first 64 columns), dP^T [128,256) (dS^T packed over its first 64), dV [256, 256+D),
-// dK [256+D, 256+2D).
+// Q_i and dO_i of one TN-row query tile of one query head of the group (a 2-item ring
+// pair) plus that tile's L * log2(e) and D vectors. TMEM: S^T [0,TN) (P^T packed over its
+// first TN/2 columns), dP^T [TN,2TN) (dS^T packed over its first TN/2), dV [2TN, 2TN+D),
+// dK [2TN+D, 2TN+2D).
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::CTAS)
 fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                    const BwdParams p) {
@@ -321,20 +333,21 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh_kv = blockIdx.y;
   const int b = bh_kv / p.Hkv, hk = bh_kv - b * p.Hkv;
+  constexpr int TN = C::TN;
   const int k0 = blockIdx.x * kBwdTile;
-  const int n_q = (p.Nq + kBwdTile - 1) / kBwdTile;
+  const int n_q = (p.Nq + TN - 1) / TN;
   // Query tiles that see any key of this tile: queries i with k0 <= i + offset.
   int q_first = 0;
   if (CAUSAL) {
     const int need = k0 - p.causal_offset;                  // smallest visible query row
-    q_first = need <= 0 ? 0 : min(n_q, need / kBwdTile);
+    q_first = need <= 0 ? 0 : min(n_q, need / TN);
   }
   const int per_head = n_q - q_first;
   const int n_steps = per_head * p.group;                   // (head of the group, tile)
   auto step_of = [&](int s, int& h, int& q0) {
     const int g = s / max(per_head, 1);
     h = hk * p.group + g;
-    q0 = (q_first + (s - g * per_head)) * kBwdTile;
+    q0 = (q_first + (s - g * per_head)) * TN;
   };
 
   const uint32_t bar0 = base + C::BAR_OFF;
@@ -342,7 +355,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   auto bar_full = [&](int i) { return bar0 + 8u * (1 + i); };        // pair slot i (Q, dO, vecs)
   auto bar_empty = [&](int i) { return bar0 + 8u * (1 + C::NS + i); };
   const uint32_t bar_s = bar0 + 8u * (1 + 2 * C::NS);                // S^T and dP^T ready
-  const uint32_t bar_ps = bar0 + 8u * (2 + 2 * C::NS);               // P^T, dS^T in TMEM (128)
+  const uint32_t bar_ps = bar0 + 8u * (2 + 2 * C::NS);               // P^T, dS^T in TMEM (128 rows)
   const uint32_t bar_done = bar0 + 8u * (3 + 2 * C::NS);
   const uint32_t bar_drain = bar0 + 8u * (4 + 2 * C::NS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + C::MISC_OFF);
@@ -368,9 +381,9 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, &g_fa_status, p.timeout_ns};
-  auto q_tile = [&](int slot) { return base + C::RING_OFF + (2 * slot) * C::TILE_BYTES; };
-  auto do_tile = [&](int slot) { return base + C::RING_OFF + (2 * slot + 1) * C::TILE_BYTES; };
-  auto vec = [&](int slot) { return sbase + C::VEC_OFF + slot * 2 * kBwdTile * 4; };
+  auto q_tile = [&](int slot) { return base + C::RING_OFF + (2 * slot) * C::STILE_BYTES; };
+  auto do_tile = [&](int slot) { return base + C::RING_OFF + (2 * slot + 1) * C::STILE_BYTES; };
+  auto vec = [&](int slot) { return sbase + C::VEC_OFF + slot * 2 * TN * 4; };
 
   if (warp == kBwdWarpProd) {
     // ------------------------------------------------------------------ TMA producer
@@ -388,14 +401,14 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         int h, q0;
         step_of(s, h, q0);
         const int bhq = b * p.Hq + h;
-        mbar_arrive_expect_tx(bar_full(slot), 2 * C::TILE_BYTES + 2 * kBwdTile * 4);
+        mbar_arrive_expect_tx(bar_full(slot), 2 * C::STILE_BYTES + 2 * TN * 4);
         for (int ch = 0; ch < C::NCH; ++ch) {
-          tma_load_3d(q_tile(slot) + ch * C::CHUNK, &tmQ, bar_full(slot), ch * 64, q0, bhq);
-          tma_load_3d(do_tile(slot) + ch * C::CHUNK, &tmDO, bar_full(slot), ch * 64, q0, bhq);
+          tma_load_3d(q_tile(slot) + ch * C::SCHUNK, &tmQ, bar_full(slot), ch * 64, q0, bhq);
+          tma_load_3d(do_tile(slot) + ch * C::SCHUNK, &tmDO, bar_full(slot), ch * 64, q0, bhq);
         }
         const size_t vrow = static_cast<size_t>(bhq) * p.Nq_pad + q0;
-        bulk_load(smem_u32(vec(slot)), p.lse2 + vrow, kBwdTile * 4, bar_full(slot));
-        bulk_load(smem_u32(vec(slot) + kBwdTile * 4), p.dsum + vrow, kBwdTile * 4, bar_full(slot));
+        bulk_load(smem_u32(vec(slot)), p.lse2 + vrow, TN * 4, bar_full(slot));
+        bulk_load(smem_u32(vec(slot) + TN * 4), p.dsum + vrow, TN * 4, bar_full(slot));
       }
       if (!ok || *abort_flag) {
         for (int i = max(0, s - NP); i < s; ++i)
@@ -406,21 +419,22 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   } else if (warp == kBwdWarpMma) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_steps > 0) {
-      constexpr uint32_t IDESC_S = idesc_f16(kBwdTile, kBwdTile, BF16 ? 1u : 0u, 0u, 0u);
+      constexpr uint32_t IDESC_S = idesc_f16(kBwdTile, TN, BF16 ? 1u : 0u, 0u, 0u);
       constexpr uint32_t IDESC_G = idesc_f16(kBwdTile, D, BF16 ? 1u : 0u, 0u, 1u);
+      // X[cols col, +TN) = A[128 x D] (resident) B[TN x D]^T (streamed), both K-major.
       auto issue_abt = [&](uint32_t col, uint32_t a, uint32_t bt) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk & 3) * 32;
           mma_f16_ss(tmem + col, sdesc_k_sw128(a + (kk >> 2) * C::CHUNK + koff),
-                     sdesc_k_sw128(bt + (kk >> 2) * C::CHUNK + koff), IDESC_S, kk > 0 ? 1u : 0u);
+                     sdesc_k_sw128(bt + (kk >> 2) * C::SCHUNK + koff), IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
-      // X[acc] += A[128 x 128] (packed 16-bit in TMEM at col a) B[128 x D] (MN-major).
+      // X[acc] += A[128 x TN] (packed 16-bit in TMEM at col a) B[TN x D] (streamed, MN-major).
       auto issue_tb = [&](uint32_t acc, uint32_t a, uint32_t bmn, bool acc0) {
 #pragma unroll
-        for (int kk = 0; kk < kBwdTile / 16; ++kk)
-          mma_f16_ts(tmem + acc, tmem + a + kk * 8, sdesc_mn_sw128(bmn + kk * 2048, C::CHUNK), IDESC_G,
+        for (int kk = 0; kk < TN / 16; ++kk)
+          mma_f16_ts(tmem + acc, tmem + a + kk * 8, sdesc_mn_sw128(bmn + kk * 2048, C::SCHUNK), IDESC_G,
                      (acc0 || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar_a, 0, wc);
@@ -432,13 +446,13 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (!mbar_wait(bar_full(slot), (s / NP) & 1, wc)) { ok = false; break; }
         tc_fence_after();
         issue_abt(0, ka, q_tile(slot));                 // S^T = K Q_i^T
-        issue_abt(128, va, do_tile(slot));              // dP^T = V dO_i^T
+        issue_abt(C::P_COL, va, do_tile(slot));         // dP^T = V dO_i^T
         issued = true;
         mma_commit(bar_s);
         if (!mbar_wait(bar_ps, s & 1, wc)) { ok = false; break; }
         tc_fence_after();
         issue_tb(C::ACC_COL, 0, do_tile(slot), s > 0);          // dV += P^T dO_i
-        issue_tb(C::ACC_COL + D, 128, q_tile(slot), s > 0);     // dK += dS^T Q_i
+        issue_tb(C::ACC_COL + D, C::P_COL, q_tile(slot), s > 0);  // dK += dS^T Q_i
         mma_commit(bar_empty(slot));
       }
       if (issued) mma_commit(ok ? bar_done : bar_drain);
@@ -449,7 +463,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int r = threadIdx.x;                              // key row of the tile
     const int key = k0 + r;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base, tP = tS + 128;
+    const uint32_t tS = tmem + lane_base, tP = tS + C::P_COL;
     const uint32_t tV = tS + C::ACC_COL, tK = tS + C::ACC_COL + D;
     const float c = p.scale_log2;
     bool ok = true;
@@ -462,12 +476,12 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       int h, q0;
       step_of(s, h, q0);
       const float* lv = reinterpret_cast<const float*>(vec(slot));
-      const float* dv = lv + kBwdTile;
+      const float* dv = lv + TN;
       // Key `key` is visible to query q0 + col iff key <= q0 + col + offset.
       const int first_vis = key - p.causal_offset - q0;     // smallest visible column
       const bool masked = CAUSAL && __any_sync(0xffffffffu, first_vis > 0);
 #pragma unroll
-      for (int cc = 0; cc < kBwdTile / 32; ++cc) {
+      for (int cc = 0; cc < TN / 32; ++cc) {
         uint32_t st[32], dpt[32];
         tmem_ld32x32b_x32(tS + 32 * cc, st);
         tmem_ld32x32b_x32(tP + 32 * cc, dpt);

@@ -116,9 +116,15 @@ bool set_smem(K kernel, int bytes) {
          cudaSuccess;
 }
 
+// Tensor maps of the backward pass: 128-row boxes for the tile a CTA keeps resident and
+// TN-row boxes (BwdCfg<D>::TN) for the tiles it streams.
+struct BwdMaps {
+  CUtensorMap q, dout, k, v;          // 128-row boxes
+  CUtensorMap q_s, dout_s, k_s, v_s;  // TN-row boxes
+};
+
 template <int D, bool BF16>
-fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const CUtensorMap& mdo, const void* o, const void* dout, const float* lse,
+fa_status launch_bwd(int dev, const BwdMaps& m, const void* o, const void* dout, const float* lse,
                      void* dq, void* dk, void* dv, fa::BwdParams prm, long long BH, long long BHkv,
                      int n_q, int n_k, int causal, cudaStream_t st) {
   using C = fa::BwdCfg<D>;
@@ -144,13 +150,13 @@ fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
   prm.out = dq;
   prm.out2 = nullptr;
   const dim3 gq(n_q, static_cast<unsigned>(BH));
-  if (causal) dq_c<<<gq, fa::kBwdThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, prm);
-  else dq_n<<<gq, fa::kBwdThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, prm);
+  if (causal) dq_c<<<gq, fa::kBwdThreads, C::SMEM_BYTES, st>>>(m.q, m.k_s, m.v_s, m.dout, prm);
+  else dq_n<<<gq, fa::kBwdThreads, C::SMEM_BYTES, st>>>(m.q, m.k_s, m.v_s, m.dout, prm);
   prm.out = dk;
   prm.out2 = dv;
   const dim3 gk(n_k, static_cast<unsigned>(BHkv));
-  if (causal) kv_c<<<gk, fa::kBwdThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, prm);
-  else kv_n<<<gk, fa::kBwdThreads, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, prm);
+  if (causal) kv_c<<<gk, fa::kBwdThreads, C::SMEM_BYTES, st>>>(m.q_s, m.k, m.v, m.dout_s, prm);
+  else kv_n<<<gk, fa::kBwdThreads, C::SMEM_BYTES, st>>>(m.q_s, m.k, m.v, m.dout_s, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -549,11 +555,16 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   float* lse2 = static_cast<float*>(workspace);
   float* dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                          fa_bwd_workspace_bytes(B, Hq, Nq) / 2);
-  CUtensorMap mq, mk, mv, mdo;
-  if (!make_tile_map(&mq, q, d, Nq, BH, bf16, fa::kBwdTile) ||
-      !make_tile_map(&mdo, dout, d, Nq, BH, bf16, fa::kBwdTile) ||
-      !make_tile_map(&mk, k, d, Nk, BHkv, bf16, fa::kBwdTile) ||
-      !make_tile_map(&mv, v, d, Nk, BHkv, bf16, fa::kBwdTile))
+  BwdMaps mp;
+  const int tn = (d == 64) ? fa::BwdCfg<64>::TN : fa::BwdCfg<128>::TN;
+  if (!make_tile_map(&mp.q, q, d, Nq, BH, bf16, fa::kBwdTile) ||
+      !make_tile_map(&mp.dout, dout, d, Nq, BH, bf16, fa::kBwdTile) ||
+      !make_tile_map(&mp.k, k, d, Nk, BHkv, bf16, fa::kBwdTile) ||
+      !make_tile_map(&mp.v, v, d, Nk, BHkv, bf16, fa::kBwdTile) ||
+      !make_tile_map(&mp.q_s, q, d, Nq, BH, bf16, tn) ||
+      !make_tile_map(&mp.dout_s, dout, d, Nq, BH, bf16, tn) ||
+      !make_tile_map(&mp.k_s, k, d, Nk, BHkv, bf16, tn) ||
+      !make_tile_map(&mp.v_s, v, d, Nk, BHkv, bf16, tn))
     return FA_ERR_CUDA;
   fa::BwdParams prm;
   prm.lse2 = lse2;
@@ -570,10 +581,10 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   prm.timeout_ns = g_timeout_ns;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 64)
-    return bf16 ? launch_bwd<64, true>(dev, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st)
-                : launch_bwd<64, false>(dev, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st);
-  return bf16 ? launch_bwd<128, true>(dev, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st)
-              : launch_bwd<128, false>(dev, mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st);
+    return bf16 ? launch_bwd<64, true>(dev, mp, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st)
+                : launch_bwd<64, false>(dev, mp, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st);
+  return bf16 ? launch_bwd<128, true>(dev, mp, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st)
+              : launch_bwd<128, false>(dev, mp, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st);
 }
 
 fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* vcache, void* o,
