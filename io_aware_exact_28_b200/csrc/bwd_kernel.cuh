@@ -31,9 +31,15 @@
 namespace fa {
 
 constexpr int kBwdTile = 128;          // query rows and key rows per tile
-constexpr int kBwdThreads = 192;       // warps 0-3 elementwise, 4 producer, 5 MMA
-constexpr int kBwdWarpProd = 4;
-constexpr int kBwdWarpMma = 5;
+// TMEM column of the 16-bit operand that one 16-element K step kk of a P.X product reads.
+// With G elementwise groups, group g owns the streamed columns [g*TN/G, (g+1)*TN/G) of S
+// and dP and packs its share of P (or dS) at the start of that range, so K step kk lies in
+// the range of group (16 kk) / (TN/G), at packed column (16 kk - g*TN/G) / 2 past its start.
+template <int TN, int G>
+__device__ __forceinline__ uint32_t packed_col(int kk) {
+  const int g = (16 * kk) / (TN / G);
+  return static_cast<uint32_t>(g * (TN / G) + (16 * kk - g * (TN / G)) / 2);
+}
 
 struct BwdParams {
   const float* lse2;      // [B*Hq, Nq_pad] L * log2(e), +inf where P must be 0
@@ -90,6 +96,14 @@ template <int D>
 struct BwdCfg {
   static constexpr int TN = (D == 64) ? 64 : 128;    // rows of a streamed tile
   static constexpr int CTAS = (D == 64) ? 2 : 1;     // resident CTAs per SM
+  // Elementwise groups of 4 warps (128 rows each), each taking TN/G streamed columns:
+  // two at d = 128 (one CTA per SM), one at d = 64, where a second group measured slower
+  // (two CTAs already share the SM, and registers are capped at 96 per thread).
+  static constexpr int G = (D == 64) ? 1 : 2;
+  static constexpr int EW_THREADS = 128 * G;
+  static constexpr int WARP_PROD = 4 * G;
+  static constexpr int WARP_MMA = 4 * G + 1;
+  static constexpr int THREADS = 32 * (4 * G + 2);
   static constexpr int NCH = D / 64;                 // 128-byte swizzle chunks along d
   static constexpr int CHUNK = kBwdTile * 128;       // resident tile: 128 rows x 128 bytes
   static constexpr int SCHUNK = TN * 128;            // streamed tile: TN rows x 128 bytes
@@ -114,7 +128,7 @@ struct BwdCfg {
 // dQ: CTA (query tile qt, head bh), key tiles of TN rows. TMEM: S [0,TN) (dS packed
 // over its first TN/2 columns), dP [TN,2TN), dQ [2TN, 2TN+D).
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::CTAS)
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, BwdCfg<D>::CTAS)
 fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                  const BwdParams p) {
@@ -154,20 +168,20 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mbar_init(bar_empty(i), 1);
     }
     mbar_init(bar_s, 1);
-    mbar_init(bar_ds, kBwdTile);
+    mbar_init(bar_ds, C::EW_THREADS);
     mbar_init(bar_done, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == kBwdWarpMma) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+  if (warp == C::WARP_MMA) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{abort_flag, &g_fa_status, p.timeout_ns};
 
-  if (warp == kBwdWarpProd) {
+  if (warp == C::WARP_PROD) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && n_kv > 0) {
       mbar_arrive_expect_tx(bar_a, 2 * C::TILE_BYTES);
@@ -194,7 +208,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         mbar_wait_drain(bar_a, 0, kDrainNs);
       }
     }
-  } else if (warp == kBwdWarpMma) {
+  } else if (warp == C::WARP_MMA) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_kv > 0) {
       constexpr uint32_t IDESC_S = idesc_f16(kBwdTile, TN, BF16 ? 1u : 0u, 0u, 0u);
@@ -226,11 +240,11 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         mma_commit(bar_empty(vslot));                  // V_j no longer needed
         if (!mbar_wait(bar_ds, j & 1, wc)) { ok = false; break; }
         tc_fence_after();
-        // dQ += dS K_j: A = dS (packed 16-bit in TMEM columns [0, TN/2)), B = K_j MN-major.
+        // dQ += dS K_j: A = dS (packed 16-bit in TMEM, per elementwise group), B = K_j MN-major.
 #pragma unroll
         for (int kk = 0; kk < TN / 16; ++kk)
-          mma_f16_ts(tmem + C::ACC_COL, tmem + kk * 8, sdesc_mn_sw128(ka + kk * 2048, C::SCHUNK),
-                     IDESC_Q, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_f16_ts(tmem + C::ACC_COL, tmem + packed_col<TN, C::G>(kk),
+                     sdesc_mn_sw128(ka + kk * 2048, C::SCHUNK), IDESC_Q, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar_empty(kslot));
       }
       if (issued) mma_commit(ok ? bar_done : bar_drain);
@@ -238,10 +252,15 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------------ elementwise + epilogue
-    const int r = threadIdx.x;                              // query row of the tile
+    // Group g = warp / 4 takes key columns [g*TN/G, (g+1)*TN/G) of every row; warp w reads
+    // TMEM lanes 32*(w % 4) .. +31, i.e. rows r of the tile.
+    constexpr int G = C::G;
+    const int g = (G == 1) ? 0 : (warp >> 2);
+    const int r = (warp & 3) * 32 + lane;                   // query row of the tile
     const int row = q0 + r;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base, tP = tS + C::P_COL, tQ = tS + C::ACC_COL;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + g * (TN / G), tP = tS + C::P_COL;
+    const uint32_t tQ = tmem + lane_base + C::ACC_COL + g * (D / G);
     const float lse2 = p.lse2[static_cast<size_t>(bh) * p.Nq_pad + row];
     const float dsum = p.dsum[static_cast<size_t>(bh) * p.Nq_pad + row];
     const int lim = CAUSAL ? min(row + p.causal_offset, p.Nk - 1) : p.Nk - 1;
@@ -251,10 +270,10 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     for (int j = 0; j < n_kv; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(bar_s, j & 1, wc))) { ok = false; break; }
       tc_fence_after();
-      const int key0 = j * TN;
-      const bool masked = key0 + TN - 1 > lim_min;           // warp-uniform per CTA
+      const int key0 = j * TN + g * (TN / G);                // first key of this group's columns
+      const bool masked = key0 + TN / G - 1 > lim_min;       // warp-uniform per CTA
 #pragma unroll
-      for (int cc = 0; cc < TN / 32; ++cc) {
+      for (int cc = 0; cc < TN / (32 * G); ++cc) {
         uint32_t s[32], dp[32];
         tmem_ld32x32b_x32(tS + 32 * cc, s);
         tmem_ld32x32b_x32(tP + 32 * cc, dp);
@@ -280,12 +299,13 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (ok && n_kv > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, wc));
     if (ok) {
       tc_fence_after();
-      // dQ = scale * (dS K), rows past Nq skipped; a tile without keys writes zeros.
+      // dQ = scale * (dS K), rows past Nq skipped; a tile without keys writes zeros. Group g
+      // writes columns [g*D/G, (g+1)*D/G) of the row.
       const bool row_ok = row < p.Nq;
       uint16_t* orow = static_cast<uint16_t*>(p.out) +
-                       (static_cast<size_t>(bh) * p.Nq + (row_ok ? row : 0)) * D;
+                       (static_cast<size_t>(bh) * p.Nq + (row_ok ? row : 0)) * D + g * (D / G);
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
+      for (int ch = 0; ch < D / (32 * G); ++ch) {
         uint32_t a[32];
         if (n_kv > 0) {
           tmem_ld32x32b_x32(tQ + 32 * ch, a);
@@ -308,7 +328,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kBwdWarpMma) {
+  if (warp == C::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -321,7 +341,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // first TN/2 columns), dP^T [TN,2TN) (dS^T packed over its first TN/2), dV [2TN, 2TN+D),
 // dK [2TN+D, 2TN+2D).
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(kBwdThreads, BwdCfg<D>::CTAS)
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, BwdCfg<D>::CTAS)
 fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                    const BwdParams p) {
@@ -369,13 +389,13 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(bar_empty(i), 1);
     }
     mbar_init(bar_s, 1);
-    mbar_init(bar_ps, kBwdTile);
+    mbar_init(bar_ps, C::EW_THREADS);
     mbar_init(bar_done, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == kBwdWarpMma) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+  if (warp == C::WARP_MMA) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -385,7 +405,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   auto do_tile = [&](int slot) { return base + C::RING_OFF + (2 * slot + 1) * C::STILE_BYTES; };
   auto vec = [&](int slot) { return sbase + C::VEC_OFF + slot * 2 * TN * 4; };
 
-  if (warp == kBwdWarpProd) {
+  if (warp == C::WARP_PROD) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && n_steps > 0) {
       mbar_arrive_expect_tx(bar_a, 2 * C::TILE_BYTES);
@@ -416,7 +436,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         mbar_wait_drain(bar_a, 0, kDrainNs);
       }
     }
-  } else if (warp == kBwdWarpMma) {
+  } else if (warp == C::WARP_MMA) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_steps > 0) {
       constexpr uint32_t IDESC_S = idesc_f16(kBwdTile, TN, BF16 ? 1u : 0u, 0u, 0u);
@@ -430,12 +450,13 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                      sdesc_k_sw128(bt + (kk >> 2) * C::SCHUNK + koff), IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
-      // X[acc] += A[128 x TN] (packed 16-bit in TMEM at col a) B[TN x D] (streamed, MN-major).
+      // X[acc] += A[128 x TN] (packed 16-bit in TMEM from col a, per elementwise group)
+      // B[TN x D] (streamed, MN-major).
       auto issue_tb = [&](uint32_t acc, uint32_t a, uint32_t bmn, bool acc0) {
 #pragma unroll
         for (int kk = 0; kk < TN / 16; ++kk)
-          mma_f16_ts(tmem + acc, tmem + a + kk * 8, sdesc_mn_sw128(bmn + kk * 2048, C::SCHUNK), IDESC_G,
-                     (acc0 || kk > 0) ? 1u : 0u);
+          mma_f16_ts(tmem + acc, tmem + a + packed_col<TN, C::G>(kk), sdesc_mn_sw128(bmn + kk * 2048, C::SCHUNK),
+                     IDESC_G, (acc0 || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar_a, 0, wc);
       bool issued = false;
@@ -460,11 +481,16 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
   } else {
     // ------------------------------------------------------------------ elementwise + epilogue
-    const int r = threadIdx.x;                              // key row of the tile
+    // Group g = warp / 4 takes query columns [g*TN/G, (g+1)*TN/G) of every key row; warp w
+    // reads TMEM lanes 32*(w % 4) .. +31. In the epilogue, with two groups group 0 writes
+    // dV and group 1 dK; a single group writes both.
+    constexpr int G = C::G;
+    const int g = (G == 1) ? 0 : (warp >> 2);
+    const int r = (warp & 3) * 32 + lane;                   // key row of the tile
     const int key = k0 + r;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_base, tP = tS + C::P_COL;
-    const uint32_t tV = tS + C::ACC_COL, tK = tS + C::ACC_COL + D;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + g * (TN / G), tP = tS + C::P_COL;
+    const uint32_t tV = tmem + lane_base + C::ACC_COL, tK = tV + D;
     const float c = p.scale_log2;
     bool ok = true;
     for (int s = 0; s < n_steps; ++s) {
@@ -481,7 +507,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int first_vis = key - p.causal_offset - q0;     // smallest visible column
       const bool masked = CAUSAL && __any_sync(0xffffffffu, first_vis > 0);
 #pragma unroll
-      for (int cc = 0; cc < TN / 32; ++cc) {
+      for (int cc = 0; cc < TN / (32 * G); ++cc) {
         uint32_t st[32], dpt[32];
         tmem_ld32x32b_x32(tS + 32 * cc, st);
         tmem_ld32x32b_x32(tP + 32 * cc, dpt);
@@ -491,7 +517,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           float pv[2], dsv[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int col = 32 * cc + 2 * i + e;
+            const int col = g * (TN / G) + 32 * cc + 2 * i + e;
             float x = ex2_approx(__uint_as_float(st[2 * i + e]) * c - lv[col]);
             if (masked && col < first_vis) x = 0.f;
             pv[e] = x;
@@ -513,7 +539,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const bool row_ok = key < p.Nk;
       const size_t orow = (static_cast<size_t>(bh_kv) * p.Nk + (row_ok ? key : 0)) * D;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {             // dV, then dK (times scale)
+      for (int which = g; which < 2; which += G) {          // dV, then dK (times scale)
         uint16_t* dst = static_cast<uint16_t*>(which ? p.out : p.out2) + orow;
         const float f = which ? p.scale : 1.0f;
 #pragma unroll
@@ -541,7 +567,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kBwdWarpMma) {
+  if (warp == C::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -150,13 +150,13 @@ fa_status launch_bwd(int dev, const BwdMaps& m, const void* o, const void* dout,
   prm.out = dq;
   prm.out2 = nullptr;
   const dim3 gq(n_q, static_cast<unsigned>(BH));
-  if (causal) dq_c<<<gq, fa::kBwdThreads, C::SMEM_BYTES, st>>>(m.q, m.k_s, m.v_s, m.dout, prm);
-  else dq_n<<<gq, fa::kBwdThreads, C::SMEM_BYTES, st>>>(m.q, m.k_s, m.v_s, m.dout, prm);
+  if (causal) dq_c<<<gq, C::THREADS, C::SMEM_BYTES, st>>>(m.q, m.k_s, m.v_s, m.dout, prm);
+  else dq_n<<<gq, C::THREADS, C::SMEM_BYTES, st>>>(m.q, m.k_s, m.v_s, m.dout, prm);
   prm.out = dk;
   prm.out2 = dv;
   const dim3 gk(n_k, static_cast<unsigned>(BHkv));
-  if (causal) kv_c<<<gk, fa::kBwdThreads, C::SMEM_BYTES, st>>>(m.q_s, m.k, m.v, m.dout_s, prm);
-  else kv_n<<<gk, fa::kBwdThreads, C::SMEM_BYTES, st>>>(m.q_s, m.k, m.v, m.dout_s, prm);
+  if (causal) kv_c<<<gk, C::THREADS, C::SMEM_BYTES, st>>>(m.q_s, m.k, m.v, m.dout_s, prm);
+  else kv_n<<<gk, C::THREADS, C::SMEM_BYTES, st>>>(m.q_s, m.k, m.v, m.dout_s, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
