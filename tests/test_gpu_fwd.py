@@ -204,3 +204,21 @@ def test_long_gqa_workloads_sampled_rows(name):
     # properties at every row: finite, and |O| bounded by max |V| (O is a convex combination)
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
     assert o.float().abs().max() <= v.float().abs().max() + 1e-2
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk,d,dtype,causal", [
+    (8, 12, 12, 1024, 1024, 64, "fp16", False),   # 384 units: every unit has equal tile counts
+    (2, 32, 8, 2048, 2048, 128, "bf16", False),   # 512 units on 148 SMs
+    (8, 12, 12, 1024, 512, 64, "fp16", True),     # early query rows see no key
+    (2, 32, 8, 2048, 1024, 128, "bf16", True),
+])
+def test_more_units_than_resident_ctas(B, Hq, Hkv, Nq, Nk, d, dtype, causal):
+    """More work units than resident CTAs, so running CTAs take over the rest (cluster launch
+    control); sampled rows of the first and last head against the oracle."""
+    q, k, v = make_fwd_inputs(B, Hq, Hkv, Nq, Nk, d, dtype, seed=Nq + Nk + d)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_fwd(q, k, v, causal, scale)
+    rows = sample_rows(Nq, 24, seed=1)
+    for (b, h) in [(0, 0), (B - 1, Hq - 1)]:
+        O, L = attention_rows_f64(q, k, v, causal, scale, b, h, rows)
+        assert_close(o[b, h, rows], lse[b, h, rows], O, L, dtype, f"takeover b{b} h{h}", strict=False)
