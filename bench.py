@@ -404,8 +404,10 @@ def run_ours(args):
                        "frac_of_spec_8000_gbs": dec_bytes / dec_avg_s / 1e9 / 8000.0},
             "roofline": dominant, "rooflines": [roof_fwd, roof_dec],
             "e2e": e2e, "cpu_baseline": cpu,
-            "gpu_launches": K * 3,
-            "gpu_launches_note": f"per step: fa_fwd_kernel + {dec_kernel} + fa_decode_combine_kernel",
+            "gpu_launches": K * (4 if dec_kernel == "fa_decode_tc_kernel" else 3),
+            "gpu_launches_note": (f"per step: fa_fwd_kernel + "
+                                  + ("fa_decode_ticket_reset_kernel + " if dec_kernel == "fa_decode_tc_kernel" else "")
+                                  + f"{dec_kernel} + fa_decode_combine_kernel"),
             "clocks": clocks,
             "device_status": fa.status_string(status),
         }
