@@ -55,30 +55,38 @@ struct BwdParams {
 
 // ------------------------------------------------------------------------------------
 // D_i = sum_d dO_id O_id and L_i * log2(e), padded per head to Nq_pad rows.
-// One warp per row; d = 64 or 128.
+// D/8 threads per row, each loading 16 bytes (8 elements) of O and of dO; the row's
+// partial sums meet by shuffles within its group of lanes. The grid covers
+// BH * Nq_pad * (D/8) threads; lanes past the end only take part in the shuffles.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256)
 fa_bwd_preprocess_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                          const float* __restrict__ lse, float* __restrict__ lse2,
                          float* __restrict__ dsum, int BH, int Nq, int Nq_pad) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= BH * Nq_pad) return;
-  const int bh = warp / Nq_pad, row = warp - bh * Nq_pad;
+  constexpr int TPR = D / 8;                          // threads per row (8 or 16)
+  const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long rowid = gt / TPR;
+  const int sub = static_cast<int>(gt - rowid * TPR);
+  const bool valid = rowid < static_cast<long long>(BH) * Nq_pad;
+  const int bh = valid ? static_cast<int>(rowid / Nq_pad) : 0;
+  const int row = valid ? static_cast<int>(rowid - static_cast<long long>(bh) * Nq_pad) : 0;
   float acc = 0.f;
-  if (row < Nq) {
-    const size_t base = (static_cast<size_t>(bh) * Nq + row) * D;
+  if (valid && row < Nq) {
+    const size_t off = (static_cast<size_t>(bh) * Nq + row) * D + sub * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+    const uint4 g = *reinterpret_cast<const uint4*>(dout + off);
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
-    for (int e = lane * 2; e < D; e += 64) {
+    for (int e = 0; e < 4; ++e) {
       float o0, o1, g0, g1;
-      unpack_half2(*reinterpret_cast<const uint32_t*>(o + base + e), o0, o1, BF16);
-      unpack_half2(*reinterpret_cast<const uint32_t*>(dout + base + e), g0, g1, BF16);
+      unpack_half2(av[e], o0, o1, BF16);
+      unpack_half2(gv[e], g0, g1, BF16);
       acc = fmaf(o0, g0, fmaf(o1, g1, acc));
     }
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
+  for (int m = TPR / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if (valid && sub == 0) {
     const float l = row < Nq ? lse[static_cast<size_t>(bh) * Nq + row] : -CUDART_INF_F;
     lse2[static_cast<size_t>(bh) * Nq_pad + row] =
         (l == -CUDART_INF_F) ? CUDART_INF_F : l * 1.4426950408889634f;

@@ -142,8 +142,8 @@ fa_status launch_bwd(int dev, const BwdMaps& m, const void* o, const void* dout,
       ready[dev] = 1;
     }
   }
-  const long long warps = BH * prm.Nq_pad;
-  fa::fa_bwd_preprocess_kernel<D, BF16><<<static_cast<unsigned>((warps * 32 + 255) / 256), 256, 0, st>>>(
+  const long long threads = BH * prm.Nq_pad * (D / 8);
+  fa::fa_bwd_preprocess_kernel<D, BF16><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(
       static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse,
       const_cast<float*>(prm.lse2), const_cast<float*>(prm.dsum), static_cast<int>(BH), prm.Nq,
       prm.Nq_pad);
