@@ -36,6 +36,24 @@ L2_FLUSH_BYTES = 256 << 20
 MUFU_EX2_PER_CLK_SM = 16.0
 
 
+def max_over_ranks(local_ms, world: int, device):
+    """Per-rank device times (a list of floats) reduced to their maximum over all ranks.
+    Every rank calls this at the same point with the same list length; with one rank it
+    returns the list unchanged. The job is as slow as its slowest rank."""
+    import torch
+    t = torch.tensor([float(x) for x in local_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_rate(world: int, steps: int, work_per_step: float, max_ms: float) -> float:
+    """Whole-job throughput: every rank did `steps` steps of `work_per_step` units (weak
+    scaling, replicas), and the job took the slowest rank's `max_ms`."""
+    return world * steps * work_per_step / (max_ms * 1e-3)
+
+
 def measured_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu capture for (kernel, workload), or None
     if there is none or the kernel sources changed since it was taken."""
@@ -277,16 +295,12 @@ def run_ours(args):
     sampler.stop()
     if world > 1:
         dist.barrier()
-    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
-    dec_ms = sum(e[2].elapsed_time(e[3]) for e in ev)
-    t = torch.tensor([fwd_ms, dec_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    fwd_ms, dec_ms = float(t[0]), float(t[1])
+    fwd_ms, dec_ms = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in ev),
+                                     sum(e[2].elapsed_time(e[3]) for e in ev)], world, dev)
     status = fa.device_status()
 
-    fwd_tflops = world * K * fl / (fwd_ms * 1e-3) / 1e12
-    dec_gbs = world * K * dec_bytes / (dec_ms * 1e-3) / 1e9
+    fwd_tflops = job_rate(world, K, fl, fwd_ms) / 1e12
+    dec_gbs = job_rate(world, K, dec_bytes, dec_ms) / 1e9
     fwd_avg_s = fwd_ms / K * 1e-3
     dec_avg_s = dec_ms / K * 1e-3
     roof_fwd = {"kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": fl / fwd_avg_s / 1e12,
@@ -373,10 +387,8 @@ def run_ours(args):
         s_in.wait_stream(s_cmp)
         s1.record(s_in)
         torch.cuda.synchronize()
-        tt = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * E * fl / (float(tt[0]) * 1e-3) / 1e12, "unit": "TFLOP/s",
+        (e2e_ms,) = max_over_ranks([s0.elapsed_time(s1)], world, dev)
+        e2e = {"value": job_rate(world, E, fl, e2e_ms) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": 2 * (q.numel() + k.numel() + v.numel()),
                "d2h_bytes_per_step": 2 * o.numel() + 4 * lse.numel(), "steps": E,
                "path": "fa.fwd (C ABI fa_fwd) with pinned host buffers; copies on separate "
