@@ -276,7 +276,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, u
 }
 
 // ---------------------------------------------------------------------------------------
-// TMA (tensor) copies. No multicast form is used anywhere in this library.
+// TMA (tensor) copies. Every copy fills only the issuing CTA's own shared memory.
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar,
                                             int c0, int c1, int c2) {
