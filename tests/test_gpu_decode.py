@@ -110,3 +110,29 @@ def test_workspace_reuse_and_determinism():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     O, L = decode_f64(q, kc, vc, kv_lens, w.scale)
     assert_close(o1.cpu(), l1.cpu(), O, L, w.dtype, "reuse", strict=False)
+
+
+def test_many_sequences_every_tail_size():
+    """160 sequences on the d = 128 tensor-core path (562 work units over the 148
+    persistent CTAs) with lengths that give every ragged last-split size (1 to 8 tiles of
+    128 tokens), exact multiples of the 1024-token split, single splits, empty, negative
+    and over-capacity lengths, in a seeded shuffle. Outputs start as NaN, so a unit or a
+    merge that is skipped shows."""
+    B, Hq, Hkv, cache, d = 160, 8, 2, 2304, 128
+    edge = [0, 1, 127, 128, 129, 255, 640, 1000, 1023, 1024, 1025, 1151, 1152, 1153, 1500,
+            2047, 2048, 2049, 2175, 2176, 2303, 2304, -5, 9999]
+    gen = torch.Generator().manual_seed(5)
+    rand = torch.randint(0, cache + 1, (B - len(edge),), generator=gen).tolist()
+    lens = edge + rand
+    lens = [lens[i] for i in torch.randperm(B, generator=gen).tolist()]
+    kv_lens, q, kc, vc = make_decode_inputs(B, Hq, Hkv, cache, d, "bf16", 1, cache, 6,
+                                            kv_lens=torch.tensor(lens))
+    scale = 1.0 / math.sqrt(d)
+    o = torch.full((B, Hq, d), float("nan"), dtype=q.dtype, device=DEV)
+    lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=DEV)
+    fa.decode(q.to(DEV), kc.to(DEV), vc.to(DEV), kv_lens.to(DEV), scale=scale, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert fa.device_status() == fa.FA_OK
+    clamped = torch.tensor([min(max(n, 0), cache) for n in lens])
+    O, L = decode_f64(q, kc, vc, clamped, scale)
+    assert_close(o.cpu(), lse.cpu(), O, L, "bf16", "every tail size", strict=False)
