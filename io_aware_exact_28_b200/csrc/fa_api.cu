@@ -70,10 +70,9 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [heads, rows, d] 16-bit tensor, box = 64 columns (128 bytes) x box_rows rows x 1 head,
-// 128-byte swizzle; rows past `rows` read as zero and are clipped on store.
-// [heads, rows, d] 16-bit view; a head's rows start head_rows rows apart in memory
-// (head_rows >= rows; 0 = rows). Rows past `rows` read as zero.
+// [heads, rows, d] 16-bit view whose heads start head_rows rows apart in memory
+// (head_rows >= rows; 0 means rows). Box = 64 columns (128 bytes) x box_rows rows x 1
+// head, 128-byte swizzle; rows past `rows` read as zero and are clipped on store.
 bool make_tile_map(CUtensorMap* m, const void* ptr, int d, int rows, long long heads, bool bf16,
                    int box_rows, long long head_rows = 0) {
   EncodeTiledFn enc = encode_fn();
