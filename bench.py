@@ -31,6 +31,8 @@ from workloads import (WORKLOADS, decode_kv_bytes, fwd_flops, make_decode_inputs
 METRIC = "attn fwd TFLOP/s & % BF16 TC peak; decode KV-read GB/s & % HBM peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
+L2_NOTE = ("flushed before each step: a 256 MiB write, then a 256 MiB read so that the lines "
+           "left in L2 are clean; decode caches exceed L2")
 # ex2.approx.f32 results per clock per SM, measured on this machine's B200s with a throughput
 # probe (independent chains, 4-32 warps per SM); f16x2/bf16x2 forms give the same rate.
 MUFU_EX2_PER_CLK_SM = 16.0
@@ -70,6 +72,24 @@ def measured_traffic(kernel: str, workload: str):
         return cap["dram_read_bytes"] + cap["dram_write_bytes"]
     except Exception:
         return None
+
+
+def make_l2_flush(dev):
+    """A callable that empties L2 (126 MB) of everything a timed launch could reuse.
+
+    It writes a 256 MiB buffer and then reads another one. The read matters: after the
+    write alone, L2 is full of dirty lines, and whichever timed kernel runs next pays for
+    writing them back (about 19 us of HBM time for a bandwidth-bound kernel). After the
+    read, the lines in L2 are clean and unrelated to the workload."""
+    import torch
+    wbuf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    rbuf = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def flush():
+        wbuf.zero_()
+        rbuf.sum()
+
+    return flush
 
 
 def load_peaks():
@@ -252,7 +272,7 @@ def run_ours(args):
     do = torch.empty_like(dq)
     dlse = torch.empty((wd.B, wd.Hq), dtype=torch.float32, device=dev)
     ws = torch.empty(fa.decode_workspace_bytes(wd.B, wd.Hq, wd.N, wd.d), dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    l2_flush = make_l2_flush(dev)
 
     # Head dimension 128 decodes on the tensor-core split kernel, other sizes on CUDA cores.
     dec_kernel = ("fa_decode_tc_kernel" if wd.d == 128 and os.environ.get("FA_DECODE_CUDA_CORES") != "1"
@@ -269,7 +289,7 @@ def run_ours(args):
         fa.decode(dq, kc, vc, kv_lens, scale=wd.scale, out=do, lse=dlse, workspace=ws)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        l2_flush()
         fwd_call()
         dec_call()
     torch.cuda.synchronize()
@@ -284,7 +304,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     sampler.start()
     for i in range(K):
-        flush.zero_()                 # L2 flush between steps, outside the timed events
+        l2_flush()                    # L2 flush between steps, outside the timed events
         ev[i][0].record()
         fwd_call()
         ev[i][1].record()
@@ -405,7 +425,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.describe(), "decode_workload": wd.describe(),
-                       "l2": "flushed (256 MiB write) before each step; decode caches exceed L2",
+                       "l2": L2_NOTE,
                        "parallelism": "replicas" if world > 1 else "single GPU",
                        "value_is": "forward TFLOP/s, causal-adjusted algorithmic FLOPs"},
             "fwd": {"tflops": fwd_tflops, "ms_per_launch": fwd_ms / K,
@@ -535,14 +555,14 @@ def run_single_kernel(args):
 
         def call():
             fa.decode(dq, kc, vc, kv_lens, scale=w.scale, out=do, lse=dlse, workspace=ws)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    l2_flush = make_l2_flush(dev)
     for _ in range(args.warmup):
-        flush.zero_()
+        l2_flush()
         call()
     torch.cuda.synchronize()
     ms = []
     for _ in range(args.steps):
-        flush.zero_()
+        l2_flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         call()
