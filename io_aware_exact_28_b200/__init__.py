@@ -154,6 +154,25 @@ def _check(t, name: str, ndim: int, device) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
+def _check_buf(t, name: str, shape, dtype, device) -> None:
+    """A caller-supplied tensor whose size the kernels trust (an output, the LSE input of
+    the backward pass): exact shape and dtype, on `device`, contiguous."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    _check(t, name, len(shape), device)
+
+
+def _check_workspace(ws, device) -> None:
+    """Scratch passed by the caller: device memory on `device`, contiguous (its byte size
+    is passed on and checked by the library)."""
+    if not ws.is_cuda or ws.device != device:
+        raise ValueError(f"workspace must be a CUDA tensor on {device}")
+    if not ws.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+
+
 def _stream_ptr(stream) -> int:
     import torch
     s = stream if stream is not None else torch.cuda.current_stream()
@@ -182,11 +201,11 @@ def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, 
     if out is None:
         out = torch.empty_like(q)
     else:
-        _check(out, "out", 4, q.device)
+        _check_buf(out, "out", q.shape, q.dtype, q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     elif lse is not None:
-        _check(lse, "lse", 3, q.device)
+        _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q.device)
     st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                       lse.data_ptr() if lse is not None else None,
                       B, Hq, Hkv, Nq, Nk, d, 1 if causal else 0, float(scale), _dtype_code(q),
@@ -217,11 +236,11 @@ def fwd_kvcache(q, kcache, vcache, nk: int, causal: bool = True, scale: Optional
     if out is None:
         out = torch.empty_like(q)
     else:
-        _check(out, "out", 4, q.device)
+        _check_buf(out, "out", q.shape, q.dtype, q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     elif lse is not None:
-        _check(lse, "lse", 3, q.device)
+        _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q.device)
     st = lib().fa_fwd_kvcache(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), out.data_ptr(),
                               lse.data_ptr() if lse is not None else None,
                               B, Hq, Hkv, Nq, int(nk), cache_len, d, 1 if causal else 0,
@@ -261,12 +280,14 @@ def fwd_paged(q, kpool, vpool, block_table, nk: int, causal: bool = True,
     num_pages, Hkv, page_size, _ = kpool.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    out = torch.empty_like(q) if out is None else out
-    _check(out, "out", 4, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_buf(out, "out", q.shape, q.dtype, q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     elif lse is not None:
-        _check(lse, "lse", 3, q.device)
+        _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q.device)
     st = lib().fa_fwd_paged(q.data_ptr(), kpool.data_ptr(), vpool.data_ptr(),
                             block_table.data_ptr(), out.data_ptr(),
                             lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, int(nk),
@@ -295,12 +316,19 @@ def decode_paged(q, kpool, vpool, block_table, kv_lens, scale: Optional[float] =
     max_pages = block_table.shape[1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    out = torch.empty_like(q) if out is None else out
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_buf(out, "out", q.shape, q.dtype, q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _check_buf(lse, "lse", (B, Hq), torch.float32, q.device)
     if workspace is None:
         workspace = torch.empty(decode_workspace_bytes(B, Hq, max_pages * page_size, d),
                                 dtype=torch.uint8, device=q.device)
+    else:
+        _check_workspace(workspace, q.device)
     st = lib().fa_decode_paged(q.data_ptr(), kpool.data_ptr(), vpool.data_ptr(),
                                block_table.data_ptr(), kv_lens.data_ptr(), out.data_ptr(),
                                lse.data_ptr() if lse is not None else None, B, Hq, Hkv, num_pages,
@@ -331,11 +359,12 @@ def fwd_fp8(q8, k8, v8, q_descale: float, k_descale: float, v_descale: float,
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=q8.device)
-    _check(out, "out", 4, q8.device)
-    if out.dtype != torch.bfloat16:
-        raise TypeError("out must be bfloat16")
+    else:
+        _check_buf(out, "out", (B, Hq, Nq, d), torch.bfloat16, q8.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q8.device)
+    elif lse is not None:
+        _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q8.device)
     st = lib().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
                           lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d,
                           1 if causal else 0, float(scale), float(q_descale), float(k_descale),
@@ -359,7 +388,6 @@ def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: Optional[float] = No
     import torch
     for t, name in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
         _check(t, name, 4, q.device)
-    _check(lse, "lse", 3, q.device)
     if any(t.dtype != q.dtype for t in (k, v, o, dout)):
         raise TypeError("q, k, v, o, dout must share one dtype")
     B, Hq, Nq, d = q.shape
@@ -367,14 +395,20 @@ def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: Optional[float] = No
     if tuple(v.shape) != tuple(k.shape) or Bk != B or dk_ != d or tuple(o.shape) != tuple(q.shape) \
             or tuple(dout.shape) != tuple(q.shape):
         raise ValueError("shape mismatch")
+    _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    for t, name, like in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        if t is not None:
+            _check_buf(t, name, like.shape, like.dtype, q.device)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     need = bwd_workspace_bytes(B, Hq, Nq)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    else:
+        _check_workspace(workspace, q.device)
     st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                       dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq,
                       Nk, d, 1 if causal else 0, float(scale), _dtype_code(q), workspace.data_ptr(),
@@ -408,11 +442,17 @@ def decode(q, kcache, vcache, kv_lens, scale: Optional[float] = None, out=None, 
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
+    else:
+        _check_buf(out, "out", q.shape, q.dtype, q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _check_buf(lse, "lse", (B, Hq), torch.float32, q.device)
     need = decode_workspace_bytes(B, Hq, max_len, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    else:
+        _check_workspace(workspace, q.device)
     st = lib().fa_decode(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), kv_lens.data_ptr(),
                          out.data_ptr(), lse.data_ptr() if lse is not None else None,
                          B, Hq, Hkv, max_len, d, float(scale), _dtype_code(q),
@@ -450,8 +490,12 @@ def decode_noalloc(q, kcache, vcache, kv_lens, scale: Optional[float] = None, ou
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
+    else:
+        _check_buf(out, "out", q.shape, q.dtype, q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _check_buf(lse, "lse", (B, Hq), torch.float32, q.device)
     st = lib().fa_decode_noalloc(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
                                  kv_lens.data_ptr(), out.data_ptr(),
                                  lse.data_ptr() if lse is not None else None,

@@ -1,0 +1,155 @@
+"""Host-side checks of the Python binding on caller-supplied buffers (CPU only).
+
+The kernels write outputs at offsets computed from the problem sizes, so an `out`, `lse`,
+`dq`/`dk`/`dv` or workspace of the wrong shape, dtype, device or layout must be refused
+before anything is launched. A stand-in for a CUDA tensor (shape, dtype, device, layout,
+no memory) lets these checks run without a GPU: it fails the test if the binding ever
+takes its data pointer, which only happens after every check has passed."""
+import pytest
+import torch
+
+import io_aware_exact_28_b200 as fa
+
+
+class FakeCuda:
+    """Just enough of a CUDA tensor for the binding's argument checks."""
+
+    def __init__(self, shape, dtype=torch.float16, index=0, contiguous=True):
+        self.shape = torch.Size(shape)
+        self.dtype = dtype
+        self.device = torch.device("cuda", index)
+        self.is_cuda = True
+        self._contiguous = contiguous
+
+    def dim(self):
+        return len(self.shape)
+
+    def is_contiguous(self):
+        return self._contiguous
+
+    def numel(self):
+        n = 1
+        for s in self.shape:
+            n *= s
+        return n
+
+    def element_size(self):
+        return torch.empty((), dtype=self.dtype).element_size()
+
+    def data_ptr(self):
+        raise AssertionError("a data pointer was taken before the checks refused the call")
+
+
+H16, F32 = torch.float16, torch.float32
+
+
+def fwd_args(**over):
+    a = dict(q=FakeCuda((2, 4, 96, 64)), k=FakeCuda((2, 2, 80, 64)), v=FakeCuda((2, 2, 80, 64)),
+             out=FakeCuda((2, 4, 96, 64)), lse=FakeCuda((2, 4, 96), F32))
+    a.update(over)
+    return a
+
+
+@pytest.mark.parametrize("bad, err", [
+    (dict(out=FakeCuda((2, 4, 96, 32))), ValueError),                 # wrong shape
+    (dict(out=FakeCuda((2, 4, 96, 64), torch.bfloat16)), TypeError),  # wrong dtype
+    (dict(out=FakeCuda((2, 4, 96, 64), index=1)), ValueError),        # other device
+    (dict(out=FakeCuda((2, 4, 96, 64), contiguous=False)), ValueError),
+    (dict(lse=FakeCuda((2, 4, 95), F32)), ValueError),
+    (dict(lse=FakeCuda((2, 4, 96), H16)), TypeError),
+])
+def test_fwd_refuses_bad_outputs(bad, err):
+    a = fwd_args(**bad)
+    with pytest.raises(err):
+        fa.fwd(a["q"], a["k"], a["v"], causal=True, out=a["out"], lse=a["lse"])
+    with pytest.raises(err):
+        fa.fwd_kvcache(a["q"], a["k"], a["v"], 80, out=a["out"], lse=a["lse"])
+
+
+def test_fwd_paged_refuses_bad_outputs():
+    q = FakeCuda((2, 4, 96, 64))
+    pool = FakeCuda((40, 2, 16, 64))
+    table = FakeCuda((2, 8), torch.int32)
+    with pytest.raises(ValueError):
+        fa.fwd_paged(q, pool, pool, table, 100, out=FakeCuda((2, 4, 97, 64)),
+                     lse=FakeCuda((2, 4, 96), F32))
+    with pytest.raises(TypeError):
+        fa.fwd_paged(q, pool, pool, table, 100, out=FakeCuda((2, 4, 96, 64)),
+                     lse=FakeCuda((2, 4, 96), torch.float64))
+
+
+def test_fwd_fp8_refuses_bad_outputs():
+    q8 = FakeCuda((1, 4, 64, 128), torch.uint8)
+    k8 = FakeCuda((1, 2, 64, 128), torch.uint8)
+    with pytest.raises(TypeError):       # the FP8 path writes bf16
+        fa.fwd_fp8(q8, k8, k8, 1.0, 1.0, 1.0, out=FakeCuda((1, 4, 64, 128), H16),
+                   lse=FakeCuda((1, 4, 64), F32))
+    with pytest.raises(ValueError):
+        fa.fwd_fp8(q8, k8, k8, 1.0, 1.0, 1.0, out=FakeCuda((1, 4, 64, 128), torch.bfloat16),
+                   lse=FakeCuda((1, 4, 63), F32))
+
+
+def bwd_call(**over):
+    a = dict(q=FakeCuda((1, 4, 64, 64)), k=FakeCuda((1, 2, 64, 64)), v=FakeCuda((1, 2, 64, 64)),
+             o=FakeCuda((1, 4, 64, 64)), lse=FakeCuda((1, 4, 64), F32),
+             dout=FakeCuda((1, 4, 64, 64)), dq=FakeCuda((1, 4, 64, 64)),
+             dk=FakeCuda((1, 2, 64, 64)), dv=FakeCuda((1, 2, 64, 64)),
+             workspace=FakeCuda((1 << 20,), torch.uint8))
+    a.update(over)
+    return fa.bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["dout"], causal=True, dq=a["dq"],
+                  dk=a["dk"], dv=a["dv"], workspace=a["workspace"])
+
+
+@pytest.mark.parametrize("bad, err", [
+    (dict(lse=FakeCuda((1, 4, 32), F32)), ValueError),
+    (dict(lse=FakeCuda((1, 4, 64), H16)), TypeError),
+    (dict(dq=FakeCuda((1, 2, 64, 64))), ValueError),       # dq takes q's shape
+    (dict(dk=FakeCuda((1, 4, 64, 64))), ValueError),       # dk takes k's shape
+    (dict(dv=FakeCuda((1, 2, 64, 64), torch.bfloat16)), TypeError),
+    (dict(workspace=FakeCuda((1 << 20,), torch.uint8, index=1)), ValueError),
+    (dict(workspace=FakeCuda((1 << 20,), torch.uint8, contiguous=False)), ValueError),
+])
+def test_bwd_refuses_bad_buffers(bad, err):
+    with pytest.raises(err):
+        bwd_call(**bad)
+
+
+def decode_args(**over):
+    a = dict(q=FakeCuda((3, 8, 128)), kc=FakeCuda((3, 2, 512, 128)), vc=FakeCuda((3, 2, 512, 128)),
+             lens=FakeCuda((3,), torch.int32), out=FakeCuda((3, 8, 128)),
+             lse=FakeCuda((3, 8), F32), workspace=FakeCuda((1 << 22,), torch.uint8))
+    a.update(over)
+    return a
+
+
+@pytest.mark.parametrize("bad, err", [
+    (dict(out=FakeCuda((3, 8, 64))), ValueError),
+    (dict(out=FakeCuda((3, 8, 128), torch.bfloat16)), TypeError),
+    (dict(lse=FakeCuda((3, 4), F32)), ValueError),
+    (dict(lse=FakeCuda((3, 8), H16)), TypeError),
+    (dict(workspace=FakeCuda((1 << 22,), torch.uint8, index=2)), ValueError),
+])
+def test_decode_refuses_bad_buffers(bad, err):
+    a = decode_args(**bad)
+    with pytest.raises(err):
+        fa.decode(a["q"], a["kc"], a["vc"], a["lens"], out=a["out"], lse=a["lse"],
+                  workspace=a["workspace"])
+    if "workspace" not in bad:
+        with pytest.raises(err):
+            fa.decode_noalloc(a["q"], a["kc"], a["vc"], a["lens"], out=a["out"], lse=a["lse"])
+
+
+def test_decode_paged_refuses_bad_buffers():
+    q = FakeCuda((3, 8, 128))
+    pool = FakeCuda((64, 2, 16, 128))
+    table = FakeCuda((3, 32), torch.int32)
+    lens = FakeCuda((3,), torch.int32)
+    good = dict(out=FakeCuda((3, 8, 128)), lse=FakeCuda((3, 8), F32),
+                workspace=FakeCuda((1 << 22,), torch.uint8))
+    for bad, err in ((dict(out=FakeCuda((3, 8, 127))), ValueError),
+                     (dict(lse=FakeCuda((3, 8), torch.float64)), TypeError),
+                     (dict(workspace=FakeCuda((1 << 22,), torch.uint8, contiguous=False)), ValueError)):
+        a = dict(good, **bad)
+        with pytest.raises(err):
+            fa.decode_paged(q, pool, pool, table, lens, out=a["out"], lse=a["lse"],
+                            workspace=a["workspace"])
