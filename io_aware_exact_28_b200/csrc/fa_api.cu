@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -20,8 +21,10 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;   // 2 s
 
-uint64_t g_timeout_ns = kDefaultTimeoutNs;
-int g_skip_q_load = 0;
+// Test hooks, set by fa_set_wait_timeout_ns / fa_debug_skip_q_load and read by every
+// launch; atomics, since the setters may run on another host thread.
+std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<int> g_skip_q_load{0};
 
 // ---------------------------------------------------------------------------------------
 // Device checks (cached per device)
@@ -391,7 +394,7 @@ fa_status launch_decode_tc_t(int dev, const void* q, const void* kc, const void*
   tp.split_tokens = L.split_tokens;
   tp.n_split = L.n_split;
   tp.scale_log2 = scale * 1.4426950408889634f;
-  tp.timeout_ns = g_timeout_ns;
+  tp.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
   tp.pk = PAGED ? pg->device(Hkv) : fa::PagedKV{};
   const long long n_units = static_cast<long long>(L.n_split) * B * Hkv * tp.n_gt;
   if (n_units >= (1LL << 31)) return FA_ERR_INVALID_ARG;
@@ -502,8 +505,8 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   prm.Nk = Nk;
   prm.causal_offset = Nk - Nq;
   prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.timeout_ns = g_timeout_ns;
-  prm.skip_q_load = g_skip_q_load;
+  prm.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  prm.skip_q_load = g_skip_q_load.load(std::memory_order_relaxed);
   prm.o_scale = 1.f;
   prm.pk = pg ? pg->device(Hkv) : fa::PagedKV{};
   prm.last_page = pg ? (Nk - 1) / pg->page_size : 0;
@@ -577,7 +580,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   prm.causal_offset = Nk - Nq;
   prm.scale = scale;
   prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.timeout_ns = g_timeout_ns;
+  prm.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 64)
     return bf16 ? launch_bwd<64, true>(dev, mp, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st)
@@ -637,8 +640,8 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
   prm.causal_offset = Nk - Nq;
   // Scores of the stored values carry the Q and K descales; O carries V's.
   prm.scale_log2 = scale * q_descale * k_descale * 1.4426950408889634f;
-  prm.timeout_ns = g_timeout_ns;
-  prm.skip_q_load = g_skip_q_load;
+  prm.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  prm.skip_q_load = g_skip_q_load.load(std::memory_order_relaxed);
   prm.pk = fa::PagedKV{};
   prm.last_page = 0;
   prm.o_scale = v_descale;
@@ -738,7 +741,7 @@ fa_status decode_impl(const void* q, const void* kcache, const void* vcache, con
   dp.split_tokens = L.split_tokens;
   dp.n_split = L.n_split;
   dp.scale_log2 = scale * 1.4426950408889634f;
-  dp.timeout_ns = g_timeout_ns;
+  dp.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
   dp.pk = pg ? pg->device(Hkv) : fa::PagedKV{};
 #define FA_DEC_CASE(D_, BF_)                                                         \
   return pg ? launch_decode_g<D_, BF_, true>(dev, dp, cp, B, Hkv, G, st)             \
@@ -845,9 +848,11 @@ fa_status fa_device_status(int clear) {
   return v == 0 ? FA_OK : static_cast<fa_status>(v);
 }
 
-void fa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : kDefaultTimeoutNs; }
+void fa_set_wait_timeout_ns(uint64_t ns) {
+  g_timeout_ns.store(ns ? ns : kDefaultTimeoutNs, std::memory_order_relaxed);
+}
 
-void fa_debug_skip_q_load(int enable) { g_skip_q_load = enable ? 1 : 0; }
+void fa_debug_skip_q_load(int enable) { g_skip_q_load.store(enable ? 1 : 0, std::memory_order_relaxed); }
 
 #ifdef FA_TC_TRACE
 // Debug builds only: copy the tensor-core decode trace (8 events x 1024 tiles of clock64).
