@@ -173,10 +173,15 @@ def _check_workspace(ws, device) -> None:
         raise ValueError("workspace must be contiguous")
 
 
-def _stream_ptr(stream) -> int:
+def _launch(device, stream, fn, *args) -> int:
+    """Call library entry point `fn` with `device` (the tensors' device) current, passing
+    `stream`, or that device's current stream, as the last argument. The library enqueues
+    on the current device, so tensors on another GPU would otherwise be read from the
+    wrong one."""
     import torch
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return int(s.cuda_stream)
+    with torch.cuda.device(device):
+        s = stream if stream is not None else torch.cuda.current_stream(device)
+        return int(fn(*args, int(s.cuda_stream)))
 
 
 def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, lse=None,
@@ -206,10 +211,10 @@ def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, 
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q.device)
-    st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                      lse.data_ptr() if lse is not None else None,
-                      B, Hq, Hkv, Nq, Nk, d, 1 if causal else 0, float(scale), _dtype_code(q),
-                      _stream_ptr(stream))
+    st = _launch(q.device, stream, lib().fa_fwd,
+                 q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                 lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d,
+                 1 if causal else 0, float(scale), _dtype_code(q))
     if st != FA_OK:
         raise FAError(st, "fa_fwd")
     return out, lse
@@ -241,10 +246,10 @@ def fwd_kvcache(q, kcache, vcache, nk: int, causal: bool = True, scale: Optional
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q.device)
-    st = lib().fa_fwd_kvcache(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), out.data_ptr(),
-                              lse.data_ptr() if lse is not None else None,
-                              B, Hq, Hkv, Nq, int(nk), cache_len, d, 1 if causal else 0,
-                              float(scale), _dtype_code(q), _stream_ptr(stream))
+    st = _launch(q.device, stream, lib().fa_fwd_kvcache,
+                 q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), out.data_ptr(),
+                 lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, int(nk), cache_len, d,
+                 1 if causal else 0, float(scale), _dtype_code(q))
     if st != FA_OK:
         raise FAError(st, "fa_fwd_kvcache")
     return out, lse
@@ -288,11 +293,11 @@ def fwd_paged(q, kpool, vpool, block_table, nk: int, causal: bool = True,
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q.device)
-    st = lib().fa_fwd_paged(q.data_ptr(), kpool.data_ptr(), vpool.data_ptr(),
-                            block_table.data_ptr(), out.data_ptr(),
-                            lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, int(nk),
-                            num_pages, page_size, block_table.shape[1], d, 1 if causal else 0,
-                            float(scale), _dtype_code(q), _stream_ptr(stream))
+    st = _launch(q.device, stream, lib().fa_fwd_paged,
+                 q.data_ptr(), kpool.data_ptr(), vpool.data_ptr(), block_table.data_ptr(),
+                 out.data_ptr(), lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq,
+                 int(nk), num_pages, page_size, block_table.shape[1], d, 1 if causal else 0,
+                 float(scale), _dtype_code(q))
     if st != FA_OK:
         raise FAError(st, "fa_fwd_paged")
     return out, lse
@@ -329,12 +334,11 @@ def decode_paged(q, kpool, vpool, block_table, kv_lens, scale: Optional[float] =
                                 dtype=torch.uint8, device=q.device)
     else:
         _check_workspace(workspace, q.device)
-    st = lib().fa_decode_paged(q.data_ptr(), kpool.data_ptr(), vpool.data_ptr(),
-                               block_table.data_ptr(), kv_lens.data_ptr(), out.data_ptr(),
-                               lse.data_ptr() if lse is not None else None, B, Hq, Hkv, num_pages,
-                               page_size, max_pages, d, float(scale), _dtype_code(q),
-                               workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                               _stream_ptr(stream))
+    st = _launch(q.device, stream, lib().fa_decode_paged,
+                 q.data_ptr(), kpool.data_ptr(), vpool.data_ptr(), block_table.data_ptr(),
+                 kv_lens.data_ptr(), out.data_ptr(), lse.data_ptr() if lse is not None else None, B,
+                 Hq, Hkv, num_pages, page_size, max_pages, d, float(scale), _dtype_code(q),
+                 workspace.data_ptr(), workspace.numel() * workspace.element_size())
     if st != FA_OK:
         raise FAError(st, "fa_decode_paged")
     return out, lse
@@ -365,10 +369,11 @@ def fwd_fp8(q8, k8, v8, q_descale: float, k_descale: float, v_descale: float,
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q8.device)
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q8.device)
-    st = lib().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
-                          lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d,
-                          1 if causal else 0, float(scale), float(q_descale), float(k_descale),
-                          float(v_descale), _stream_ptr(stream))
+    st = _launch(q8.device, stream, lib().fa_fwd_fp8,
+                 q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
+                 lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d,
+                 1 if causal else 0, float(scale), float(q_descale), float(k_descale),
+                 float(v_descale))
     if st != FA_OK:
         raise FAError(st, "fa_fwd_fp8")
     return out, lse
@@ -409,10 +414,11 @@ def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: Optional[float] = No
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     else:
         _check_workspace(workspace, q.device)
-    st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                      dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq,
-                      Nk, d, 1 if causal else 0, float(scale), _dtype_code(q), workspace.data_ptr(),
-                      workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    st = _launch(q.device, stream, lib().fa_bwd,
+                 q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                 dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nk,
+                 d, 1 if causal else 0, float(scale), _dtype_code(q), workspace.data_ptr(),
+                 workspace.numel() * workspace.element_size())
     if st != FA_OK:
         raise FAError(st, "fa_bwd")
     return dq, dk, dv
@@ -453,11 +459,11 @@ def decode(q, kcache, vcache, kv_lens, scale: Optional[float] = None, out=None, 
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     else:
         _check_workspace(workspace, q.device)
-    st = lib().fa_decode(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), kv_lens.data_ptr(),
-                         out.data_ptr(), lse.data_ptr() if lse is not None else None,
-                         B, Hq, Hkv, max_len, d, float(scale), _dtype_code(q),
-                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                         _stream_ptr(stream))
+    st = _launch(q.device, stream, lib().fa_decode,
+                 q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), kv_lens.data_ptr(),
+                 out.data_ptr(), lse.data_ptr() if lse is not None else None, B, Hq, Hkv, max_len,
+                 d, float(scale), _dtype_code(q), workspace.data_ptr(),
+                 workspace.numel() * workspace.element_size())
     if st != FA_OK:
         raise FAError(st, "fa_decode")
     return out, lse
@@ -496,11 +502,10 @@ def decode_noalloc(q, kcache, vcache, kv_lens, scale: Optional[float] = None, ou
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq), torch.float32, q.device)
-    st = lib().fa_decode_noalloc(q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
-                                 kv_lens.data_ptr(), out.data_ptr(),
-                                 lse.data_ptr() if lse is not None else None,
-                                 B, Hq, Hkv, max_len, d, float(scale), _dtype_code(q),
-                                 _stream_ptr(stream))
+    st = _launch(q.device, stream, lib().fa_decode_noalloc,
+                 q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), kv_lens.data_ptr(),
+                 out.data_ptr(), lse.data_ptr() if lse is not None else None, B, Hq, Hkv, max_len,
+                 d, float(scale), _dtype_code(q))
     if st != FA_OK:
         raise FAError(st, "fa_decode_noalloc")
     return out, lse

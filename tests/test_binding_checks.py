@@ -153,3 +153,89 @@ def test_decode_paged_refuses_bad_buffers():
         with pytest.raises(err):
             fa.decode_paged(q, pool, pool, table, lens, out=a["out"], lse=a["lse"],
                             workspace=a["workspace"])
+
+
+def test_launch_makes_the_tensors_device_current_and_passes_its_stream(monkeypatch):
+    """`_launch` enters the tensors' device, takes that device's current stream unless one
+    is given, and appends its handle as the last argument of the entry point."""
+    events = []
+
+    class Dev:
+        def __init__(self, device):
+            self.device = device
+
+        def __enter__(self):
+            events.append(("enter", self.device))
+
+        def __exit__(self, *exc):
+            events.append(("exit", self.device))
+            return False
+
+    class Stream:
+        def __init__(self, handle):
+            self.cuda_stream = handle
+
+    monkeypatch.setattr(torch.cuda, "device", Dev)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: Stream(4242))
+    calls = []
+
+    def entry(*args):
+        calls.append(args)
+        events.append(("call", None))
+        return 0
+
+    dev1 = torch.device("cuda", 1)
+    assert fa._launch(dev1, None, entry, 11, 22) == 0
+    assert calls[-1] == (11, 22, 4242)
+    assert events == [("enter", dev1), ("call", None), ("exit", dev1)]
+    assert fa._launch(dev1, Stream(7), entry, 5) == 0
+    assert calls[-1] == (5, 7)
+
+
+class ValidFake(FakeCuda):
+    """A stand-in that passes every check and hands out a distinct fake address."""
+    _next = 0x10000
+
+    def data_ptr(self):
+        ValidFake._next += 0x1000
+        return ValidFake._next
+
+
+def test_every_entry_point_receives_its_declared_argument_count(monkeypatch):
+    """Each binding function passes exactly the arguments its C entry point declares (the
+    stream handle is appended last by `_launch`)."""
+    seen = {}
+
+    def capture(device, stream, fn, *args):
+        seen[fn.__name__] = (len(args) + 1, len(fn.argtypes), args)
+        return fa.FA_OK
+
+    monkeypatch.setattr(fa, "_launch", capture)
+    V = ValidFake
+    q4, k4 = V((2, 4, 96, 64)), V((2, 2, 80, 64))
+    fa.fwd(q4, k4, k4, out=V((2, 4, 96, 64)), lse=V((2, 4, 96), F32))
+    fa.fwd_kvcache(q4, k4, k4, 80, out=V((2, 4, 96, 64)), lse=V((2, 4, 96), F32))
+    pool, table = V((40, 2, 16, 64)), V((2, 8), torch.int32)
+    fa.fwd_paged(q4, pool, pool, table, 100, out=V((2, 4, 96, 64)), lse=V((2, 4, 96), F32))
+    q8, k8 = V((1, 4, 64, 128), torch.uint8), V((1, 2, 64, 128), torch.uint8)
+    fa.fwd_fp8(q8, k8, k8, 1.0, 1.0, 1.0, out=V((1, 4, 64, 128), torch.bfloat16),
+               lse=V((1, 4, 64), F32))
+    qb, kb = V((1, 4, 64, 64)), V((1, 2, 64, 64))
+    fa.bwd(qb, kb, kb, V((1, 4, 64, 64)), V((1, 4, 64), F32), V((1, 4, 64, 64)),
+           dq=V((1, 4, 64, 64)), dk=V((1, 2, 64, 64)), dv=V((1, 2, 64, 64)),
+           workspace=V((1 << 20,), torch.uint8))
+    q3, cache, lens = V((3, 8, 128)), V((3, 2, 512, 128)), V((3,), torch.int32)
+    fa.decode(q3, cache, cache, lens, out=V((3, 8, 128)), lse=V((3, 8), F32),
+              workspace=V((1 << 22,), torch.uint8))
+    fa.decode_noalloc(q3, cache, cache, lens, out=V((3, 8, 128)), lse=V((3, 8), F32))
+    dpool, dtable = V((64, 2, 16, 128)), V((3, 32), torch.int32)
+    fa.decode_paged(q3, dpool, dpool, dtable, lens, out=V((3, 8, 128)), lse=V((3, 8), F32),
+                    workspace=V((1 << 22,), torch.uint8))
+    assert set(seen) == {"fa_fwd", "fa_fwd_kvcache", "fa_fwd_paged", "fa_fwd_fp8", "fa_bwd",
+                         "fa_decode", "fa_decode_noalloc", "fa_decode_paged"}
+    for name, (passed, declared, _) in seen.items():
+        assert passed == declared, (name, passed, declared)
+    # spot checks of sizes in their places
+    assert seen["fa_fwd"][2][5:11] == (2, 4, 2, 96, 80, 64)
+    assert seen["fa_decode"][2][6:11] == (3, 8, 2, 512, 128)
+    assert seen["fa_decode_paged"][2][7:13] == (3, 8, 2, 64, 16, 32)
