@@ -50,6 +50,23 @@ def max_over_ranks(local_ms, world: int, device):
     return [float(x) for x in t]
 
 
+def spread_ms(ms):
+    """Mean, median, 10th and 90th percentile and extremes of per-launch times (ms)."""
+    xs = sorted(float(x) for x in ms)
+    n = len(xs)
+
+    def pct(p):
+        if n == 1:
+            return xs[0]
+        pos = p * (n - 1)
+        lo = int(math.floor(pos))
+        hi = min(lo + 1, n - 1)
+        return xs[lo] + (xs[hi] - xs[lo]) * (pos - lo)
+
+    return {"mean": sum(xs) / n, "median": pct(0.5), "p10": pct(0.1), "p90": pct(0.9),
+            "min": xs[0], "max": xs[-1], "n": n}
+
+
 def job_rate(world: int, steps: int, work_per_step: float, max_ms: float) -> float:
     """Whole-job throughput: every rank did `steps` steps of `work_per_step` units (weak
     scaling, replicas), and the job took the slowest rank's `max_ms`."""
@@ -571,10 +588,12 @@ def run_single_kernel(args):
         ms.append(e0.elapsed_time(e1))
     status = fa.status_string(fa.device_status())
     avg = sum(ms) / len(ms)
+    spread = spread_ms(ms)
     print(json.dumps({"only": args.only, "workload": w.describe(),
                       **({"chunk": args.chunk} if args.only == "chunked" else {}),
                       **({"page_size": args.page_size} if "paged" in args.only else {}), "ms_per_launch": avg,
-                      "value": work / (avg * 1e-3), "unit": unit, "device_status": status}))
+                      "value": work / (avg * 1e-3), "value_at_median": work / (spread["median"] * 1e-3),
+                      "unit": unit, "ms_spread": spread, "device_status": status}))
     return 0 if status == "FA_OK" else 1
 
 

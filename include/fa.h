@@ -273,7 +273,10 @@ FA_API fa_status fa_decode_paged(const void* q, const void* kpool, const void* v
  *    process exits; calls whose fa_decode_workspace_bytes(B, Hq, max_kv_len, d) exceeds
  *    it return FA_ERR_WORKSPACE without launching anything;
  *  - the first call on each device looks up the scratch's device address (with that
- *    device current); make that first call before any stream capture;
+ *    device current) and keeps it for the life of the process; make that first call
+ *    before any stream capture. A cudaDeviceReset (or any other teardown of the device's
+ *    primary context) unloads the array, so the kept address is stale afterwards: do not
+ *    call fa_decode_noalloc on a device after resetting it in the same process;
  *  - every call on a device shares the one scratch array, which keeps the previous call's
  *    contents (the kernels overwrite every slot they later read, so nothing needs
  *    clearing); two calls whose kernels may overlap on the GPU (different streams, or

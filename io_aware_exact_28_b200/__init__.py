@@ -173,15 +173,31 @@ def _check_workspace(ws, device) -> None:
         raise ValueError("workspace must be contiguous")
 
 
-def _launch(device, stream, fn, *args) -> int:
+def _launch(device, stream, fn, *args, owned=()) -> int:
     """Call library entry point `fn` with `device` (the tensors' device) current, passing
     `stream`, or that device's current stream, as the last argument. The library enqueues
     on the current device, so tensors on another GPU would otherwise be read from the
-    wrong one."""
+    wrong one.
+
+    `owned` lists the tensors this wrapper allocated (outputs, workspaces). They come from
+    torch's caching allocator on the device's current stream; when the kernels run on
+    another stream, each is recorded on that stream, so that its memory is not handed out
+    again while those kernels may still use it. A stream of another device is refused."""
     import torch
     with torch.cuda.device(device):
-        s = stream if stream is not None else torch.cuda.current_stream(device)
-        return int(fn(*args, int(s.cuda_stream)))
+        cur = torch.cuda.current_stream(device)
+        if stream is None:
+            s = cur
+        else:
+            if torch.device(stream.device) != torch.device(device):
+                raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
+            s = stream
+        status = int(fn(*args, int(s.cuda_stream)))
+        if int(s.cuda_stream) != int(cur.cuda_stream):
+            for t in owned:
+                if t is not None:
+                    t.record_stream(s)
+        return status
 
 
 def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, lse=None,
@@ -203,18 +219,21 @@ def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, 
         raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    owned = []
     if out is None:
         out = torch.empty_like(q)
+        owned.append(out)
     else:
         _check_buf(out, "out", q.shape, q.dtype, q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+        owned.append(lse)
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q.device)
     st = _launch(q.device, stream, lib().fa_fwd,
                  q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                  lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d,
-                 1 if causal else 0, float(scale), _dtype_code(q))
+                 1 if causal else 0, float(scale), _dtype_code(q), owned=owned)
     if st != FA_OK:
         raise FAError(st, "fa_fwd")
     return out, lse
@@ -238,18 +257,21 @@ def fwd_kvcache(q, kcache, vcache, nk: int, causal: bool = True, scale: Optional
         raise ValueError(f"shape mismatch q{tuple(q.shape)} kcache{tuple(kcache.shape)}")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    owned = []
     if out is None:
         out = torch.empty_like(q)
+        owned.append(out)
     else:
         _check_buf(out, "out", q.shape, q.dtype, q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+        owned.append(lse)
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q.device)
     st = _launch(q.device, stream, lib().fa_fwd_kvcache,
                  q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), out.data_ptr(),
                  lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, int(nk), cache_len, d,
-                 1 if causal else 0, float(scale), _dtype_code(q))
+                 1 if causal else 0, float(scale), _dtype_code(q), owned=owned)
     if st != FA_OK:
         raise FAError(st, "fa_fwd_kvcache")
     return out, lse
@@ -285,19 +307,22 @@ def fwd_paged(q, kpool, vpool, block_table, nk: int, causal: bool = True,
     num_pages, Hkv, page_size, _ = kpool.shape
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    owned = []
     if out is None:
         out = torch.empty_like(q)
+        owned.append(out)
     else:
         _check_buf(out, "out", q.shape, q.dtype, q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+        owned.append(lse)
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q.device)
     st = _launch(q.device, stream, lib().fa_fwd_paged,
                  q.data_ptr(), kpool.data_ptr(), vpool.data_ptr(), block_table.data_ptr(),
                  out.data_ptr(), lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq,
                  int(nk), num_pages, page_size, block_table.shape[1], d, 1 if causal else 0,
-                 float(scale), _dtype_code(q))
+                 float(scale), _dtype_code(q), owned=owned)
     if st != FA_OK:
         raise FAError(st, "fa_fwd_paged")
     return out, lse
@@ -321,24 +346,28 @@ def decode_paged(q, kpool, vpool, block_table, kv_lens, scale: Optional[float] =
     max_pages = block_table.shape[1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    owned = []
     if out is None:
         out = torch.empty_like(q)
+        owned.append(out)
     else:
         _check_buf(out, "out", q.shape, q.dtype, q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        owned.append(lse)
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq), torch.float32, q.device)
     if workspace is None:
         workspace = torch.empty(decode_workspace_bytes(B, Hq, max_pages * page_size, d),
                                 dtype=torch.uint8, device=q.device)
+        owned.append(workspace)
     else:
         _check_workspace(workspace, q.device)
     st = _launch(q.device, stream, lib().fa_decode_paged,
                  q.data_ptr(), kpool.data_ptr(), vpool.data_ptr(), block_table.data_ptr(),
                  kv_lens.data_ptr(), out.data_ptr(), lse.data_ptr() if lse is not None else None, B,
                  Hq, Hkv, num_pages, page_size, max_pages, d, float(scale), _dtype_code(q),
-                 workspace.data_ptr(), workspace.numel() * workspace.element_size())
+                 workspace.data_ptr(), workspace.numel() * workspace.element_size(), owned=owned)
     if st != FA_OK:
         raise FAError(st, "fa_decode_paged")
     return out, lse
@@ -361,19 +390,22 @@ def fwd_fp8(q8, k8, v8, q_descale: float, k_descale: float, v_descale: float,
         raise ValueError(f"shape mismatch q{tuple(q8.shape)} k{tuple(k8.shape)}")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    owned = []
     if out is None:
         out = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=q8.device)
+        owned.append(out)
     else:
         _check_buf(out, "out", (B, Hq, Nq, d), torch.bfloat16, q8.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q8.device)
+        owned.append(lse)
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q8.device)
     st = _launch(q8.device, stream, lib().fa_fwd_fp8,
                  q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
                  lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d,
                  1 if causal else 0, float(scale), float(q_descale), float(k_descale),
-                 float(v_descale))
+                 float(v_descale), owned=owned)
     if st != FA_OK:
         raise FAError(st, "fa_fwd_fp8")
     return out, lse
@@ -406,19 +438,27 @@ def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: Optional[float] = No
     for t, name, like in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
         if t is not None:
             _check_buf(t, name, like.shape, like.dtype, q.device)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
+    owned = []
+    if dq is None:
+        dq = torch.empty_like(q)
+        owned.append(dq)
+    if dk is None:
+        dk = torch.empty_like(k)
+        owned.append(dk)
+    if dv is None:
+        dv = torch.empty_like(v)
+        owned.append(dv)
     need = bwd_workspace_bytes(B, Hq, Nq)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        owned.append(workspace)
     else:
         _check_workspace(workspace, q.device)
     st = _launch(q.device, stream, lib().fa_bwd,
                  q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                  dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nk,
                  d, 1 if causal else 0, float(scale), _dtype_code(q), workspace.data_ptr(),
-                 workspace.numel() * workspace.element_size())
+                 workspace.numel() * workspace.element_size(), owned=owned)
     if st != FA_OK:
         raise FAError(st, "fa_bwd")
     return dq, dk, dv
@@ -446,24 +486,28 @@ def decode(q, kcache, vcache, kv_lens, scale: Optional[float] = None, out=None, 
         raise ValueError("shape mismatch between q, caches and kv_lens")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    owned = []
     if out is None:
         out = torch.empty_like(q)
+        owned.append(out)
     else:
         _check_buf(out, "out", q.shape, q.dtype, q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        owned.append(lse)
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq), torch.float32, q.device)
     need = decode_workspace_bytes(B, Hq, max_len, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        owned.append(workspace)
     else:
         _check_workspace(workspace, q.device)
     st = _launch(q.device, stream, lib().fa_decode,
                  q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), kv_lens.data_ptr(),
                  out.data_ptr(), lse.data_ptr() if lse is not None else None, B, Hq, Hkv, max_len,
                  d, float(scale), _dtype_code(q), workspace.data_ptr(),
-                 workspace.numel() * workspace.element_size())
+                 workspace.numel() * workspace.element_size(), owned=owned)
     if st != FA_OK:
         raise FAError(st, "fa_decode")
     return out, lse
@@ -494,18 +538,21 @@ def decode_noalloc(q, kcache, vcache, kv_lens, scale: Optional[float] = None, ou
         raise ValueError("shape mismatch between q, caches and kv_lens")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    owned = []
     if out is None:
         out = torch.empty_like(q)
+        owned.append(out)
     else:
         _check_buf(out, "out", q.shape, q.dtype, q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        owned.append(lse)
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq), torch.float32, q.device)
     st = _launch(q.device, stream, lib().fa_decode_noalloc,
                  q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), kv_lens.data_ptr(),
                  out.data_ptr(), lse.data_ptr() if lse is not None else None, B, Hq, Hkv, max_len,
-                 d, float(scale), _dtype_code(q))
+                 d, float(scale), _dtype_code(q), owned=owned)
     if st != FA_OK:
         raise FAError(st, "fa_decode_noalloc")
     return out, lse

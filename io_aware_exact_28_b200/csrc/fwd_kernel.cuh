@@ -57,6 +57,9 @@ constexpr int kWarpMma = 9;
 #ifndef FA_EMU_PAIRS_D128
 #define FA_EMU_PAIRS_D128 0u
 #endif
+#ifndef FA_D64_BN
+#define FA_D64_BN 64
+#endif
 #ifndef FA_REGSPLIT
 #define FA_REGSPLIT 1
 #endif
@@ -74,19 +77,20 @@ template <int D, bool FP8 = false>
 struct FwdCfg {
   static constexpr int ELEM = FP8 ? 1 : 2;            // bytes per Q/K/V element
   static constexpr int ROWB = D * ELEM;               // bytes per Q/K/V row
-  static constexpr int BN = (D == 64) ? 64 : 128;     // keys per K/V tile
-  static constexpr int CTAS = (D == 64) ? 2 : 1;      // resident CTAs per SM
-  // d = 128: 3 warpgroups (warps 10-11 idle) so the register re-split below can apply;
-  // d = 64: 10 warps, two CTAs per SM share the register file (96 registers per thread).
-  static constexpr int THREADS = (D == 64) ? 320 : 384;
-  static constexpr bool REGSPLIT = (D == 128) && FA_REGSPLIT;
+  static constexpr int BN = (D == 64) ? FA_D64_BN : 128;   // keys per K/V tile
+  static constexpr bool NARROW = (BN == 64);          // 64-key tiles, two CTAs per SM
+  static constexpr int CTAS = NARROW ? 2 : 1;         // resident CTAs per SM
+  // 128-key tiles: 3 warpgroups (warps 10-11 idle) so the register re-split below can
+  // apply; 64-key tiles: 10 warps, two CTAs per SM share the register file (96 each).
+  static constexpr int THREADS = NARROW ? 320 : 384;
+  static constexpr bool REGSPLIT = !NARROW && FA_REGSPLIT;
   static constexpr int NCH = ROWB / 128;              // 128-byte swizzle chunks along d
   static constexpr int OCH = D / 64;                  // 64-column chunks of an O row
   static constexpr int Q_CHUNK = kBM * 128;           // 128 rows x 128 bytes
   static constexpr int KV_CHUNK = BN * 128;
   static constexpr int Q_TILE_BYTES = kBM * ROWB;     // one 128-row tile of Q
   static constexpr int KV_TILE_BYTES = BN * ROWB;
-  static constexpr int NS = (D == 64 || FP8) ? 8 : 4; // K/V ring stages
+  static constexpr int NS = (ROWB == 128) ? 8 : 4;    // K/V ring stages
   // Keys per P.V instruction (32 bytes of K) and TMEM columns of P per 32 scores.
   static constexpr int KPI = 32 / ELEM;
   static constexpr int P_COLS32 = 8 * ELEM;
@@ -103,14 +107,14 @@ struct FwdCfg {
   static constexpr int CLC_OFF = BAR_OFF + ((NBARS * 8 + 15) / 16) * 16;   // 2 x 16-byte responses
   static constexpr int MISC_OFF = CLC_OFF + 32;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;   // + slack for 1 KB alignment
-  static constexpr uint32_t TMEM_COLS = (D == 64) ? 256 : 512;
+  static constexpr uint32_t TMEM_COLS = NARROW ? 256 : 512;
   static constexpr uint32_t S_COL = 0;                // S_t at t * BN
   static constexpr uint32_t O_COL = kQTiles * BN;     // O_t at O_COL + t * D
   // Registers per thread: the launch allocation (65536 / (threads * CTAS), rounded down
   // to 8) is re-split so that warpgroup 2 (producer, MMA, 2 idle warps) keeps REGS_OTHER
   // and the two softmax warpgroups get REGS_SOFTMAX; the split uses exactly the launch
   // allocation (checked on the host against the compiled register count).
-  static constexpr uint32_t REGS_LAUNCH = (D == 64) ? 96 : 168;
+  static constexpr uint32_t REGS_LAUNCH = NARROW ? 96 : 168;
   static constexpr uint32_t REGS_OTHER = 72;
   static constexpr uint32_t REGS_SOFTMAX = 216;
   static_assert(!REGSPLIT || 128 * REGS_OTHER + 256 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH,

@@ -6,13 +6,9 @@ normaliser gives the same result as the untiled definition (page "Kotaemon
 FlashAttention", algorithm bullets: Q split into row blocks, K_j/V_j blocks loaded per
 row block, running max and normaliser updated, result identical to the original).
 
-It follows the pages' outer/inner loop order (page "Flash Attention ... IO-aware exact"
-(fr), tiling pseudo-code: loop over row blocks Q_i, load K_j and V_j, form
-S_ij = Q_i K_j^T / sqrt(d), accumulate O_i, write O_i once at the end and return O and
-L). That listing is garbled: it has no loop over j, leaves Tr undefined and applies a
-local softmax to each tile with a plain ``+=``. The reading taken here, stated in the
-pages' own terms elsewhere (page "Flash Attention" (zh), online-softmax bullet), is the
-running-max rescale: for every tile,
+The loop is derived from the online-softmax recurrence (page "Flash Attention" (zh),
+online-softmax bullet; page "Kotaemon FlashAttention", running max and normaliser): query
+rows in blocks of Br, keys in blocks of Bc inside each row block, and for every key tile
 
     m_new = max(m, rowmax(S_ij));  alpha = exp(m - m_new)
     P_ij  = exp(S_ij - m_new);     l = alpha * l + rowsum(P_ij)
@@ -20,6 +16,11 @@ running-max rescale: for every tile,
 
 and after the last tile ``O_i / l`` and ``L_i = m + log(l)``. Tr = ceil(Nq/Br),
 Tc = ceil(Nk/Bc); masked scores are -inf.
+
+Prior art, not followed: the tiling pseudo-code of page "Flash Attention ... IO-aware
+exact" (fr) has the same outer loop over Q_i and returns O and L, but it has no loop over
+j, leaves Tr undefined and applies a separate softmax to each tile before a plain ``+=``,
+which is not exact; this code does not take that form.
 """
 from __future__ import annotations
 

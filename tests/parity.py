@@ -129,3 +129,78 @@ def assert_close_fp8(o_gpu, lse_gpu, O_ref, L_ref, sigma, what: str = ""):
     return {"max_err_over_sigma": ratio, "max_abs": float(err.max()) if err.size else 0.0,
             "rms": float(np.sqrt(np.mean(err ** 2))) if err.size else 0.0,
             "rms_sigma": float(np.sqrt(np.mean(sigma ** 2))) if sigma.size else 0.0}
+
+
+# Backward pass (fa_bwd). The kernels recompute S and P in fp32 from Q, K and the
+# forward's fp32 LSE, and every product accumulates in fp32; the errors that matter are
+# the 16-bit roundings, each modelled as an independent relative error uniform on
+# [-u, u] (variance u^2/3 times the value squared), u = 2^-8 (bf16) or 2^-11 (fp16):
+#   * P rounded to 16 bits as the A operand of dV = P^T dO;
+#   * dS = P * (dP - D), formed in fp32, rounded to 16 bits as the operand of dQ = scale dS K
+#     and of dK = scale dS^T Q;
+#   * D = sum_c dO_ic O_ic taken from the forward's 16-bit O, whose own error is its output
+#     rounding plus the forward's P rounding; an error in D_i moves every dS_ij of row i by
+#     -P_ij dD_i;
+#   * the 16-bit rounding of each output element.
+# Per element (one query head; a KV head's dK and dV sum its query heads' variances):
+#   var dV_jc = c (sum_i P_ij^2 dO_ic^2)
+#   var dQ_ic = c scale^2 (sum_j dS_ij^2 K_jc^2) + scale^2 var(D_i) (sum_j P_ij K_jc)^2
+#   var dK_jc = c scale^2 (sum_i dS_ij^2 Q_ic^2) + scale^2 sum_i P_ij^2 var(D_i) Q_ic^2
+#   var D_i   = sum_c dO_ic^2 c (O_ic^2 + sum_j P_ij^2 V_jc^2),      c = u^2 / 3,
+# plus c x^2 for the output rounding of the final value x. Uniform relative error on
+# [-u, u] overstates round-to-nearest-even (whose relative error shrinks towards the top
+# of each binade) by about sqrt(2) in RMS, so the model is conservative.
+BWD_U = {"bf16": 2.0 ** -8, "fp16": 2.0 ** -11}
+BWD_SIGMAS = 6.0
+
+
+def bwd_head_terms(Q, K, V, dO, vis, scale: float, dtype: str):
+    """Exact gradients and the error-model variances (before output rounding) of one
+    (batch, query head) problem, float64: (dQ, dK, dV, var_dQ, var_dK, var_dV)."""
+    c = BWD_U[dtype] ** 2 / 3.0
+    S = np.where(vis, scale * (Q @ K.T), -np.inf)
+    m = S.max(axis=1)
+    has = np.isfinite(m)
+    P = np.zeros_like(S)
+    P[has] = np.exp(S[has] - m[has, None])
+    del S
+    P[has] /= P[has].sum(axis=1, keepdims=True)
+    O = P @ V
+    P2 = P * P
+    var_o = c * (O * O + P2 @ (V * V))
+    var_d = ((dO * dO) * var_o).sum(axis=1)
+    dP = dO @ V.T
+    D = (P * dP).sum(axis=1)
+    dS = P * (dP - D[:, None])
+    del dP
+    dQ = scale * (dS @ K)
+    dK = scale * (dS.T @ Q)
+    dV = P.T @ dO
+    dS2 = dS * dS
+    del dS
+    PK = P @ K
+    var_dq = c * scale ** 2 * (dS2 @ (K * K)) + scale ** 2 * var_d[:, None] * PK * PK
+    var_dk = c * scale ** 2 * (dS2.T @ (Q * Q)) + scale ** 2 * ((P2 * var_d[:, None]).T @ (Q * Q))
+    var_dv = c * (P2.T @ (dO * dO))
+    return dQ, dK, dV, var_dq, var_dk, var_dv
+
+
+def assert_close_bwd(got, want, var, dtype: str, what: str = ""):
+    """One gradient (float64 arrays) against the model: every element within 6 sigma (plus
+    1e-6 of the gradient's largest magnitude for fp32 accumulation), and the RMS error
+    within the model's RMS sigma. `var` excludes the output rounding, added here."""
+    c = BWD_U[dtype] ** 2 / 3.0
+    sigma = np.sqrt(var + c * want * want)
+    err = np.abs(got - want)
+    floor = 1e-6 * float(np.max(np.abs(want))) if want.size else 0.0
+    bound = BWD_SIGMAS * sigma + floor
+    assert np.isfinite(got).all(), f"{what}: non-finite gradient"
+    ratio = float((err / np.maximum(sigma, 1e-300)).max()) if err.size else 0.0
+    rms_err = float(np.sqrt(np.mean(err ** 2))) if err.size else 0.0
+    rms_sig = float(np.sqrt(np.mean(sigma ** 2))) if err.size else 0.0
+    stats = {"max_err_over_sigma": ratio, "rms_err_over_rms_sigma": rms_err / max(rms_sig, 1e-300),
+             "rel_rms": rms_err / max(float(np.sqrt(np.mean(want ** 2))), 1e-300)}
+    assert (err <= bound).all(), \
+        f"{what}: {int((err > bound).sum())} elements past 6 sigma {stats}"
+    assert rms_err <= rms_sig + floor, f"{what}: RMS error above the model's {stats}"
+    return stats

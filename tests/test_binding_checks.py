@@ -34,7 +34,7 @@ class FakeCuda:
         return n
 
     def element_size(self):
-        return torch.empty((), dtype=self.dtype).element_size()
+        return self.dtype.itemsize
 
     def data_ptr(self):
         raise AssertionError("a data pointer was taken before the checks refused the call")
@@ -172,8 +172,9 @@ def test_launch_makes_the_tensors_device_current_and_passes_its_stream(monkeypat
             return False
 
     class Stream:
-        def __init__(self, handle):
+        def __init__(self, handle, device=torch.device("cuda", 1)):
             self.cuda_stream = handle
+            self.device = device
 
     monkeypatch.setattr(torch.cuda, "device", Dev)
     monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: Stream(4242))
@@ -192,6 +193,102 @@ def test_launch_makes_the_tensors_device_current_and_passes_its_stream(monkeypat
     assert calls[-1] == (5, 7)
 
 
+def test_launch_records_owned_tensors_on_a_side_stream(monkeypatch):
+    """Tensors the wrapper allocated come from the current stream's pool; when the kernels
+    run on another stream they are recorded on it (so the allocator does not reuse their
+    memory while those kernels may still run), and a stream of another device is refused
+    before anything is launched."""
+    class Dev:
+        def __init__(self, device):
+            pass
+
+        def __enter__(self):
+            return None
+
+        def __exit__(self, *exc):
+            return False
+
+    class Stream:
+        def __init__(self, handle, device):
+            self.cuda_stream = handle
+            self.device = device
+
+    class Owned:
+        def __init__(self):
+            self.recorded = []
+
+        def record_stream(self, s):
+            self.recorded.append(s.cuda_stream)
+
+    dev0 = torch.device("cuda", 0)
+    monkeypatch.setattr(torch.cuda, "device", Dev)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: Stream(100, dev0))
+    calls = []
+
+    def entry(*args):
+        calls.append(args)
+        return 0
+
+    a, b = Owned(), Owned()
+    fa._launch(dev0, None, entry, 1, owned=[a, None, b])        # current stream: nothing to record
+    assert a.recorded == [] and b.recorded == []
+    fa._launch(dev0, Stream(100, dev0), entry, 1, owned=[a])     # the current stream, passed in
+    assert a.recorded == []
+    fa._launch(dev0, Stream(555, dev0), entry, 2, owned=[a, None, b])
+    assert calls[-1] == (2, 555) and a.recorded == [555] and b.recorded == [555]
+    n = len(calls)
+    with pytest.raises(ValueError):
+        fa._launch(dev0, Stream(9, torch.device("cuda", 3)), entry, 3, owned=[a])
+    assert len(calls) == n and a.recorded == [555]
+
+
+def test_wrappers_hand_their_own_allocations_to_launch(monkeypatch):
+    """Each wrapper lists exactly the tensors it allocated (outputs it was not given, the
+    workspace) as owned; caller-supplied buffers are not listed."""
+    seen = {}
+
+    def capture(device, stream, fn, *args, owned=()):
+        seen[fn.__name__] = list(owned)
+        return fa.FA_OK
+
+    made = []
+
+    def fake_empty(*shape, dtype=None, device=None, **kw):
+        t = ValidFake(shape[0] if len(shape) == 1 and isinstance(shape[0], (tuple, list, torch.Size)) else shape,
+                      dtype or torch.float32)
+        made.append(t)
+        return t
+
+    def fake_empty_like(x, **kw):
+        t = ValidFake(tuple(x.shape), x.dtype)
+        made.append(t)
+        return t
+
+    monkeypatch.setattr(fa, "_launch", capture)
+    monkeypatch.setattr(torch, "empty", fake_empty)
+    monkeypatch.setattr(torch, "empty_like", fake_empty_like)
+    monkeypatch.setattr(fa, "decode_workspace_bytes", lambda *a: 1 << 20)
+    monkeypatch.setattr(fa, "bwd_workspace_bytes", lambda *a: 1 << 20)
+    V = ValidFake
+    q4, k4 = V((2, 4, 96, 64)), V((2, 2, 80, 64))
+    o, l = fa.fwd(q4, k4, k4)
+    assert seen["fa_fwd"] == [o, l]
+    given = V((2, 4, 96, 64))
+    o, l = fa.fwd(q4, k4, k4, out=given)
+    assert o is given and seen["fa_fwd"] == [l]
+    q3, cache, lens = V((3, 8, 128)), V((3, 2, 512, 128)), V((3,), torch.int32)
+    made.clear()
+    fa.decode(q3, cache, cache, lens)
+    assert seen["fa_decode"] == made and len(made) == 3     # out, lse, workspace
+    made.clear()
+    fa.decode(q3, cache, cache, lens, workspace=V((1 << 22,), torch.uint8), return_lse=False)
+    assert seen["fa_decode"] == made and len(made) == 1     # out only
+    qb, kb = V((1, 4, 64, 64)), V((1, 2, 64, 64))
+    made.clear()
+    fa.bwd(qb, kb, kb, V((1, 4, 64, 64)), V((1, 4, 64), F32), V((1, 4, 64, 64)))
+    assert seen["fa_bwd"] == made and len(made) == 4        # dq, dk, dv, workspace
+
+
 class ValidFake(FakeCuda):
     """A stand-in that passes every check and hands out a distinct fake address."""
     _next = 0x10000
@@ -206,7 +303,7 @@ def test_every_entry_point_receives_its_declared_argument_count(monkeypatch):
     stream handle is appended last by `_launch`)."""
     seen = {}
 
-    def capture(device, stream, fn, *args):
+    def capture(device, stream, fn, *args, owned=()):
         seen[fn.__name__] = (len(args) + 1, len(fn.argtypes), args)
         return fa.FA_OK
 
