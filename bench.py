@@ -1,10 +1,14 @@
 """Benchmark of the exact-attention hot path on B200.
 
-One step = one pass over the whole path on one batch of synthetic input:
-  * fa_fwd on the causal self-attention workload B=8 H=12 N=2048 d=64 fp16 (O and LSE),
+One step = one pass over the whole path, one launch per workload, each timed with CUDA
+events after its own L2 flush:
+  * fa_fwd on tiny (B=1 H=2 N=128 d=64 fp16, non-causal), mha2k (B=8 H=12 N=2048 d=64
+    fp16, causal), gqa8k (B=1 Hq=32 Hkv=8 N=8192 d=128 bf16, causal) and gqa32k (the same
+    at N=32768), each writing O and LSE;
   * fa_decode on the GQA decode workload B=64 Hq=32 Hkv=8 d=128 bf16, kv_len ~ U[512,4096].
-`value` is the forward's throughput in TFLOP/s (algorithmic, causal-adjusted FLOPs:
-4*d per visible query-key pair); the decode's KV-read GB/s is reported beside it.
+`value` is the long-context GQA prefill's throughput in TFLOP/s (algorithmic,
+causal-adjusted FLOPs: 4*d per visible query-key pair); every workload's throughput,
+spread and roofline is in `configs` (TFLOP/s for the prefills, KV-read GB/s for the decode).
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun (N > 1) each rank runs an independent replica (the path needs no
@@ -36,6 +40,10 @@ L2_NOTE = ("flushed before each step: a 256 MiB write, then a 256 MiB read so th
 # ex2.approx.f32 results per clock per SM, measured on this machine's B200s with a throughput
 # probe (independent chains, 4-32 warps per SM); f16x2/bf16x2 forms give the same rate.
 MUFU_EX2_PER_CLK_SM = 16.0
+# One step runs every workload once, in this order, then the decode; the headline value is
+# the long-context GQA prefill.
+FWD_ORDER = ["tiny", "mha2k", "gqa8k", "gqa32k"]
+HEADLINE = "gqa32k"
 
 
 def max_over_ranks(local_ms, world: int, device):
@@ -195,66 +203,136 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------------
-def oracle_cpu_baseline(w, budget_s: float):
-    """Time the float64 oracle as it stands on this host on a bounded sample of the forward
-    workload's heads (whole (batch, head) problems, in order, until `budget_s` elapses)."""
+# CPU oracle timings (the float64 oracle as it stands, on this host's cores)
+# ---------------------------------------------------------------------------------------
+def host_cpu():
+    """Host CPU model name (lscpu) and the cores this process may run on."""
+    model = None
+    try:
+        import subprocess
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.lower().startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except Exception:
+        pass
+    return {"model_name": model, "cores": len(os.sched_getaffinity(0))}
+
+
+def causal_pairs(rows, Nq: int, Nk: int) -> int:
+    """Visible (query, key) pairs of the given query rows under the bottom-right causal mask."""
+    off = Nk - Nq
+    return int(sum(max(0, min(Nk, int(i) + off + 1)) for i in rows))
+
+
+def oracle_rows_time(w, rows, heads, q=None, k=None, v=None):
+    """Time the oracle on `rows` of each (batch, head) in `heads`; returns (seconds,
+    algorithmic FLOPs of that work)."""
     import numpy as np
     from oracle import attention_rows_f64
+    if q is None:
+        q, k, v = make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed)
+    rows = np.asarray(rows, dtype=np.int64)
+    pairs = causal_pairs(rows, w.N, w.N) if w.causal else len(rows) * w.N
+    t0 = time.perf_counter()
+    for b, h in heads:
+        attention_rows_f64(q, k, v, w.causal, w.scale, b, h, rows)
+    return time.perf_counter() - t0, 4.0 * w.d * pairs * len(heads)
+
+
+def oracle_baselines(budget_s: float):
+    """Per-workload CPU oracle figures on bounded samples (about 10 s of host time in all):
+    tiny in full; mha2k on as many whole (batch, head) problems as a quarter of `budget_s`
+    allows; gqa8k on 1024 rows of one head; gqa32k on 256 seeded rows of one head (rows 0,
+    1, 127, 128 and N-1 among them); the decode on 16 of its 64 sequences. Full-size times
+    are extrapolated from the samples and labelled estimates."""
+    import numpy as np
+    from oracle import decode_f64
+    host = host_cpu()
+    res = {}
+    w = WORKLOADS["tiny"]
+    el, fl = oracle_rows_time(w, np.arange(w.N), [(b, h) for b in range(w.B) for h in range(w.Hq)])
+    res["tiny"] = {"value": fl / el / 1e12, "unit": "TFLOP/s", "seconds": el,
+                   "sample": "the whole workload"}
+    w = WORKLOADS["mha2k"]
     q, k, v = make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed)
-    rows = np.arange(w.N)
-    heads, t0 = 0, time.perf_counter()
-    for b in range(w.B):
-        for h in range(w.Hq):
-            attention_rows_f64(q, k, v, w.causal, w.scale, b, h, rows)
-            heads += 1
-            if time.perf_counter() - t0 >= budget_s:
-                break
-        else:
-            continue
-        break
+    heads, el, fl = 0, 0.0, 0.0
+    order = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    while heads < len(order) and el < 0.25 * budget_s:
+        e, f = oracle_rows_time(w, np.arange(w.N), [order[heads]], q, k, v)
+        el, fl, heads = el + e, fl + f, heads + 1
+    res["mha2k"] = {"value": fl / el / 1e12, "unit": "TFLOP/s", "seconds": el,
+                    "sample": f"{heads} of {len(order)} whole (batch, head) problems",
+                    "full_workload_seconds_estimate": el * len(order) / heads}
+    w = WORKLOADS["gqa8k"]
+    rows = np.concatenate([np.arange(r, r + 256) for r in (0, w.N // 4, w.N // 2, w.N - 256)])
+    el, fl = oracle_rows_time(w, rows, [(0, 0)])
+    res["gqa8k"] = {"value": fl / el / 1e12, "unit": "TFLOP/s", "seconds": el,
+                    "sample": f"{len(rows)} rows of one head (four 256-row blocks spread over the "
+                              f"sequence) of {w.Hq} heads",
+                    "full_workload_seconds_estimate": el / len(rows) * w.N * w.Hq,
+                    "estimate_note": "estimate: the sample's time per row times all rows of all heads"}
+    w = WORKLOADS["gqa32k"]
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, w.N - 1],
+                                     np.random.default_rng(w.N).choice(w.N, 251, replace=False)]))
+    el, fl = oracle_rows_time(w, rows, [(0, 0)])
+    per_row = el / len(rows)
+    res["gqa32k"] = {"value": fl / el / 1e12, "unit": "TFLOP/s", "seconds": el,
+                     "sample": f"{len(rows)} seeded rows (0, 1, 127, 128, N-1 among them) of one head",
+                     "full_workload_seconds_estimate": per_row * w.N * w.Hq,
+                     "estimate_note": "estimate: the sample's time per row times all rows of all "
+                                      "heads (the oracle forms every row over all N keys)"}
+    w = WORKLOADS["decode"]
+    kv_lens, dq, kc, vc = make_decode_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.dtype, w.kv_len_lo,
+                                             w.kv_len_hi, w.seed)
+    nb = 16
+    t0 = time.perf_counter()
+    decode_f64(dq[:nb], kc[:nb], vc[:nb], kv_lens[:nb], w.scale)
     el = time.perf_counter() - t0
-    flops = fwd_flops(1, 1, w.N, w.N, w.d, w.causal) * heads
-    cores = len(os.sched_getaffinity(0))
-    return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{heads} of {w.B * w.Hq} (batch, head) problems of {w.describe()}, "
-                      f"float64 NumPy, {el:.1f} s"}
+    res["decode"] = {"value": decode_kv_bytes(kv_lens[:nb], w.Hkv, w.d) / el / 1e9, "unit": "GB/s",
+                     "seconds": el, "sample": f"the first {nb} of {w.B} sequences",
+                     "full_workload_seconds_estimate": el * decode_kv_bytes(kv_lens, w.Hkv, w.d)
+                     / decode_kv_bytes(kv_lens[:nb], w.Hkv, w.d),
+                     "estimate_note": "estimate: scaled by the KV bytes of all sequences"}
+    for r in res.values():
+        r.update({"kind": "oracle", "cores": host["cores"]})
+    return res, host
 
 
 def run_reference(args):
-    """Reference arm: the float64 CPU oracle as it stands, on rank 0 only."""
+    """Reference arm: the float64 CPU oracle as it stands, on rank 0 only, on the headline
+    workload (long-context GQA prefill): each step is 256 seeded query rows of one head
+    (rows 0, 1, 127, 128 and N-1 among them), heads taken in turn."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = WORKLOADS[args.workload]
     import numpy as np
-    from oracle import attention_rows_f64
+    w = WORKLOADS[HEADLINE]
     q, k, v = make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed)
-    rows = np.arange(w.N)
-    per_step = max(1, args.ref_heads_per_step)
-    order = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, w.N - 1],
+                                     np.random.default_rng(w.N).choice(w.N, 251, replace=False)]))
 
     def step(i):
-        for j in range(per_step):
-            b, h = order[(i * per_step + j) % len(order)]
-            attention_rows_f64(q, k, v, w.causal, w.scale, b, h, rows)
+        return oracle_rows_time(w, rows, [(0, i % w.Hq)], q, k, v)
 
     for i in range(args.warmup):
         step(i)
-    t0 = time.perf_counter()
+    el, fl = 0.0, 0.0
     for i in range(args.steps):
-        step(args.warmup + i)
-    el = time.perf_counter() - t0
-    flops = fwd_flops(1, 1, w.N, w.N, w.d, w.causal) * per_step * args.steps
-    val = flops / el / 1e12
-    cores = len(os.sched_getaffinity(0))
+        e, f = step(args.warmup + i)
+        el, fl = el + e, fl + f
+    val = fl / el / 1e12
+    host = host_cpu()
+    sample = f"{len(rows)} seeded query rows of one head per step, heads in turn"
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": w.describe(), "parallelism": "single process, host cores",
-                       "sample_per_step": f"{per_step} (batch, head) problems of the workload"},
-            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{per_step} (batch, head) problems per step"},
+                       "sample_per_step": sample},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": host["cores"], "kind": "oracle",
+                             "sample": sample, "host_cpu": host["model_name"]},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -276,105 +354,134 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     peaks, peak_src = load_peaks()
-    w = WORKLOADS[args.workload]
-    wd = WORKLOADS[args.decode_workload]
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    l2_flush = make_l2_flush(dev)
 
-    # Inputs (seeded, CPU-generated), resident on the device before timing.
-    q, k, v = (t.to(dev) for t in make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed))
-    o = torch.empty_like(q)
-    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    # Inputs (seeded, CPU-generated), resident on the device before timing. One entry per
+    # workload: the call, its work per launch and what bounds it.
+    calls = []
+    for name in FWD_ORDER:
+        w = WORKLOADS[name]
+        q, k, v = (t.to(dev) for t in make_fwd_inputs(w.B, w.Hq, w.Hkv, w.N, w.N, w.d, w.dtype, w.seed))
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+
+        def call(q=q, k=k, v=v, o=o, lse=lse, w=w):
+            fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+
+        calls.append({"name": name, "w": w, "call": call, "kind": "fwd",
+                      "work": fwd_flops(w.B, w.Hq, w.N, w.N, w.d, w.causal),
+                      "bytes": 2 * (2 * q.numel() + 2 * k.numel()) + 4 * lse.numel(),
+                      "tensors": (q, k, v, o, lse)})
+    wd = WORKLOADS["decode"]
     kv_lens_cpu, dq, kc, vc = make_decode_inputs(wd.B, wd.Hq, wd.Hkv, wd.N, wd.d, wd.dtype,
                                                  wd.kv_len_lo, wd.kv_len_hi, wd.seed)
     kv_lens, dq, kc, vc = kv_lens_cpu.to(dev), dq.to(dev), kc.to(dev), vc.to(dev)
     do = torch.empty_like(dq)
     dlse = torch.empty((wd.B, wd.Hq), dtype=torch.float32, device=dev)
     ws = torch.empty(fa.decode_workspace_bytes(wd.B, wd.Hq, wd.N, wd.d), dtype=torch.uint8, device=dev)
-    l2_flush = make_l2_flush(dev)
-
-    # Head dimension 128 decodes on the tensor-core split kernel, other sizes on CUDA cores.
-    dec_kernel = ("fa_decode_tc_kernel" if wd.d == 128 and os.environ.get("FA_DECODE_CUDA_CORES") != "1"
-                  else "fa_decode_split_kernel")
-    fl = fwd_flops(w.B, w.Hq, w.N, w.N, w.d, w.causal)
-    fwd_bytes = 2 * (2 * q.numel() + 2 * k.numel()) + 4 * lse.numel()   # Q,K,V read, O write, LSE
-    kv_bytes = decode_kv_bytes(kv_lens_cpu, wd.Hkv, wd.d)
-    dec_bytes = kv_bytes + 2 * (dq.numel() + do.numel()) + 4 * dlse.numel()
-
-    def fwd_call():
-        fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
 
     def dec_call():
         fa.decode(dq, kc, vc, kv_lens, scale=wd.scale, out=do, lse=dlse, workspace=ws)
 
+    kv_bytes = decode_kv_bytes(kv_lens_cpu, wd.Hkv, wd.d)
+    calls.append({"name": "decode", "w": wd, "call": dec_call, "kind": "decode",
+                  "work": kv_bytes + 2 * (dq.numel() + do.numel()) + 4 * dlse.numel(),
+                  "kv_bytes": kv_bytes})
+    dec_kernel = ("fa_decode_tc_kernel" if wd.d == 128 and os.environ.get("FA_DECODE_CUDA_CORES") != "1"
+                  else "fa_decode_split_kernel")
+
+    def step(ev=None):
+        for i, c in enumerate(calls):
+            l2_flush()                # every kernel starts from a cold, clean L2
+            if ev is not None:
+                ev[i][0].record()
+            c["call"]()
+            if ev is not None:
+                ev[i][1].record()
+
     for _ in range(args.warmup):
-        l2_flush()
-        fwd_call()
-        dec_call()
+        step()
     torch.cuda.synchronize()
     if fa.device_status() != fa.FA_OK:
         raise RuntimeError("device status not OK after warm-up")
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in calls] for _ in range(K)]
     sampler = ClockSampler(local)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
-    for i in range(K):
-        l2_flush()                    # L2 flush between steps, outside the timed events
-        ev[i][0].record()
-        fwd_call()
-        ev[i][1].record()
-        ev[i][2].record()             # decode inputs (1 GiB+) exceed L2 by themselves
-        dec_call()
-        ev[i][3].record()
+    for s_ in range(K):
+        step(evs[s_])
     torch.cuda.synchronize()
     sampler.stop()
     if world > 1:
         dist.barrier()
-    fwd_ms, dec_ms = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in ev),
-                                     sum(e[2].elapsed_time(e[3]) for e in ev)], world, dev)
+    # per-launch times, then the max over ranks of every number (same list length everywhere)
+    per = [[evs[s_][i][0].elapsed_time(evs[s_][i][1]) for s_ in range(K)] for i in range(len(calls))]
+    flat = max_over_ranks([x for row in per for x in row], world, dev)
+    per = [flat[i * K:(i + 1) * K] for i in range(len(calls))]
     status = fa.device_status()
-
-    fwd_tflops = job_rate(world, K, fl, fwd_ms) / 1e12
-    dec_gbs = job_rate(world, K, dec_bytes, dec_ms) / 1e9
-    fwd_avg_s = fwd_ms / K * 1e-3
-    dec_avg_s = dec_ms / K * 1e-3
-    roof_fwd = {"kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": fl / fwd_avg_s / 1e12,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": fl / fwd_avg_s / 1e12 / peaks["bf16_tflops"],
-                "traffic": measured_traffic("fa_fwd_kernel", args.workload),
-                "peak_source": f"{peak_src} dense bf16 burst (fp16 dense rate is the same)",
-                "algorithmic_flops_per_launch": fl, "algorithmic_bytes_per_launch": fwd_bytes}
-    roof_dec = {"kernel": f"fa_decode ({dec_kernel} + fa_decode_combine_kernel)", "bound": "hbm",
-                "achieved": dec_bytes / dec_avg_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": dec_bytes / dec_avg_s / 1e9 / peaks["hbm_gbs"],
-                "traffic": measured_traffic(dec_kernel, args.decode_workload),
-                "traffic_note": f"{dec_kernel} only (the combine kernel moves ~2% more)",
-                "peak_source": f"{peak_src} HBM copy bandwidth",
-                "algorithmic_bytes_per_launch": dec_bytes, "kv_bytes_per_launch": kv_bytes}
-    # The forward's other bound: one exponential (MUFU ex2) per visible score, against the
-    # measured 16.0 per clock per SM of this machine's B200s at the SM clock sampled during
-    # the timed region.
     clocks = sampler.summary()
     sm_mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz")
-    if sm_mhz:
-        n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
-        exps = fl / (4.0 * w.d)
-        peak_exps = MUFU_EX2_PER_CLK_SM * n_sm * sm_mhz * 1e6
-        roof_fwd["exp_unit"] = {"bound": "alu", "unit": "exp2/s", "achieved": exps / fwd_avg_s,
-                                "peak": peak_exps, "frac": exps / fwd_avg_s / peak_exps,
-                                "exps_per_launch": exps,
-                                "peak_source": f"measured {MUFU_EX2_PER_CLK_SM} ex2.approx/clk/SM x "
-                                               f"{n_sm} SMs x sampled {sm_mhz} MHz"}
-    dominant = roof_fwd if fwd_ms >= dec_ms else roof_dec
 
-    # End to end through the public API: host (pinned) inputs in, host outputs back, every
-    # step. Copies run on their own streams with double-buffered device tensors, so the
-    # upload of step i+1 and the download of step i overlap the forward of step i (as a
-    # serving loop would); the copy bytes per step are unchanged.
+    configs = []
+    for c, ms in zip(calls, per):
+        w, tot = c["w"], sum(ms)
+        sp = spread_ms(ms)
+        rate = job_rate(world, K, c["work"], tot)          # per second, whole job
+        per_launch_rate = c["work"] / (sp["mean"] * 1e-3)
+        entry = {"name": c["name"], "workload": w.describe(), "ms_per_launch": sp, "launches": K}
+        if c["kind"] == "fwd":
+            entry.update({"value": rate / 1e12, "unit": "TFLOP/s",
+                          "value_at_median": c["work"] / (sp["median"] * 1e-3) / 1e12 * world,
+                          "algorithmic_flops_per_launch": c["work"],
+                          "algorithmic_bytes_per_launch": c["bytes"]})
+            roof = {"kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": per_launch_rate / 1e12,
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": per_launch_rate / 1e12 / peaks["bf16_tflops"],
+                    "frac_of_sustained": per_launch_rate / 1e12 / peaks["bf16_tflops_sustained"],
+                    "frac_of_spec_2250": per_launch_rate / 1e12 / 2250.0,
+                    "traffic": measured_traffic("fa_fwd_kernel", c["name"]),
+                    "peak_source": f"{peak_src} dense bf16 burst (fp16 has the same dense rate)"}
+            if sm_mhz:
+                exps = c["work"] / (4.0 * w.d)
+                peak_exps = MUFU_EX2_PER_CLK_SM * n_sm * sm_mhz * 1e6
+                roof["exp_unit"] = {"bound": "alu", "unit": "exp2/s",
+                                    "achieved": exps / (sp["mean"] * 1e-3), "peak": peak_exps,
+                                    "frac": exps / (sp["mean"] * 1e-3) / peak_exps,
+                                    "peak_source": f"measured {MUFU_EX2_PER_CLK_SM} ex2.approx/clk/SM x "
+                                                   f"{n_sm} SMs x sampled {sm_mhz} MHz"}
+            if c["name"] == "tiny":
+                roof["note"] = "launch-latency bound: report the microseconds, not the fraction"
+        else:
+            entry.update({"value": rate / 1e9, "unit": "GB/s",
+                          "value_at_median": c["work"] / (sp["median"] * 1e-3) / 1e9 * world,
+                          "algorithmic_bytes_per_launch": c["work"], "kv_bytes_per_launch": c["kv_bytes"]})
+            roof = {"kernel": f"fa_decode ({dec_kernel} + fa_decode_combine_kernel)", "bound": "hbm",
+                    "achieved": per_launch_rate / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": per_launch_rate / 1e9 / peaks["hbm_gbs"],
+                    "frac_of_spec_8000": per_launch_rate / 1e9 / 8000.0,
+                    "traffic": measured_traffic(dec_kernel, "decode"),
+                    "traffic_note": f"{dec_kernel} only (the combine kernel moves ~2% more)",
+                    "peak_source": f"{peak_src} HBM copy bandwidth"}
+        entry["roofline"] = roof
+        configs.append(entry)
+    head = next(e for e in configs if e["name"] == HEADLINE)
+    dominant = max(configs, key=lambda e: e["ms_per_launch"]["mean"])["roofline"]
+
+    # End to end through the public API for the headline workload: host (pinned) inputs in,
+    # host outputs back, every step. Copies run on their own streams with double-buffered
+    # device tensors, so the upload of step i+1 and the download of step i overlap the
+    # forward of step i (as a serving loop would); the copy bytes per step are unchanged.
     e2e = None
     if not args.no_e2e:
+        hc = next(c for c in calls if c["name"] == HEADLINE)
+        w = hc["w"]
+        q, k, v, o, lse = hc["tensors"]
         hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
         ho = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
         hl = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
@@ -387,7 +494,7 @@ def run_ours(args):
         e_in = [torch.cuda.Event() for _ in range(2)]
         e_cmp = [torch.cuda.Event() for _ in range(2)]
         e_out = [torch.cuda.Event() for _ in range(2)]
-        E = max(3, min(K, 50))
+        E = max(3, min(K, args.e2e_steps))
 
         def e2e_step(n):
             bi = n & 1
@@ -425,36 +532,40 @@ def run_ours(args):
         s1.record(s_in)
         torch.cuda.synchronize()
         (e2e_ms,) = max_over_ranks([s0.elapsed_time(s1)], world, dev)
-        e2e = {"value": job_rate(world, E, fl, e2e_ms) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_rate(world, E, hc["work"], e2e_ms) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": 2 * (q.numel() + k.numel() + v.numel()),
                "d2h_bytes_per_step": 2 * o.numel() + 4 * lse.numel(), "steps": E,
+               "workload": w.describe(),
                "path": "fa.fwd (C ABI fa_fwd) with pinned host buffers; copies on separate "
                        "streams, double-buffered, overlapping the previous/next step"}
 
-    cpu = None
+    cpu, host = None, None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_cpu_baseline(w, args.cpu_budget_s)
+        per_cfg, host = oracle_baselines(args.cpu_budget_s)
+        for e in configs:
+            e["cpu_baseline"] = per_cfg[e["name"]]
+        cpu = dict(per_cfg[HEADLINE])
+        cpu["host_cpu"] = host["model_name"]
 
     if rank == 0:
+        ms_step = sum(sum(ms) for ms in per) / K
         line = {
-            "metric": METRIC, "value": fwd_tflops, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": K, "warmup": args.warmup, "ms_per_step": (fwd_ms + dec_ms) / K,
+            "metric": METRIC, "value": head["value"], "unit": "TFLOP/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": w.describe(), "decode_workload": wd.describe(),
+            "dtype": head_dtype(), "data": "synthetic",
+            "config": {"workload": WORKLOADS[HEADLINE].describe(),
+                       "step": "one launch of each workload: " + ", ".join(
+                           WORKLOADS[n].describe() for n in FWD_ORDER + ["decode"]),
                        "l2": L2_NOTE,
                        "parallelism": "replicas" if world > 1 else "single GPU",
-                       "value_is": "forward TFLOP/s, causal-adjusted algorithmic FLOPs"},
-            "fwd": {"tflops": fwd_tflops, "ms_per_launch": fwd_ms / K,
-                    "frac_of_measured_bf16_peak": roof_fwd["frac"],
-                    "frac_of_spec_2250_tflops": fl / fwd_avg_s / 1e12 / 2250.0},
-            "decode": {"value": dec_gbs, "unit": "GB/s", "ms_per_launch": dec_ms / K,
-                       "dtype": wd.dtype, "frac_of_measured_hbm": roof_dec["frac"],
-                       "frac_of_spec_8000_gbs": dec_bytes / dec_avg_s / 1e9 / 8000.0},
-            "roofline": dominant, "rooflines": [roof_fwd, roof_dec],
-            "e2e": e2e, "cpu_baseline": cpu,
-            "gpu_launches": K * (4 if dec_kernel == "fa_decode_tc_kernel" else 3),
-            "gpu_launches_note": (f"per step: fa_fwd_kernel + "
+                       "value_is": "long-context GQA causal prefill TFLOP/s (causal-adjusted "
+                                   "algorithmic FLOPs); every workload's figure is in configs"},
+            "configs": configs,
+            "roofline": dominant, "rooflines": [e["roofline"] for e in configs],
+            "e2e": e2e, "cpu_baseline": cpu, "host_cpu": host,
+            "gpu_launches": K * (len(FWD_ORDER) + (3 if dec_kernel == "fa_decode_tc_kernel" else 2)),
+            "gpu_launches_note": (f"per step: fa_fwd_kernel x {len(FWD_ORDER)} + "
                                   + ("fa_decode_ticket_reset_kernel + " if dec_kernel == "fa_decode_tc_kernel" else "")
                                   + f"{dec_kernel} + fa_decode_combine_kernel"),
             "clocks": clocks,
@@ -465,6 +576,10 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def head_dtype():
+    return WORKLOADS[HEADLINE].dtype
 
 
 def run_single_kernel(args):
@@ -604,7 +719,7 @@ def main():
                     default=None,
                     help="launch one entry point alone (profiling helper; prints its own line)")
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mha2k", choices=[k for k, v in WORKLOADS.items() if v.kind == "fwd"])
@@ -614,7 +729,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
-    ap.add_argument("--ref-heads-per-step", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
     if args.impl == "reference":

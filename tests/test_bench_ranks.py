@@ -68,8 +68,7 @@ def _reference_arm(rank: int):
     env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank),
                MASTER_ADDR="127.0.0.1")
     return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                           "--gpus", "2", "--steps", "1", "--warmup", "3",
-                           "--ref-heads-per-step", "1"],
+                           "--gpus", "2", "--steps", "1", "--warmup", "3"],
                           capture_output=True, text=True, env=env, timeout=600, cwd=ROOT)
 
 
@@ -82,3 +81,4 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert "N=32768" in line["config"]["workload"]          # the headline workload
