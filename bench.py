@@ -642,6 +642,22 @@ def run_single_kernel(args):
 
         def call():
             fa.fwd_fp8(q8, k8, v8, dq_, dk_, dv_, causal=w.causal, scale=w.scale, out=o, lse=lse)
+    elif args.only == "fwd_varlen":
+        # A ragged batch with the workload's head shape: sequences of different lengths
+        # (--varlen-lens, each a full causal prefill) in one fa_fwd_kvcache call with
+        # per-sequence lengths; FLOPs are the sum of each sequence's causal FLOPs.
+        w = WORKLOADS[args.workload]
+        lens = [int(x) for x in args.varlen_lens.split(",")]
+        B, cap = len(lens), max(lens)
+        q, k, v = (t.to(dev) for t in make_fwd_inputs(B, w.Hq, w.Hkv, cap, cap, w.d, w.dtype, w.seed))
+        o, lse = torch.empty_like(q), torch.empty((B, w.Hq, cap), dtype=torch.float32, device=dev)
+        ln = torch.tensor(lens, dtype=torch.int32, device=dev)
+        work = sum(fwd_flops(1, w.Hq, n, n, w.d, True) for n in lens) / 1e12
+        unit = "TFLOP/s"
+
+        def call():
+            fa.fwd_kvcache(q, k, v, cap, causal=True, scale=w.scale, out=o, lse=lse, q_lens=ln,
+                           kv_lens=ln)
     elif args.only == "fwd_paged":
         # Prefill of the workload with K and V in a page pool (fa_fwd_paged), pages drawn by
         # a seeded random table; same causal FLOPs as --only fwd.
@@ -706,7 +722,8 @@ def run_single_kernel(args):
     spread = spread_ms(ms)
     print(json.dumps({"only": args.only, "workload": w.describe(),
                       **({"chunk": args.chunk} if args.only == "chunked" else {}),
-                      **({"page_size": args.page_size} if "paged" in args.only else {}), "ms_per_launch": avg,
+                      **({"page_size": args.page_size} if "paged" in args.only else {}),
+                      **({"lens": args.varlen_lens} if args.only == "fwd_varlen" else {}), "ms_per_launch": avg,
                       "value": work / (avg * 1e-3), "value_at_median": work / (spread["median"] * 1e-3),
                       "unit": unit, "ms_spread": spread, "device_status": status}))
     return 0 if status == "FA_OK" else 1
@@ -715,7 +732,7 @@ def run_single_kernel(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--only", choices=["fwd", "decode", "chunked", "bwd", "fwd_paged", "decode_paged",
-                                       "fwd_fp8"],
+                                       "fwd_fp8", "fwd_varlen"],
                     default=None,
                     help="launch one entry point alone (profiling helper; prints its own line)")
     ap.add_argument("--gpus", type=int, default=1)
@@ -725,6 +742,8 @@ def main():
     ap.add_argument("--workload", default="mha2k", choices=[k for k, v in WORKLOADS.items() if v.kind == "fwd"])
     ap.add_argument("--chunk", type=int, default=1024, help="--only chunked: tokens per chunk")
     ap.add_argument("--page-size", type=int, default=64, help="--only *_paged: tokens per page")
+    ap.add_argument("--varlen-lens", default="8192,6144,3072,1024",
+                    help="--only fwd_varlen: comma-separated sequence lengths of the batch")
     ap.add_argument("--decode-workload", default="decode")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -81,23 +81,35 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
 /*
  * fa_fwd_kvcache — fa_fwd for a chunk of queries against the first Nk rows of a KV cache
  * whose capacity per head is cache_len >= Nk (chunked prefill: the newest Nq tokens
- * attend to the whole prefix, causally aligned to its end).
+ * attend to the whole prefix, causally aligned to its end), optionally with lengths that
+ * differ per sequence.
  *
  * Defined by: page "Flash Attention ... IO-aware exact" (fr), "Erreurs courantes et
  * solutions" (the manual chunking example: a chunk of queries attends to every key up to
- * the chunk's end) and "Optimisation avancée : KV Cache" (keys and values kept in a cache
- * across calls); the result is fa_fwd's with k, v = the caches' first Nk rows.
+ * the chunk's end) and "Optimisation avancée : KV Cache et persistent attention" (keys and
+ * values cached per session, each session with its own length); the result for sequence
+ * b is fa_fwd's with q = its first nq_b query rows and k, v = its cache's first nk_b rows.
  *
- *   q, o, lse           as fa_fwd, [B, Hq, Nq, d] / [B, Hq, Nq]
- *   kcache, vcache      [B, Hkv, cache_len, d]; rows [0, Nk) of each head are used, rows
- *                       [Nk, cache_len) are never read
- *   causal              0 or 1; with Nq <= Nk the chunk is the cache's last Nq tokens
+ *   q, o, lse           as fa_fwd, [B, Hq, Nq, d] / [B, Hq, Nq]: Nq is the row capacity
+ *   kcache, vcache      [B, Hkv, cache_len, d]
+ *   q_lens              NULL (every sequence has nq_b = Nq query rows) or [B] int32 in
+ *                       device memory, 4-byte aligned: nq_b = q_lens[b] clamped to [0, Nq]
+ *   kv_lens             NULL (nk_b = Nk keys each) or [B] int32 in device memory, 4-byte
+ *                       aligned: nk_b = kv_lens[b] clamped to [0, Nk]
+ *   causal              0 or 1; query row i of sequence b sees key j iff j <= i + nk_b - nq_b
+ *                       (the chunk is the last nq_b of the sequence's nk_b tokens)
+ *
+ * Rows [0, nk_b) of each head of sequence b are used; rows [nk_b, cache_len) and query
+ * rows [nq_b, Nq) may hold anything (NaN included) and never affect a written value.
+ * Output rows [nq_b, Nq) of o and lse are not written. A row with no visible key
+ * (nk_b = 0, or nq_b > nk_b causal) gets O = 0 and LSE = -inf.
  *
  * Requirements: those of fa_fwd, plus 1 <= Nk <= cache_len. Same errors and ownership.
  */
-FA_API fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* vcache, void* o,
-                         float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int cache_len,
-                         int d, int causal, float scale, fa_dtype dtype, void* stream);
+FA_API fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* vcache,
+                         const int* q_lens, const int* kv_lens, void* o, float* lse, int B,
+                         int Hq, int Hkv, int Nq, int Nk, int cache_len, int d, int causal,
+                         float scale, fa_dtype dtype, void* stream);
 
 /*
  * Paged KV cache (fa_fwd_paged, fa_decode_paged).
@@ -127,18 +139,25 @@ FA_API fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* v
 
 /*
  * fa_fwd_paged — fa_fwd_kvcache with the keys and values in a paged pool: each of the B
- * sequences attends to its first Nk tokens, found through its block-table row.
+ * sequences attends to its first nk_b tokens, found through its block-table row.
  *
- *   q, o, lse   as fa_fwd, [B, Hq, Nq, d] / [B, Hq, Nq]
- *   causal      0 or 1, bottom-right aligned (the chunk is the last Nq of the Nk tokens)
+ *   q, o, lse         as fa_fwd, [B, Hq, Nq, d] / [B, Hq, Nq]: Nq is the row capacity
+ *   q_lens, kv_lens   as fa_fwd_kvcache (NULL: Nq rows and Nk keys for every sequence;
+ *                     otherwise per-sequence values clamped to [0, Nq] and [0, Nk])
+ *   causal            0 or 1, bottom-right aligned per sequence (the chunk is the last
+ *                     nq_b of the sequence's nk_b tokens)
+ *
+ * Only the table entries that cover tokens [0, nk_b) of sequence b are read; output rows
+ * [nq_b, Nq) are not written.
  *
  * Requirements: those of fa_fwd and of the paged cache above, plus
  * Nk <= max_pages_per_seq * page_size.
  */
 FA_API fa_status fa_fwd_paged(const void* q, const void* kpool, const void* vpool,
-                       const int* block_table, void* o, float* lse, int B, int Hq, int Hkv,
-                       int Nq, int Nk, int num_pages, int page_size, int max_pages_per_seq,
-                       int d, int causal, float scale, fa_dtype dtype, void* stream);
+                       const int* block_table, const int* q_lens, const int* kv_lens, void* o,
+                       float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int num_pages,
+                       int page_size, int max_pages_per_seq, int d, int causal, float scale,
+                       fa_dtype dtype, void* stream);
 
 /*
  * fa_fwd_fp8 — fa_fwd with 8-bit (E4M3) Q, K and V and per-tensor descale factors: the

@@ -76,7 +76,7 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.argtypes = [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p] + [c_int] * 7 + \
             [c_float, c_int, c_void_p]
         L.fa_fwd.restype = c_int
-        L.fa_fwd_kvcache.argtypes = [c_void_p] * 5 + [c_int] * 8 + [c_float, c_int, c_void_p]
+        L.fa_fwd_kvcache.argtypes = [c_void_p] * 7 + [c_int] * 8 + [c_float, c_int, c_void_p]
         L.fa_fwd_kvcache.restype = c_int
         L.fa_bwd.argtypes = [c_void_p] * 9 + [c_int] * 7 + [c_float, c_int, c_void_p, c_size_t, c_void_p]
         L.fa_bwd.restype = c_int
@@ -99,7 +99,7 @@ def lib() -> ctypes.CDLL:
         L.fa_build_info.restype = ctypes.c_char_p
         L.fa_decode_noalloc.argtypes = [c_void_p] * 6 + [c_int] * 5 + [c_float, c_int, c_void_p]
         L.fa_decode_noalloc.restype = c_int
-        L.fa_fwd_paged.argtypes = [c_void_p] * 6 + [c_int] * 10 + [c_float, c_int, c_void_p]
+        L.fa_fwd_paged.argtypes = [c_void_p] * 8 + [c_int] * 10 + [c_float, c_int, c_void_p]
         L.fa_fwd_paged.restype = c_int
         L.fa_decode_paged.argtypes = [c_void_p] * 7 + [c_int] * 7 + [c_float, c_int, c_void_p,
                                                                      c_size_t, c_void_p]
@@ -239,16 +239,31 @@ def fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, 
     return out, lse
 
 
+def _check_lens(t, name: str, B: int, device) -> None:
+    """Per-sequence lengths: int32 [B] on the tensors' device, contiguous (or None)."""
+    import torch
+    if t is None:
+        return
+    _check(t, name, 1, device)
+    if t.dtype != torch.int32 or t.shape[0] != B:
+        raise TypeError(f"{name} must be int32 [B={B}], got {t.dtype} {tuple(t.shape)}")
+
+
 def fwd_kvcache(q, kcache, vcache, nk: int, causal: bool = True, scale: Optional[float] = None,
-                out=None, lse=None, return_lse: bool = True, stream=None):
+                out=None, lse=None, return_lse: bool = True, stream=None, q_lens=None,
+                kv_lens=None):
     """Chunked prefill via ``fa_fwd_kvcache``: q [B,Hq,Nq,d] against the first ``nk`` rows of
     kcache, vcache [B,Hkv,cache_len,d] (causal: the chunk is the prefix's last Nq tokens).
+    q_lens / kv_lens (int32 [B] on the device, optional) give sequence b its own nq_b <= Nq
+    query rows and nk_b <= nk keys; output rows past nq_b are left as they are.
     Returns (o [B,Hq,Nq,d], lse [B,Hq,Nq] fp32 or None).
     """
     import torch
     _check(q, "q", 4, q.device)
     _check(kcache, "kcache", 4, q.device)
     _check(vcache, "vcache", 4, q.device)
+    _check_lens(q_lens, "q_lens", q.shape[0], q.device)
+    _check_lens(kv_lens, "kv_lens", q.shape[0], q.device)
     if kcache.dtype != q.dtype or vcache.dtype != q.dtype:
         raise TypeError("q, kcache, vcache must share one dtype")
     B, Hq, Nq, d = q.shape
@@ -269,7 +284,9 @@ def fwd_kvcache(q, kcache, vcache, nk: int, causal: bool = True, scale: Optional
     elif lse is not None:
         _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q.device)
     st = _launch(q.device, stream, lib().fa_fwd_kvcache,
-                 q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(), out.data_ptr(),
+                 q.data_ptr(), kcache.data_ptr(), vcache.data_ptr(),
+                 q_lens.data_ptr() if q_lens is not None else None,
+                 kv_lens.data_ptr() if kv_lens is not None else None, out.data_ptr(),
                  lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, int(nk), cache_len, d,
                  1 if causal else 0, float(scale), _dtype_code(q), owned=owned)
     if st != FA_OK:
@@ -294,15 +311,19 @@ def _check_pool(q, kpool, vpool, block_table):
 
 def fwd_paged(q, kpool, vpool, block_table, nk: int, causal: bool = True,
               scale: Optional[float] = None, out=None, lse=None, return_lse: bool = True,
-              stream=None):
+              stream=None, q_lens=None, kv_lens=None):
     """Prefill against a paged KV cache via ``fa_fwd_paged``: q [B,Hq,Nq,d] attends to the
     first ``nk`` tokens of each sequence, kept in pools [num_pages,Hkv,page_size,d] at the
     pages listed by block_table int32 [B, max_pages] (causal: the chunk is the last Nq of
-    the nk tokens). Returns (o [B,Hq,Nq,d], lse [B,Hq,Nq] fp32 or None).
+    the nk tokens). q_lens / kv_lens (int32 [B] on the device, optional) give sequence b
+    its own nq_b <= Nq query rows and nk_b <= nk tokens; output rows past nq_b are left
+    as they are. Returns (o [B,Hq,Nq,d], lse [B,Hq,Nq] fp32 or None).
     """
     import torch
     _check(q, "q", 4, q.device)
     _check_pool(q, kpool, vpool, block_table)
+    _check_lens(q_lens, "q_lens", q.shape[0], q.device)
+    _check_lens(kv_lens, "kv_lens", q.shape[0], q.device)
     B, Hq, Nq, d = q.shape
     num_pages, Hkv, page_size, _ = kpool.shape
     if scale is None:
@@ -320,7 +341,8 @@ def fwd_paged(q, kpool, vpool, block_table, nk: int, causal: bool = True,
         _check_buf(lse, "lse", (B, Hq, Nq), torch.float32, q.device)
     st = _launch(q.device, stream, lib().fa_fwd_paged,
                  q.data_ptr(), kpool.data_ptr(), vpool.data_ptr(), block_table.data_ptr(),
-                 out.data_ptr(), lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq,
+                 q_lens.data_ptr() if q_lens is not None else None,
+                 kv_lens.data_ptr() if kv_lens is not None else None, out.data_ptr(), lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq,
                  int(nk), num_pages, page_size, block_table.shape[1], d, 1 if causal else 0,
                  float(scale), _dtype_code(q), owned=owned)
     if st != FA_OK:

@@ -84,16 +84,6 @@ static_assert(kTcOffMisc % 16 == 0 && kTcOffSched % 16 == 0 && kTcOffRing % 16 =
 constexpr uint32_t kTcTmemCols = 64;                      // S^T x2 [0,32), O^T x2 [32,64)
 static_assert(kTcSmemBytes <= 227 * 1024, "shared memory budget");
 
-// Debug builds only (-DFA_TC_TRACE): CTA 0 records clock64() at pipeline events of its
-// first 1024 tiles into g_fa_tc_trace[event][tile], read back with fa_debug_tc_trace().
-#ifdef FA_TC_TRACE
-__device__ long long g_fa_tc_trace[8][1024];
-__device__ long long g_fa_tc_clock[148][6];   // per CTA: clock64 / globaltimer at start and end, tiles, SM
-#define FA_TC_EVENT(ev, idx) \
-  do { if (blockIdx.x == 0 && (idx) < 1024) g_fa_tc_trace[ev][idx] = clock64(); } while (0)
-#else
-#define FA_TC_EVENT(ev, idx) do {} while (0)
-#endif
 
 struct DecodeTcParams {
   const int* kv_lens;     // [B]
@@ -207,12 +197,6 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   uint8_t* sbase = smem_raw + (base - raw);
 
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-#ifdef FA_TC_TRACE
-  if (threadIdx.x == 0 && blockIdx.x < 148) {
-    g_fa_tc_clock[blockIdx.x][0] = clock64();
-    g_fa_tc_clock[blockIdx.x][1] = static_cast<long long>(globaltimer_ns());
-  }
-#endif
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -363,21 +347,12 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             ok = false;
             break;
           }
-          if (is_k) FA_TC_EVENT(0, jg); else FA_TC_EVENT(6, jg);
           mbar_arrive_expect_tx(full, kTcTileBytes);
           const uint32_t dst = base + stg * kTcStageBytes + (is_k ? 0 : kTcTileBytes);
           for (int ch = 0; ch < 2; ++ch) tma_load_3d(dst + ch * kTcChunk, tm, full, ch * 64, t, bhkv);
         }
         if (is_k) ticket = static_cast<long long>(gridDim.x) + next_ticket;
       }
-#ifdef FA_TC_TRACE
-      if (is_k && blockIdx.x < 148) {
-        uint32_t smid;
-        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-        g_fa_tc_clock[blockIdx.x][4] = jg;
-        g_fa_tc_clock[blockIdx.x][5] = smid;
-      }
-#endif
       if (!ok || *abort_flag) {
         // Loads still in flight must land before the CTA exits.
         for (int k = max(0, jg - kTcStages); k < jg; ++k)
@@ -571,13 +546,10 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const bool have_next = rn == 1;
         if (have_next) {
           if (!wait_s_inputs(j + 1, nxt)) { ok = false; break; }
-          FA_TC_EVENT(1, j + 1);
           issue_s(j + 1, nxt.unit_last());
         }
         if (!mbar_wait(bar_p(j & 1), (j >> 1) & 1, wc)) { ok = false; break; }
-        FA_TC_EVENT(2, j);
         if (!mbar_wait(bar_vfull(j % kTcStages), (j / kTcStages) & 1, wc)) { ok = false; break; }
-        FA_TC_EVENT(7, j);
         tc_fence_after();
         const uint32_t va = base + (j % kTcStages) * kTcStageBytes + kTcTileBytes;
         const uint32_t pa = base + kTcOffP + (j & 1) * kTcPBytes;
@@ -697,7 +669,6 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       for (int t0 = w.t0; t0 < w.t1; t0 += kTcTile, ++jg, ++tile) {
         bool got = true;
         if (lane == 0) got = mbar_wait(bar_s(jg & 1), (jg >> 1) & 1, wc);
-        if (t == 0) FA_TC_EVENT(3, jg);
         got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
         if (!got) { ok = false; break; }
         tc_fence_after();
@@ -711,7 +682,6 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           mt[h] = x[h];
         }
         if (!exchange(mt, true)) { ok = false; break; }
-        if (t == 0) FA_TC_EVENT(4, jg);
         bool need = false;
         float alpha[kTcN];
 #pragma unroll
@@ -771,7 +741,6 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar_p(jg & 1));
-        if (t == 0) FA_TC_EVENT(5, jg);
         if (tile == 0 && have_prev && !epilogue()) { ok = false; break; }
       }
       if (!ok) break;
@@ -785,12 +754,6 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 
   tc_fence_before();
   __syncthreads();
-#ifdef FA_TC_TRACE
-  if (threadIdx.x == 0 && blockIdx.x < 148) {
-    g_fa_tc_clock[blockIdx.x][2] = clock64();
-    g_fa_tc_clock[blockIdx.x][3] = static_cast<long long>(globaltimer_ns());
-  }
-#endif
   if (warp == kTcWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTcTmemCols);

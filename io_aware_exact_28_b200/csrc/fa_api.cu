@@ -170,11 +170,11 @@ struct KVMaps {
   CUtensorMap k, v, kt, vt;
 };
 
-template <int D, bool BF16, bool CAUSAL, bool PAGED, bool FP8 = false>
+template <int D, bool BF16, bool CAUSAL, bool PAGED, bool FP8 = false, bool VARLEN = false>
 fa_status launch_fwd(int dev, const CUtensorMap& mq, const KVMaps& kv, const fa::FwdParams& prm,
                      cudaStream_t stream) {
   using C = fa::FwdCfg<D, FP8>;
-  auto kernel = fa::fa_fwd_kernel<D, BF16, CAUSAL, PAGED, FP8>;
+  auto kernel = fa::fa_fwd_kernel<D, BF16, CAUSAL, PAGED, FP8, VARLEN>;
   static int attr_state[kMaxDevices];   // 0 unknown, 1 ready, 2 unusable build
   {
     std::lock_guard<std::mutex> lock(g_mu);
@@ -193,21 +193,32 @@ fa_status launch_fwd(int dev, const CUtensorMap& mq, const KVMaps& kv, const fa:
     }
     if (attr_state[dev] != 1) return FA_ERR_UNSUPPORTED;
   }
-  // One CTA per work unit (query block of a (batch, head)); running CTAs take over the
+  // One CTA per work unit (C::QT Q tiles of a (batch, head)); running CTAs take over the
   // ones that have not started, so the grid size only bounds the work, not the residency.
-  const unsigned n_units = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_qb);
-  kernel<<<n_units, C::THREADS, C::SMEM_BYTES, stream>>>(mq, kv.k, kv.v, kv.kt, kv.vt, prm);
+  fa::FwdParams p = prm;
+  const long long n_qb = (p.Nq + C::QT * fa::kBM - 1) / (C::QT * fa::kBM);
+  if (static_cast<long long>(p.BH) * n_qb >= (1LL << 31)) return FA_ERR_INVALID_ARG;
+  p.n_qb = static_cast<int>(n_qb);
+  const unsigned n_units = static_cast<unsigned>(p.BH) * static_cast<unsigned>(p.n_qb);
+  kernel<<<n_units, C::THREADS, C::SMEM_BYTES, stream>>>(mq, kv.k, kv.v, kv.kt, kv.vt, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool VARLEN>
 fa_status dispatch_causal(int causal, bool paged, int dev, const CUtensorMap& mq, const KVMaps& kv,
                           const fa::FwdParams& prm, cudaStream_t st) {
   if (paged)
-    return causal ? launch_fwd<D, BF16, true, true>(dev, mq, kv, prm, st)
-                  : launch_fwd<D, BF16, false, true>(dev, mq, kv, prm, st);
-  return causal ? launch_fwd<D, BF16, true, false>(dev, mq, kv, prm, st)
-                : launch_fwd<D, BF16, false, false>(dev, mq, kv, prm, st);
+    return causal ? launch_fwd<D, BF16, true, true, false, VARLEN>(dev, mq, kv, prm, st)
+                  : launch_fwd<D, BF16, false, true, false, VARLEN>(dev, mq, kv, prm, st);
+  return causal ? launch_fwd<D, BF16, true, false, false, VARLEN>(dev, mq, kv, prm, st)
+                : launch_fwd<D, BF16, false, false, false, VARLEN>(dev, mq, kv, prm, st);
+}
+
+template <int D, bool BF16>
+fa_status dispatch_varlen(bool varlen, int causal, bool paged, int dev, const CUtensorMap& mq,
+                          const KVMaps& kv, const fa::FwdParams& prm, cudaStream_t st) {
+  return varlen ? dispatch_causal<D, BF16, true>(causal, paged, dev, mq, kv, prm, st)
+                : dispatch_causal<D, BF16, false>(causal, paged, dev, mq, kv, prm, st);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -446,10 +457,12 @@ fa_status common_checks(int B, int Hq, int Hkv, int d, float scale, int dtype) {
 }
 
 // fa_fwd, fa_fwd_kvcache and fa_fwd_paged: K/V heads hold kv_rows rows in memory, of which
-// Nk are used; pg != nullptr reads them from a page pool instead.
+// Nk are used; pg != nullptr reads them from a page pool instead. q_lens / kv_lens (device,
+// may be null) give each sequence its own query rows (<= Nq) and keys (<= Nk).
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                    int Hkv, int Nq, int Nk, long long kv_rows, int d, int causal, float scale,
-                   fa_dtype dtype, const PagedArgs* pg, void* stream) {
+                   fa_dtype dtype, const PagedArgs* pg, void* stream, const int* q_lens = nullptr,
+                   const int* kv_lens = nullptr) {
   if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
   if (Nq <= 0 || Nk <= 0 || (causal != 0 && causal != 1)) return FA_ERR_INVALID_ARG;
   fa_status s = common_checks(B, Hq, Hkv, d, scale, dtype);
@@ -462,15 +475,16 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   const long long BH = static_cast<long long>(B) * Hq;
   const long long BHkv = static_cast<long long>(B) * Hkv;
   if (BH >= (1LL << 31)) return FA_ERR_INVALID_ARG;
-  const long long n_qb = (Nq + fa::kQTiles * fa::kBM - 1) / (fa::kQTiles * fa::kBM);
-  if (BH * n_qb >= (1LL << 31)) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGNMENT;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(q_lens) & 3u) || (reinterpret_cast<uintptr_t>(kv_lens) & 3u))
+    return FA_ERR_ALIGNMENT;
   int dev = 0;
   s = check_device(&dev);
   if (s != FA_OK) return s;
 
   const bool bf16 = dtype == FA_BF16;
+  const bool varlen = q_lens != nullptr || kv_lens != nullptr;
   CUtensorMap mq;
   KVMaps kv;
   const int kv_box = (d == 64) ? fa::FwdCfg<64>::BN : fa::FwdCfg<128>::BN;
@@ -479,6 +493,8 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     // [num_pages*Hkv, page_size, d] views; the tail maps end at the last page's used rows.
     const long long heads = static_cast<long long>(pg->num_pages) * Hkv;
     const int box = pg->page_size < kv_box ? pg->page_size : kv_box;
+    // (Per-sequence lengths do without tail maps: the kernel zeroes V rows past each
+    // sequence's last key in shared memory.)
     const int tail_rows = Nk - ((Nk - 1) / pg->page_size) * pg->page_size;
     if (!make_tile_map(&kv.k, k, d, pg->page_size, heads, bf16, box) ||
         !make_tile_map(&kv.v, v, d, pg->page_size, heads, bf16, box) ||
@@ -497,7 +513,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   prm.o = o;
   prm.lse = lse;
   prm.BH = static_cast<int>(BH);
-  prm.n_qb = static_cast<int>(n_qb);
+  prm.n_qb = 0;   // set per configuration at launch
   prm.Hq = Hq;
   prm.Hkv = Hkv;
   prm.group = Hq / Hkv;
@@ -510,13 +526,15 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   prm.o_scale = 1.f;
   prm.pk = pg ? pg->device(Hkv) : fa::PagedKV{};
   prm.last_page = pg ? (Nk - 1) / pg->page_size : 0;
+  prm.q_lens = q_lens;
+  prm.kv_lens = kv_lens;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool paged = pg != nullptr;
   if (d == 64)
-    return bf16 ? dispatch_causal<64, true>(causal, paged, dev, mq, kv, prm, st)
-                : dispatch_causal<64, false>(causal, paged, dev, mq, kv, prm, st);
-  return bf16 ? dispatch_causal<128, true>(causal, paged, dev, mq, kv, prm, st)
-              : dispatch_causal<128, false>(causal, paged, dev, mq, kv, prm, st);
+    return bf16 ? dispatch_varlen<64, true>(varlen, causal, paged, dev, mq, kv, prm, st)
+                : dispatch_varlen<64, false>(varlen, causal, paged, dev, mq, kv, prm, st);
+  return bf16 ? dispatch_varlen<128, true>(varlen, causal, paged, dev, mq, kv, prm, st)
+              : dispatch_varlen<128, false>(varlen, causal, paged, dev, mq, kv, prm, st);
 }
 }  // namespace
 
@@ -589,12 +607,13 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
               : launch_bwd<128, false>(dev, mp, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st);
 }
 
-fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* vcache, void* o,
-                         float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int cache_len,
-                         int d, int causal, float scale, fa_dtype dtype, void* stream) {
+fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* vcache,
+                         const int* q_lens, const int* kv_lens, void* o, float* lse, int B,
+                         int Hq, int Hkv, int Nq, int Nk, int cache_len, int d, int causal,
+                         float scale, fa_dtype dtype, void* stream) {
   if (cache_len < Nk || cache_len <= 0) return FA_ERR_INVALID_ARG;
   return fwd_impl(q, kcache, vcache, o, lse, B, Hq, Hkv, Nq, Nk, cache_len, d, causal, scale,
-                  dtype, nullptr, stream);
+                  dtype, nullptr, stream, q_lens, kv_lens);
 }
 
 fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -610,8 +629,6 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
   const long long BH = static_cast<long long>(B) * Hq;
   const long long BHkv = static_cast<long long>(B) * Hkv;
   if (BH >= (1LL << 31)) return FA_ERR_INVALID_ARG;
-  const long long n_qb = (Nq + fa::kQTiles * fa::kBM - 1) / (fa::kQTiles * fa::kBM);
-  if (BH * n_qb >= (1LL << 31)) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGNMENT;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return FA_ERR_ALIGNMENT;
   int dev = 0;
@@ -631,7 +648,7 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
   prm.o = o;
   prm.lse = lse;
   prm.BH = static_cast<int>(BH);
-  prm.n_qb = static_cast<int>(n_qb);
+  prm.n_qb = 0;   // set per configuration at launch
   prm.Hq = Hq;
   prm.Hkv = Hkv;
   prm.group = Hq / Hkv;
@@ -645,18 +662,21 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
   prm.pk = fa::PagedKV{};
   prm.last_page = 0;
   prm.o_scale = v_descale;
+  prm.q_lens = nullptr;
+  prm.kv_lens = nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return causal ? launch_fwd<128, true, true, false, true>(dev, mq, kv, prm, st)
                 : launch_fwd<128, true, false, false, true>(dev, mq, kv, prm, st);
 }
 
 fa_status fa_fwd_paged(const void* q, const void* kpool, const void* vpool, const int* block_table,
-                       void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int num_pages,
-                       int page_size, int max_pages_per_seq, int d, int causal, float scale,
-                       fa_dtype dtype, void* stream) {
+                       const int* q_lens, const int* kv_lens, void* o, float* lse, int B, int Hq,
+                       int Hkv, int Nq, int Nk, int num_pages, int page_size,
+                       int max_pages_per_seq, int d, int causal, float scale, fa_dtype dtype,
+                       void* stream) {
   const PagedArgs pg{block_table, num_pages, page_size, max_pages_per_seq};
   return fwd_impl(q, kpool, vpool, o, lse, B, Hq, Hkv, Nq, Nk, 0, d, causal, scale, dtype, &pg,
-                  stream);
+                  stream, q_lens, kv_lens);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq) {
@@ -853,19 +873,6 @@ void fa_set_wait_timeout_ns(uint64_t ns) {
 }
 
 void fa_debug_skip_q_load(int enable) { g_skip_q_load.store(enable ? 1 : 0, std::memory_order_relaxed); }
-
-#ifdef FA_TC_TRACE
-// Debug builds only: copy the tensor-core decode trace (8 events x 1024 tiles of clock64).
-FA_API int fa_debug_tc_trace(long long* host, int n) {
-  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-  const size_t bytes = sizeof(long long) * static_cast<size_t>(n < 8 * 1024 ? n : 8 * 1024);
-  return cudaMemcpyFromSymbol(host, fa::g_fa_tc_trace, bytes) == cudaSuccess ? 0 : -1;
-}
-FA_API int fa_debug_tc_clock(long long* host) {
-  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-  return cudaMemcpyFromSymbol(host, fa::g_fa_tc_clock, sizeof(long long) * 148 * 6) == cudaSuccess ? 0 : -1;
-}
-#endif
 
 const char* fa_build_info(void) { return "libfa_b200 0.1 sm_100a (tcgen05/TMA prefill, split-KV decode)"; }
 

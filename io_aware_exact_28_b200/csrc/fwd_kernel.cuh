@@ -40,25 +40,23 @@
 #include <cuda.h>
 #include <math_constants.h>
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace fa {
 
 constexpr int kBM = 128;           // query rows per Q tile (one TMEM lane per row)
-constexpr int kQTiles = 2;         // Q tiles per CTA
-constexpr int kWarpProducer = 8;
-constexpr int kWarpMma = 9;
+struct EmptyBase {};
 
-// Polynomial-exp2 pair masks (see FwdCfg::kEmuPairs); off by default: measured slower on
-// B200 at both head dimensions, because the softmax is latency-bound, not MUFU-bound.
-#ifndef FA_EMU_PAIRS_D64
-#define FA_EMU_PAIRS_D64 0u
-#endif
-#ifndef FA_EMU_PAIRS_D128
-#define FA_EMU_PAIRS_D128 0u
-#endif
+// Keys per K/V tile at d = 64 (64: two CTAs per SM; 128: the d = 128 structure, one CTA
+// per SM, measured slower on the mha2k workload).
 #ifndef FA_D64_BN
 #define FA_D64_BN 64
+#endif
+// d = 128: load S in 32-column chunks with the next chunk in flight (1) or in one load (0).
+#ifndef FA_D128_PIPE
+#define FA_D128_PIPE 0
 #endif
 #ifndef FA_REGSPLIT
 #define FA_REGSPLIT 1
@@ -78,11 +76,14 @@ struct FwdCfg {
   static constexpr int ELEM = FP8 ? 1 : 2;            // bytes per Q/K/V element
   static constexpr int ROWB = D * ELEM;               // bytes per Q/K/V row
   static constexpr int BN = (D == 64) ? FA_D64_BN : 128;   // keys per K/V tile
+  static constexpr int QT = 2;                         // 128-row Q tiles per CTA
   static constexpr bool NARROW = (BN == 64);          // 64-key tiles, two CTAs per SM
   static constexpr int CTAS = NARROW ? 2 : 1;         // resident CTAs per SM
   // 128-key tiles: 3 warpgroups (warps 10-11 idle) so the register re-split below can
   // apply; 64-key tiles: 10 warps, two CTAs per SM share the register file (96 each).
   static constexpr int THREADS = NARROW ? 320 : 384;
+  static constexpr int WARP_PRODUCER = 4 * QT;        // TMA producer warp
+  static constexpr int WARP_MMA = 4 * QT + 1;         // TMEM allocator and MMA issuer
   static constexpr bool REGSPLIT = !NARROW && FA_REGSPLIT;
   static constexpr int NCH = ROWB / 128;              // 128-byte swizzle chunks along d
   static constexpr int OCH = D / 64;                  // 64-column chunks of an O row
@@ -100,16 +101,16 @@ struct FwdCfg {
   static constexpr float TAU = FP8 ? 4.f : 8.f;
   static constexpr float OFF = FP8 ? 4.f : 0.f;
   static constexpr int Q_OFF = 0;
-  static constexpr int KV_OFF = kQTiles * Q_TILE_BYTES;
+  static constexpr int KV_OFF = QT * Q_TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NS * KV_TILE_BYTES;
-  // q, full[NS], empty[NS], s[2], p[2], o[2], qempty, clc_full[2], clc_empty[2], drain
-  static constexpr int NBARS = 1 + 2 * NS + 3 * kQTiles + 1 + 4 + 1;
+  // q, full[NS], empty[NS], s[2], p[2], o[2], qempty, clc_full[2], clc_empty[2], drain, tail
+  static constexpr int NBARS = 1 + 2 * NS + 3 * QT + 1 + 4 + 1 + 1;
   static constexpr int CLC_OFF = BAR_OFF + ((NBARS * 8 + 15) / 16) * 16;   // 2 x 16-byte responses
   static constexpr int MISC_OFF = CLC_OFF + 32;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;   // + slack for 1 KB alignment
   static constexpr uint32_t TMEM_COLS = NARROW ? 256 : 512;
   static constexpr uint32_t S_COL = 0;                // S_t at t * BN
-  static constexpr uint32_t O_COL = kQTiles * BN;     // O_t at O_COL + t * D
+  static constexpr uint32_t O_COL = QT * BN;          // O_t at O_COL + t * D
   // Registers per thread: the launch allocation (65536 / (threads * CTAS), rounded down
   // to 8) is re-split so that warpgroup 2 (producer, MMA, 2 idle warps) keeps REGS_OTHER
   // and the two softmax warpgroups get REGS_SOFTMAX; the split uses exactly the launch
@@ -120,9 +121,7 @@ struct FwdCfg {
   static_assert(!REGSPLIT || 128 * REGS_OTHER + 256 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH,
                 "register split");
   static_assert(THREADS * REGS_LAUNCH * CTAS <= 65536, "register file");
-  // Which of every 8 consecutive P column pairs use the polynomial exp2 (bit i = pair i).
-  static constexpr uint32_t kEmuPairs = FP8 ? 0u : (D == 64) ? FA_EMU_PAIRS_D64 : FA_EMU_PAIRS_D128;
-  static_assert(O_COL + kQTiles * D <= TMEM_COLS, "TMEM budget");
+  static_assert(O_COL + QT * D <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES * CTAS <= 227 * 1024, "shared memory budget");
 };
 
@@ -130,7 +129,7 @@ struct FwdParams {
   void* o;              // [B*Hq, Nq, D], 16-bit
   float* lse;           // [B*Hq, Nq] or nullptr
   int BH;               // B * Hq
-  int n_qb;             // query blocks of kQTiles * kBM rows per (batch, head)
+  int n_qb;             // query blocks of QT * kBM rows per (batch, head)
   int Hq, Hkv, group;   // group = Hq / Hkv
   int Nq, Nk;
   int causal_offset;    // Nk - Nq (bottom-right alignment)
@@ -140,6 +139,8 @@ struct FwdParams {
   PagedKV pk;           // PAGED kernels only
   int last_page;        // PAGED: page index (t / page_size) of key Nk - 1
   float o_scale;        // FP8 kernels: multiplies O (the descale of V)
+  const int* q_lens;    // VARLEN: [B] query rows of each sequence (nullptr: Nq for all)
+  const int* kv_lens;   // VARLEN: [B] keys of each sequence (nullptr: Nk for all)
 };
 
 template <int D>
@@ -170,13 +171,13 @@ __device__ __forceinline__ void rescale_p_cols(uint32_t taddr, float alpha) {
   tmem_st_wait();
 }
 
-template <int D, bool BF16, bool CAUSAL, bool PAGED, bool FP8 = false>
+template <int D, bool BF16, bool CAUSAL, bool PAGED, bool FP8 = false, bool VARLEN = false>
 __global__ void __launch_bounds__(FwdCfg<D, FP8>::THREADS, FwdCfg<D, FP8>::CTAS)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
               const __grid_constant__ CUtensorMap tmVt, const FwdParams p) {
   using C = FwdCfg<D, FP8>;
-  static_assert(!FP8 || (D == 128 && !PAGED), "FP8: d = 128, contiguous K/V");
+  static_assert(!FP8 || (D == 128 && !PAGED && !VARLEN), "FP8: d = 128, contiguous K/V");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -185,31 +186,53 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   constexpr int kBN = C::BN;
-  const int n_kv_total = (p.Nk + kBN - 1) / kBN;
 
   // Work unit u covers query block qb of (batch, head) bh; units are numbered heaviest
   // causal block first, which is also the order in which the hardware starts CTAs and
   // hands out not-yet-started CTAs to running ones.
   // n_t[t]: key tiles query tile t visits. A tile past the last query row visits none,
   // and under the causal mask a tile stops at the key tile of its last row's diagonal.
-  struct Unit {
+  // Lengths of the unit's sequence: query rows nq and keys nk (Nq and Nk, unless VARLEN
+  // gives per-sequence lengths, clamped to [0, Nq] and [0, Nk]); off = nk - nq aligns the
+  // causal mask to the end of the sequence. Only VARLEN units carry them; the others read
+  // the kernel parameters, so that no role keeps three more registers live.
+  const int n_kv_all = (p.Nk + kBN - 1) / kBN;   // key tiles of a sequence of Nk keys
+  struct Lens {
+    int nq, nk;
+  };
+  struct Unit : std::conditional_t<VARLEN, Lens, EmptyBase> {
     int bh, bh_kv, q0;
-    int n_t[kQTiles];
+    int n_t[C::QT];
     int n_kv;           // key tiles the unit loads: max over its query tiles
+  };
+  auto u_nq = [&](const Unit& w) -> int {
+    if constexpr (VARLEN) return w.nq; else return p.Nq;
+  };
+  auto u_nk = [&](const Unit& w) -> int {
+    if constexpr (VARLEN) return w.nk; else return p.Nk;
+  };
+  auto u_off = [&](const Unit& w) -> int {
+    if constexpr (VARLEN) return w.nk - w.nq; else return p.causal_offset;
   };
   auto decode_unit = [&](int u) {
     Unit w;
     const int qb = p.n_qb - 1 - u / p.BH;
     w.bh = u - (u / p.BH) * p.BH;
     w.bh_kv = (w.bh / p.Hq) * p.Hkv + (w.bh % p.Hq) / p.group;
-    w.q0 = qb * (kQTiles * kBM);
+    w.q0 = qb * (C::QT * kBM);
     w.n_kv = 0;
+    if constexpr (VARLEN) {
+      const int b = w.bh / p.Hq;
+      w.nq = p.q_lens ? min(max(__ldg(p.q_lens + b), 0), p.Nq) : p.Nq;
+      w.nk = p.kv_lens ? min(max(__ldg(p.kv_lens + b), 0), p.Nk) : p.Nk;
+    }
+    const int n_kv_total = VARLEN ? (u_nk(w) + kBN - 1) / kBN : n_kv_all;
 #pragma unroll
-    for (int t = 0; t < kQTiles; ++t) {
+    for (int t = 0; t < C::QT; ++t) {
       const int row_first = w.q0 + t * kBM;
-      int n = row_first < p.Nq ? n_kv_total : 0;
+      int n = row_first < u_nq(w) ? n_kv_total : 0;
       if (CAUSAL && n > 0) {
-        const int kmax = min(row_first + kBM - 1, p.Nq - 1) + p.causal_offset;
+        const int kmax = min(row_first + kBM - 1, u_nq(w) - 1) + u_off(w);
         n = kmax < 0 ? 0 : min(n_kv_total, kmax / kBN + 1);
       }
       w.n_t[t] = n;
@@ -223,17 +246,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   auto bar_full = [&](int i) { return bar0 + 8u * (1 + i); };
   auto bar_empty = [&](int i) { return bar0 + 8u * (1 + C::NS + i); };
   auto bar_s = [&](int t) { return bar0 + 8u * (1 + 2 * C::NS + t); };
-  auto bar_p = [&](int t) { return bar0 + 8u * (1 + 2 * C::NS + kQTiles + t); };
-  auto bar_o = [&](int t) { return bar0 + 8u * (1 + 2 * C::NS + 2 * kQTiles + t); };
-  const uint32_t bar_qempty = bar0 + 8u * (1 + 2 * C::NS + 3 * kQTiles);
-  auto bar_clc_full = [&](int i) { return bar0 + 8u * (2 + 2 * C::NS + 3 * kQTiles + i); };
-  auto bar_clc_empty = [&](int i) { return bar0 + 8u * (4 + 2 * C::NS + 3 * kQTiles + i); };
-  const uint32_t bar_drain = bar0 + 8u * (6 + 2 * C::NS + 3 * kQTiles);
+  auto bar_p = [&](int t) { return bar0 + 8u * (1 + 2 * C::NS + C::QT + t); };
+  auto bar_o = [&](int t) { return bar0 + 8u * (1 + 2 * C::NS + 2 * C::QT + t); };
+  const uint32_t bar_qempty = bar0 + 8u * (1 + 2 * C::NS + 3 * C::QT);
+  auto bar_clc_full = [&](int i) { return bar0 + 8u * (2 + 2 * C::NS + 3 * C::QT + i); };
+  auto bar_clc_empty = [&](int i) { return bar0 + 8u * (4 + 2 * C::NS + 3 * C::QT + i); };
+  const uint32_t bar_drain = bar0 + 8u * (6 + 2 * C::NS + 3 * C::QT);
+  const uint32_t bar_tail = bar0 + 8u * (7 + 2 * C::NS + 3 * C::QT);   // VARLEN: ragged V tile
   auto clc_resp = [&](int i) { return base + C::CLC_OFF + 16u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + C::MISC_OFF + 4);
   // Readers of each scheduling response: the MMA thread and the 8 softmax warps.
-  constexpr int kClcReaders = 1 + 2 * kQTiles * 2;
+  constexpr int kClcReaders = 1 + 4 * C::QT;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q(), 1);
@@ -241,7 +265,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_init(bar_full(i), 1);
       mbar_init(bar_empty(i), 1);
     }
-    for (int t = 0; t < kQTiles; ++t) {
+    for (int t = 0; t < C::QT; ++t) {
       mbar_init(bar_s(t), 1);
       mbar_init(bar_p(t), kBM);
       mbar_init(bar_o(t), 1);
@@ -252,11 +276,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_init(bar_clc_empty(i), kClcReaders);
     }
     mbar_init(bar_drain, 1);
+    mbar_init(bar_tail, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == kWarpMma) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
-  if (warp == kWarpProducer && lane == 0) {
+  if (warp == C::WARP_MMA) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+  if (warp == C::WARP_PRODUCER && lane == 0) {
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
@@ -274,12 +299,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   // Each role's code sits inside the branch that set its register budget. Every role
   // walks the same unit sequence: its own blockIdx.x, then the CTAs the producer takes
   // over, published through clc_resp[k & 1] (k = units finished).
-  if (warp >= 2 * 4) {
+  if (warp >= 4 * C::QT) {
     if constexpr (C::REGSPLIT) setmaxnreg_dec<C::REGS_OTHER>();
-    if (warp == kWarpProducer) {
+    if (warp == C::WARP_PRODUCER) {
     // ------------------------------------------------------------------ TMA producer
-    // Contiguous K/V: lane 0 alone issues every copy (one box per 64 columns of a tile).
-    if constexpr (!PAGED) {
+    // Contiguous K/V of one length: lane 0 alone issues every copy (one box per 64 columns
+    // of a tile).
+    if constexpr (!PAGED && !VARLEN) {
     if (lane == 0) {
       int unit = blockIdx.x, k = 0, it = 0, q_loads = 0;
       bool ok = true, clc_pending = false;
@@ -291,10 +317,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           if (q_loads > 0 && !mbar_wait(bar_qempty, (q_loads - 1) & 1, wc)) { ok = false; break; }
           int q_tiles = 0;
 #pragma unroll
-          for (int t = 0; t < kQTiles; ++t) q_tiles += w.n_t[t] > 0 ? 1 : 0;
+          for (int t = 0; t < C::QT; ++t) q_tiles += w.n_t[t] > 0 ? 1 : 0;
           mbar_arrive_expect_tx(bar_q(), q_tiles * C::Q_TILE_BYTES);
 #pragma unroll
-          for (int t = 0; t < kQTiles; ++t) {
+          for (int t = 0; t < C::QT; ++t) {
             if (w.n_t[t] == 0) continue;
             for (int ch = 0; ch < C::NCH; ++ch)
               tma_load_3d(base + C::Q_OFF + t * C::Q_TILE_BYTES + ch * C::Q_CHUNK, &tmQ, bar_q(),
@@ -345,10 +371,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // The whole warp walks the units. Lane 0 waits on the ring, arms the barriers, loads Q
     // and takes over CTAs; its decisions reach the other lanes through shuffles. Paged:
     // lane i reads the table entry of page i of a key tile and issues that page's boxes,
-    // so a tile of small pages costs one table read and NCH boxes per lane.
+    // so a tile of small pages costs one table read and NCH boxes per lane. VARLEN: the V
+    // tile that holds a sequence's last key lands on bar_tail first; the warp then zeroes
+    // its rows past that key (whatever the cache holds there, P = 0 multiplies zeros) and
+    // only then completes the ring slot.
     const bool leader = lane == 0;
-    int unit = blockIdx.x, k = 0, it = 0, q_loads = 0;
-    bool ok = true, clc_pending = false;
+    int unit = blockIdx.x, k = 0, it = 0, q_loads = 0, tail_uses = 0;
+    bool ok = true, clc_pending = false, tail_pending = false;
     while (true) {
       const Unit w = decode_unit(unit);
       // A query tile with no visible key writes zeros and needs no Q.
@@ -360,10 +389,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           } else {
             int q_tiles = 0;
 #pragma unroll
-            for (int t = 0; t < kQTiles; ++t) q_tiles += w.n_t[t] > 0 ? 1 : 0;
+            for (int t = 0; t < C::QT; ++t) q_tiles += w.n_t[t] > 0 ? 1 : 0;
             mbar_arrive_expect_tx(bar_q(), q_tiles * C::Q_TILE_BYTES);
 #pragma unroll
-            for (int t = 0; t < kQTiles; ++t) {
+            for (int t = 0; t < C::QT; ++t) {
               if (w.n_t[t] == 0) continue;
               for (int ch = 0; ch < C::NCH; ++ch)
                 tma_load_3d(base + C::Q_OFF + t * C::Q_TILE_BYTES + ch * C::Q_CHUNK, &tmQ, bar_q(),
@@ -386,17 +415,19 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           y = (j * kBN) & (ps - 1) & ~(kBN - 1);   // row of the tile in a large page
           const int b = w.bh_kv / p.Hkv;
           const int tok = j * kBN + lane * rows;
-          have = lane * rows < kBN && tok < p.Nk;
+          have = lane * rows < kBN && tok < u_nk(w);
           if (have) entry = paged_entry(p.pk, b, tok);
         }
         for (int kv = 0; kv < 2; ++kv) {
           const int slot = it % C::NS;
           const int round = it / C::NS;
+          const bool zero_tail = VARLEN && kv == 1 && (j + 1) * kBN > u_nk(w);
+          const uint32_t land = zero_tail ? bar_tail : bar_full(slot);
           if (leader) {
             if (round > 0 && !mbar_wait(bar_empty(slot), (round - 1) & 1, wc))
               ok = false;
             else
-              mbar_arrive_expect_tx(bar_full(slot), C::KV_TILE_BYTES);
+              mbar_arrive_expect_tx(land, C::KV_TILE_BYTES);
           }
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
           if (!ok) break;
@@ -408,16 +439,35 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 const int kvh = w.bh_kv - (w.bh_kv / p.Hkv) * p.Hkv;
                 z = have ? paged_z(p.pk, entry, kvh) : paged_z_oob(p.pk);
               }
-              const bool tail = have && (tok >> p.pk.page_shift) == p.last_page;
+              const bool tail = !VARLEN && have && (tok >> p.pk.page_shift) == p.last_page;
               const CUtensorMap* tm = kv ? (tail ? &tmVt : &tmV) : (tail ? &tmKt : &tmK);
               for (int ch = 0; ch < C::NCH; ++ch)
-                tma_load_3d(dst + ch * C::KV_CHUNK + lane * rows * 128, tm, bar_full(slot), ch * 64,
-                            y, z);
+                tma_load_3d(dst + ch * C::KV_CHUNK + lane * rows * 128, tm, land, ch * 64, y, z);
             }
           } else if (leader) {
             const CUtensorMap* tm = kv ? &tmV : &tmK;
             for (int ch = 0; ch < C::NCH; ++ch)
-              tma_load_3d(dst + ch * C::KV_CHUNK, tm, bar_full(slot), ch * 64, j * kBN, w.bh_kv);
+              tma_load_3d(dst + ch * C::KV_CHUNK, tm, land, ch * 64, j * kBN, w.bh_kv);
+          }
+          if (zero_tail) {
+            // Rows [nk - j*BN, BN) of the landed V tile: 128 bytes per row and swizzle chunk
+            // (the swizzle permutes 16-byte pieces within a row, so whole rows stay whole).
+            tail_pending = true;
+            if (leader && !mbar_wait(bar_tail, tail_uses & 1, wc)) ok = false;
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            tail_pending = false;
+            ++tail_uses;
+            const int r0 = u_nk(w) - j * kBN;
+            const int n16 = (kBN - r0) * 8;                  // 16-byte pieces per chunk
+            const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+            for (int ch = 0; ch < C::NCH; ++ch)
+              for (int i = lane; i < n16; i += 32)
+                *reinterpret_cast<uint4*>(sbase + C::KV_OFF + slot * C::KV_TILE_BYTES +
+                                          ch * C::KV_CHUNK + r0 * 128 + i * 16) = zero;
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (leader) mbar_arrive(bar_full(slot));
           }
           ++it;
         }
@@ -452,14 +502,15 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     }
     if (leader && (!ok || *abort_flag)) {
       // Copies still in flight must land before the CTA exits (copies issued by any lane
-      // complete on the same ring barriers).
+      // complete on the same ring barriers, or on bar_tail).
       for (int i = max(0, it - C::NS); i < it; ++i)
         mbar_wait_drain(bar_full(i % C::NS), (i / C::NS) & 1, kDrainNs);
+      if (tail_pending) mbar_wait_drain(bar_tail, tail_uses & 1, kDrainNs);
       if (q_loads > 0) mbar_wait_drain(bar_q(), (q_loads - 1) & 1, kDrainNs);
       if (clc_pending) mbar_wait_drain(bar_clc_full(k & 1), (k >> 1) & 1, kDrainNs);
     }
     }
-    } else if (warp == kWarpMma) {
+    } else if (warp == C::WARP_MMA) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       // Format code: fp16 0 / bf16 1 under kind::f16; E4M3 is code 0 under kind::f8f6f4.
@@ -494,9 +545,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       };
       int unit = blockIdx.x, k = 0, it = 0, q_uses = 0;
-      int p_seen[kQTiles];
+      int p_seen[C::QT];
 #pragma unroll
-      for (int t = 0; t < kQTiles; ++t) p_seen[t] = 0;
+      for (int t = 0; t < C::QT; ++t) p_seen[t] = 0;
       bool ok = true, issued = false;
       while (ok) {
         const Unit w = decode_unit(unit);
@@ -514,7 +565,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (j > 0 && !mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
-            for (int t = 0; t < kQTiles; ++t) {
+            for (int t = 0; t < C::QT; ++t) {
               if (j > 0 && j - 1 < w.n_t[t]) {
                 if (!mbar_wait(bar_p(t), p_seen[t] & 1, wc)) { ok = false; break; }
                 ++p_seen[t];
@@ -537,7 +588,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const int vit = it + 2 * w.n_kv - 1, vslot = vit % C::NS;
             ok = mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc);
 #pragma unroll
-            for (int t = 0; t < kQTiles; ++t) {
+            for (int t = 0; t < C::QT; ++t) {
               if (!ok || w.n_t[t] != w.n_kv) continue;
               if (!mbar_wait(bar_p(t), p_seen[t] & 1, wc)) { ok = false; break; }
               ++p_seen[t];
@@ -579,11 +630,14 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     bool ok = true;
     while (true) {
       const Unit w = decode_unit(unit);
-      const int n_t = t == 0 ? w.n_t[0] : w.n_t[kQTiles - 1];
+      int n_t = 0;   // this warp's tile, selected with static indices (no local memory)
+#pragma unroll
+      for (int tt = 0; tt < C::QT; ++tt)
+        if (tt == t) n_t = w.n_t[tt];
       const int row = w.q0 + t * kBM + r;
       const int row_min = w.q0 + t * kBM;
-      const int lim = CAUSAL ? min(row + p.causal_offset, p.Nk - 1) : p.Nk - 1;
-      const int lim_min = CAUSAL ? min(row_min + p.causal_offset, p.Nk - 1) : p.Nk - 1;
+      const int lim = CAUSAL ? min(row + u_off(w), u_nk(w) - 1) : u_nk(w) - 1;
+      const int lim_min = CAUSAL ? min(row_min + u_off(w), u_nk(w) - 1) : u_nk(w) - 1;
 
       float m_used = -CUDART_INF_F;
       float l = 0.f;
@@ -620,8 +674,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         // P = 2^(s*c - mref) in 32-column chunks, each stored to TMEM as 16 packed columns
         // (P_t occupies S_t columns [0, BN/2); chunk cc only overwrites columns already
         // read); returns the row sum of the unrounded fp32 P. With track, the row maximum
-        // of the scores is gathered in mx8 on the way. In tiles without masked scores, the
-        // pairs selected by kEmuPairs use the FMA-pipe polynomial instead of MUFU.EX2.
+        // of the scores is gathered in mx8 on the way.
         // P of one 32-column chunk v (scores of keys 32 cc ..) against mref, stored as 16
         // packed columns at tS + 16 cc; returns its row sum (unrounded fp32 P). With track,
         // the scores' maximum is gathered in mx8 on the way.
@@ -664,14 +717,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 mx8[i & 7] = fmax3(mx8[i & 7], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
               const uint64_t x2 =
                   f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2);
-              uint64_t p2;
-              if (!masked_tile && ((C::kEmuPairs >> (i & 7)) & 1u)) {
-                p2 = exp2_poly_f2(x2);
-              } else {
-                float x0, x1;
-                f2_unpack(x2, x0, x1);
-                p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
-              }
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              const uint64_t p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
               if (i & 1) l2b = f2_add(l2b, p2); else l2a = f2_add(l2a, p2);
               float p0, p1;
               f2_unpack(p2, p0, p1);
@@ -725,6 +773,25 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           if (grow) m_used = mx;
           return __any_sync(0xffffffffu, grow);
         };
+#if FA_D128_PIPE
+        // Every row of the warp has a running max: P of each 32-column chunk against it,
+        // with the next chunk's TMEM load in flight meanwhile (P of chunk c goes to columns
+        // [16c, 16c+16), which hold scores already loaded, never ones still in flight).
+        if (kResident && __all_sync(0xffffffffu, m_used != -CUDART_INF_F)) {
+          tmem_ld32x32b_x32_async(tS, &sr[0]);
+          tmem_ld_wait_tied32(&sr[0]);
+          float lsum = 0.f;
+#pragma unroll
+          for (int cc = 0; cc < kBN / 32; ++cc) {
+            if (cc + 1 < kBN / 32) tmem_ld32x32b_x32_async(tS + 32 * (cc + 1), &sr[32 * (cc + 1)]);
+            mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]), cc);
+            lsum += chunk_p(&sr[32 * cc], cc, m_used, true);
+            if (cc + 1 < kBN / 32) tmem_ld_wait_tied32(&sr[32 * (cc + 1)]);
+          }
+          if (raise_max()) lsum = p_pass(m_used, false);
+          l += lsum;
+        } else
+#endif
         if constexpr (kResident) {
           tmem_ld32x32b_x128(tS, sr);
 #pragma unroll
@@ -798,7 +865,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       // thread), then LSE = (m + log2 l) ln 2. A tile that saw no key writes zeros / -inf.
       // Every lane loads from TMEM (warp-collective); rows past Nq store nothing.
       {
-        const bool row_ok = row < p.Nq;
+        const bool row_ok = row < u_nq(w);
         uint16_t* orow = static_cast<uint16_t*>(p.o) +
                          (static_cast<size_t>(w.bh) * p.Nq + (row_ok ? row : 0)) * D;
         float inv_l = (l > 0.f) ? 1.f / l : 0.f;
@@ -845,7 +912,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpMma) {
+  if (warp == C::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -33,7 +33,8 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["attention_f64", "attention_rows_f64", "decode_f64", "visible_mask"]
+__all__ = ["attention_f64", "attention_rows_f64", "attention_varlen_f64", "decode_f64",
+           "visible_mask"]
 
 
 def _f64(x) -> np.ndarray:
@@ -122,4 +123,39 @@ def decode_f64(q, kcache, vcache, kv_lens, scale: float):
             S = scale * (Qh @ K.T)
             o, l = _softmax_rows(S, np.ones_like(S, dtype=bool), V)
             O[b, h], L[b, h] = o[0], l[0]
+    return O, L
+
+
+def attention_varlen_f64(q, k, v, q_lens, kv_lens, causal: bool, scale: float):
+    """Sequences of different lengths in one batch: sequence b has q_lens[b] query rows (the
+    first rows of q[b]) and kv_lens[b] keys and values (the first rows of k[b], v[b]), and
+    is its own attention problem, its causal mask aligned to its own end (key j visible to
+    query i iff j <= i + kv_lens[b] - q_lens[b]). This is the per-session cache of page
+    "Flash Attention ... IO-aware exact" (fr), KV-cache section (each session holds its own
+    number of tokens), with the plain definition applied to each session.
+
+    q: [B,Hq,Nq,d]; k, v: [B,Hkv,Nk,d]; lengths within [0, Nq] and [0, Nk]. Returns O
+    [B,Hq,Nq,d] and LSE [B,Hq,Nq] (float64); rows past q_lens[b] are NaN (no result)."""
+    B, Hq, Nq, d = q.shape
+    Hkv = k.shape[1]
+    g = Hq // Hkv
+    qn = np.asarray(_f64(q_lens), dtype=np.int64)
+    kn = np.asarray(_f64(kv_lens), dtype=np.int64)
+    O = np.full((B, Hq, Nq, d), np.nan, dtype=np.float64)
+    L = np.full((B, Hq, Nq), np.nan, dtype=np.float64)
+    for b in range(B):
+        nq, nk = int(qn[b]), int(kn[b])
+        if nq <= 0:
+            continue
+        rows = np.arange(nq)
+        for h in range(Hq):
+            if nk <= 0:
+                O[b, h, :nq] = 0.0
+                L[b, h, :nq] = -np.inf
+                continue
+            Q = _f64(q[b, h])[:nq]
+            K = _f64(k[b, h // g])[:nk]
+            V = _f64(v[b, h // g])[:nk]
+            S = scale * (Q @ K.T)
+            O[b, h, :nq], L[b, h, :nq] = _softmax_rows(S, visible_mask(rows, nq, nk, causal), V)
     return O, L

@@ -28,9 +28,10 @@ from __future__ import annotations
 
 import numpy as np
 
-from .attention import _f64, attention_rows_f64, decode_f64
+from .attention import _f64, attention_rows_f64, attention_varlen_f64, decode_f64
 
-__all__ = ["gather_pages", "decode_paged_f64", "attention_paged_rows_f64"]
+__all__ = ["gather_pages", "decode_paged_f64", "attention_paged_rows_f64",
+           "attention_paged_varlen_f64"]
 
 
 def gather_pages(pool, table_row, n_tokens: int, page_size: int) -> np.ndarray:
@@ -75,3 +76,25 @@ def attention_paged_rows_f64(q, kpool, vpool, block_table, Nk: int, page_size: i
     V = gather_pages(vpool, table[b], Nk, page_size)[None]
     Q = _f64(q[b])[None]
     return attention_rows_f64(Q, K, V, causal, scale, 0, h, rows)
+
+
+def attention_paged_varlen_f64(q, kpool, vpool, block_table, q_lens, kv_lens, page_size: int,
+                               causal: bool, scale: float):
+    """Sequences of different lengths over a paged cache: sequence b's first kv_lens[b]
+    tokens are gathered through its table row, then `attention_varlen_f64` applies (its
+    first q_lens[b] query rows, mask aligned to its own end). Returns O [B,Hq,Nq,d] and LSE
+    [B,Hq,Nq], NaN past q_lens[b]."""
+    B, Hq, Nq, d = q.shape
+    Hkv = kpool.shape[1]
+    table = np.asarray(_f64(block_table), dtype=np.int64)
+    qn = np.asarray(_f64(q_lens), dtype=np.int64)
+    kn = np.asarray(_f64(kv_lens), dtype=np.int64)
+    O = np.full((B, Hq, Nq, d), np.nan, dtype=np.float64)
+    L = np.full((B, Hq, Nq), np.nan, dtype=np.float64)
+    for b in range(B):
+        nk = int(kn[b])
+        K = gather_pages(kpool, table[b], nk, page_size)[None] if nk > 0 else np.zeros((1, Hkv, 0, d))
+        V = gather_pages(vpool, table[b], nk, page_size)[None] if nk > 0 else np.zeros((1, Hkv, 0, d))
+        O[b:b + 1], L[b:b + 1] = attention_varlen_f64(_f64(q[b])[None], K, V, qn[b:b + 1],
+                                                      kn[b:b + 1], causal, scale)
+    return O, L

@@ -67,15 +67,17 @@ def test_fwd_kvcache_rejects_bad_arguments_without_cuda():
         a = dict(q=16, k=16, v=16, o=16, lse=None, B=1, Hq=2, Hkv=1, Nq=64, d=64, causal=1,
                  scale=0.125, dtype=0)
         a.update(kw)
-        return L.fa_fwd_kvcache(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"],
-                                a["Hkv"], a["Nq"], Nk, cache_len, a["d"], a["causal"], a["scale"],
-                                a["dtype"], None)
+        return L.fa_fwd_kvcache(a["q"], a["k"], a["v"], a.get("q_lens"), a.get("kv_lens"), a["o"],
+                                a["lse"], a["B"], a["Hq"], a["Hkv"], a["Nq"], Nk, cache_len, a["d"],
+                                a["causal"], a["scale"], a["dtype"], None)
     assert call(Nk=257, cache_len=256) == fa.FA_ERR_INVALID_ARG    # prefix longer than the cache
     assert call(cache_len=0) == fa.FA_ERR_INVALID_ARG
     assert call(Nk=0) == fa.FA_ERR_INVALID_ARG
     assert call(q=None) == fa.FA_ERR_INVALID_ARG
     assert call(d=96) == fa.FA_ERR_UNSUPPORTED
     assert call(k=24) == fa.FA_ERR_ALIGNMENT
+    assert call(q_lens=18) == fa.FA_ERR_ALIGNMENT        # per-sequence lengths: 4-byte aligned
+    assert call(kv_lens=34) == fa.FA_ERR_ALIGNMENT
 
 
 def test_bwd_rejects_bad_arguments_without_cuda():
@@ -138,8 +140,8 @@ def test_paged_entry_points_reject_bad_arguments_without_cuda():
 
     def fwd(q=16, kp=16, vp=16, table=16, o=16, Nq=64, Nk=300, num_pages=40, page_size=32,
             max_pages=10, d=64):
-        return L.fa_fwd_paged(q, kp, vp, table, o, None, 1, 2, 1, Nq, Nk, num_pages, page_size,
-                              max_pages, d, 1, 0.125, 0, None)
+        return L.fa_fwd_paged(q, kp, vp, table, None, None, o, None, 1, 2, 1, Nq, Nk, num_pages,
+                              page_size, max_pages, d, 1, 0.125, 0, None)
     for call in (dec, fwd):
         assert call(table=None) == fa.FA_ERR_INVALID_ARG
         assert call(num_pages=0) == fa.FA_ERR_INVALID_ARG

@@ -336,3 +336,27 @@ def test_every_entry_point_receives_its_declared_argument_count(monkeypatch):
     assert seen["fa_fwd"][2][5:11] == (2, 4, 2, 96, 80, 64)
     assert seen["fa_decode"][2][6:11] == (3, 8, 2, 512, 128)
     assert seen["fa_decode_paged"][2][7:13] == (3, 8, 2, 64, 16, 32)
+    assert seen["fa_fwd_kvcache"][2][3:5] == (None, None)
+    assert seen["fa_fwd_kvcache"][2][7:13] == (2, 4, 2, 96, 80, 80)
+    assert seen["fa_fwd_paged"][2][4:6] == (None, None)
+    assert seen["fa_fwd_paged"][2][8:16] == (2, 4, 2, 96, 100, 40, 16, 8)
+    # per-sequence lengths ride in their own slots
+    ql, kl = V((2,), torch.int32), V((2,), torch.int32)
+    fa.fwd_kvcache(q4, k4, k4, 80, out=V((2, 4, 96, 64)), lse=V((2, 4, 96), F32), q_lens=ql,
+                   kv_lens=kl)
+    assert all(isinstance(x, int) for x in seen["fa_fwd_kvcache"][2][3:5])
+    assert seen["fa_fwd_kvcache"][0] == seen["fa_fwd_kvcache"][1]
+
+
+def test_per_sequence_lengths_are_checked():
+    q4, k4 = FakeCuda((2, 4, 96, 64)), FakeCuda((2, 2, 80, 64))
+    for bad, err in ((FakeCuda((3,), torch.int32), TypeError),          # one per sequence
+                     (FakeCuda((2,), torch.int64), TypeError),          # int32 only
+                     (FakeCuda((2,), torch.int32, index=1), ValueError)):
+        with pytest.raises(err):
+            fa.fwd_kvcache(q4, k4, k4, 80, q_lens=bad, out=FakeCuda((2, 4, 96, 64)),
+                           lse=FakeCuda((2, 4, 96), F32))
+        with pytest.raises(err):
+            fa.fwd_paged(q4, FakeCuda((40, 2, 16, 64)), FakeCuda((40, 2, 16, 64)),
+                         FakeCuda((2, 8), torch.int32), 100, kv_lens=bad,
+                         out=FakeCuda((2, 4, 96, 64)), lse=FakeCuda((2, 4, 96), F32))
