@@ -54,10 +54,6 @@ struct EmptyBase {};
 #ifndef FA_D64_BN
 #define FA_D64_BN 64
 #endif
-// d = 128: load S in 32-column chunks with the next chunk in flight (1) or in one load (0).
-#ifndef FA_D128_PIPE
-#define FA_D128_PIPE 0
-#endif
 #ifndef FA_REGSPLIT
 #define FA_REGSPLIT 1
 #endif
@@ -773,25 +769,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           if (grow) m_used = mx;
           return __any_sync(0xffffffffu, grow);
         };
-#if FA_D128_PIPE
-        // Every row of the warp has a running max: P of each 32-column chunk against it,
-        // with the next chunk's TMEM load in flight meanwhile (P of chunk c goes to columns
-        // [16c, 16c+16), which hold scores already loaded, never ones still in flight).
-        if (kResident && __all_sync(0xffffffffu, m_used != -CUDART_INF_F)) {
-          tmem_ld32x32b_x32_async(tS, &sr[0]);
-          tmem_ld_wait_tied32(&sr[0]);
-          float lsum = 0.f;
-#pragma unroll
-          for (int cc = 0; cc < kBN / 32; ++cc) {
-            if (cc + 1 < kBN / 32) tmem_ld32x32b_x32_async(tS + 32 * (cc + 1), &sr[32 * (cc + 1)]);
-            mask_chunk(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * cc]), cc);
-            lsum += chunk_p(&sr[32 * cc], cc, m_used, true);
-            if (cc + 1 < kBN / 32) tmem_ld_wait_tied32(&sr[32 * (cc + 1)]);
-          }
-          if (raise_max()) lsum = p_pass(m_used, false);
-          l += lsum;
-        } else
-#endif
         if constexpr (kResident) {
           tmem_ld32x32b_x128(tS, sr);
 #pragma unroll
