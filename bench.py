@@ -108,7 +108,9 @@ def make_l2_flush(dev):
     read, the lines in L2 are clean and unrelated to the workload."""
     import torch
     wbuf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    rbuf = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    # float32, so that the sum reduces it in place (an integer sum would first widen the
+    # whole buffer to int64, a 512 MiB write that leaves dirty lines behind).
+    rbuf = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     def flush():
         wbuf.zero_()
