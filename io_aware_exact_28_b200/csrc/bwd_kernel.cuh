@@ -7,14 +7,15 @@
 // D_i = sum_d dO_id O_id:
 //     dV = P^T dO      dP = dO V^T      dS = P * (dP - D)
 //     dQ = scale * dS K                  dK = scale * dS^T Q
-// Three kernels:
+// Two kernels: fa_bwd_preprocess_kernel, then fa_bwd_fused_kernel, whose grid holds the
+// CTAs of both gradient passes (independent of each other):
 //   fa_bwd_preprocess_kernel  D and L * log2(e) per query row, padded to whole 128-row
 //                             tiles; rows without a visible key and rows past Nq get
-//                             +inf, so their P is exactly 0 in both kernels below.
-//   fa_bwd_dq_kernel          one CTA per 128-row query tile: per key tile j,
+//                             +inf, so their P is exactly 0 in both passes below.
+//   dQ pass (bwd_dq_tile)     one CTA per 128-row query tile: per key tile j,
 //                             S = Q K_j^T and dP = dO V_j^T (tcgen05, TMEM), then the
 //                             elementwise warps form dS and dQ += dS K_j (A = dS in TMEM).
-//   fa_bwd_dkdv_kernel        one CTA per 128-row key tile of a KV head: per query tile i
+//   dK/dV pass (bwd_dkdv_tile) one CTA per 128-row key tile of a KV head: per query tile i
 //                             of every query head of its group, S^T = K Q_i^T and
 //                             dP^T = V dO_i^T, then P^T and dS^T, and dV += P^T dO_i,
 //                             dK += dS^T Q_i (A operands in TMEM). The group's query heads
@@ -136,21 +137,19 @@ struct BwdCfg {
 // dQ: CTA (query tile qt, head bh), key tiles of TN rows. TMEM: S [0,TN) (dS packed
 // over its first TN/2 columns), dP [TN,2TN), dQ [2TN, 2TN+D).
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(BwdCfg<D>::THREADS, BwdCfg<D>::CTAS)
-fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                 const BwdParams p) {
+__device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                            const CUtensorMap& tmV, const CUtensorMap& tmDO,
+                                            const BwdParams& p, const int tile, const int bh) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
   const int b = bh / p.Hq, h = bh - b * p.Hq;
   const int bh_kv = b * p.Hkv + h / p.group;
   constexpr int TN = C::TN;
-  const int q0 = blockIdx.x * kBwdTile;
+  const int q0 = tile * kBwdTile;
   const int n_kv_total = (p.Nk + TN - 1) / TN;
   int n_kv = n_kv_total;
   if (CAUSAL) {
@@ -349,20 +348,18 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // first TN/2 columns), dP^T [TN,2TN) (dS^T packed over its first TN/2), dV [2TN, 2TN+D),
 // dK [2TN+D, 2TN+2D).
 template <int D, bool BF16, bool CAUSAL>
-__global__ void __launch_bounds__(BwdCfg<D>::THREADS, BwdCfg<D>::CTAS)
-fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                   const BwdParams p) {
+__device__ __forceinline__ void bwd_dkdv_tile(const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                              const CUtensorMap& tmV, const CUtensorMap& tmDO,
+                                              const BwdParams& p, const int tile, const int bh_kv) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh_kv = blockIdx.y;
   const int b = bh_kv / p.Hkv, hk = bh_kv - b * p.Hkv;
   constexpr int TN = C::TN;
-  const int k0 = blockIdx.x * kBwdTile;
+  const int k0 = tile * kBwdTile;
   const int n_q = (p.Nq + TN - 1) / TN;
   // Query tiles that see any key of this tile: queries i with k0 <= i + offset.
   int q_first = 0;
@@ -578,6 +575,30 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   if (warp == C::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Both gradient passes in one grid: the dK/dV CTAs first, then the dQ CTAs, each set
+// heaviest causal tile first (key tile 0 sees the most queries; the last query tile the
+// most keys), so that dQ work fills the SMs the last dK/dV wave leaves idle. The two
+// passes are independent: both read only Q, K, V, dO and the preprocessed L and D.
+template <int D, bool BF16, bool CAUSAL>
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, BwdCfg<D>::CTAS)
+fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKs,
+                    const __grid_constant__ CUtensorMap tmVs, const __grid_constant__ CUtensorMap tmDO,
+                    const __grid_constant__ CUtensorMap tmQs, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDOs,
+                    const BwdParams pq, const BwdParams pk, const int n_k, const int n_q,
+                    const int BHkv, const int BH) {
+  const int bid = blockIdx.x;
+  const int n_kv_blocks = n_k * BHkv;
+  if (bid < n_kv_blocks) {
+    const int kt = bid / BHkv;
+    bwd_dkdv_tile<D, BF16, CAUSAL>(tmQs, tmK, tmV, tmDOs, pk, kt, bid - kt * BHkv);
+  } else {
+    const int c = bid - n_kv_blocks;
+    const int r = c / BH;
+    bwd_dq_tile<D, BF16, CAUSAL>(tmQ, tmKs, tmVs, tmDO, pq, n_q - 1 - r, c - r * BH);
   }
 }
 

@@ -167,7 +167,8 @@ __device__ __forceinline__ void rescale_p_cols(uint32_t taddr, float alpha) {
   tmem_st_wait();
 }
 
-template <int D, bool BF16, bool CAUSAL, bool PAGED, bool FP8 = false, bool VARLEN = false>
+template <int D, bool BF16, bool CAUSAL, bool PAGED, bool FP8 = false, bool VARLEN = false,
+          bool KVMAJOR = false>
 __global__ void __launch_bounds__(FwdCfg<D, FP8>::THREADS, FwdCfg<D, FP8>::CTAS)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
@@ -212,9 +213,25 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   };
   auto decode_unit = [&](int u) {
     Unit w;
-    const int qb = p.n_qb - 1 - u / p.BH;
-    w.bh = u - (u / p.BH) * p.BH;
-    w.bh_kv = (w.bh / p.Hq) * p.Hkv + (w.bh % p.Hq) / p.group;
+    // KVMAJOR (grouped-query calls whose K/V would not stay in L2): the units of one KV
+    // head (every query block, heaviest first, of each query head that reads it) are
+    // numbered together, so that the CTAs running at any time stream one or two KV heads
+    // and each K/V tile is read from DRAM about once. Otherwise query block by query
+    // block, heaviest first, all heads of a block together.
+    int qb;
+    if constexpr (KVMAJOR) {
+      const int per_kv = p.n_qb * p.group;
+      const int kv = u / per_kv;
+      const int r = u - kv * per_kv;
+      qb = p.n_qb - 1 - r / p.group;
+      const int g = r - (r / p.group) * p.group;
+      w.bh_kv = kv;
+      w.bh = (kv / p.Hkv) * p.Hq + (kv - (kv / p.Hkv) * p.Hkv) * p.group + g;
+    } else {
+      qb = p.n_qb - 1 - u / p.BH;
+      w.bh = u - (u / p.BH) * p.BH;
+      w.bh_kv = (w.bh / p.Hq) * p.Hkv + (w.bh % p.Hq) / p.group;
+    }
     w.q0 = qb * (C::QT * kBM);
     w.n_kv = 0;
     if constexpr (VARLEN) {

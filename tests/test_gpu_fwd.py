@@ -311,3 +311,17 @@ def test_more_units_than_resident_ctas(B, Hq, Hkv, Nq, Nk, d, dtype, causal):
     for (b, h) in [(0, 0), (B - 1, Hq - 1)]:
         O, L = attention_rows_f64(q, k, v, causal, scale, b, h, rows)
         assert_close(o[b, h, rows], lse[b, h, rows], O, L, dtype, f"takeover b{b} h{h}", strict=False)
+
+
+def test_kv_head_major_order_with_several_sequences():
+    """Grouped-query calls whose K and V exceed half of L2 number their work units KV
+    head by KV head (B=4, Hq=8, Hkv=4, N=8192, d=128: 67 MB of K/V); seeded rows of heads
+    spread over every sequence and KV group against the oracle."""
+    B, Hq, Hkv, N, d = 4, 8, 4, 8192, 128
+    q, k, v = make_fwd_inputs(B, Hq, Hkv, N, N, d, "bf16", seed=61)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_fwd(q, k, v, True, scale)
+    rows = sample_rows(N, 24, seed=61)
+    for b, h in ((0, 0), (0, 7), (1, 3), (2, 4), (3, 0), (3, 7)):
+        O, L = attention_rows_f64(q, k, v, True, scale, b, h, rows)
+        assert_close(o[b, h, rows], lse[b, h, rows], O, L, "bf16", f"kv-major b{b} h{h}", strict=False)

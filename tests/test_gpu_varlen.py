@@ -221,3 +221,31 @@ def test_many_units_with_empty_sequences_interleaved():
                 O, L = attention_rows_f64(q[b:b + 1], kc[b:b + 1], vc[b:b + 1], True, 0.125, 0, h, rows)
                 assert_close(o[b, h, rows], lse[b, h, rows], O, L, "fp16", f"interleaved b{b} h{h}",
                              strict=False)
+
+
+def test_ragged_grouped_query_batch_of_four_sequences():
+    """Per-sequence lengths in a grouped-query batch with 67 MB of K/V capacity (B=4,
+    Hq=8, Hkv=4, cache 8192): a full sequence, a short one, one without keys and a chunk
+    after a long prefix."""
+    B, Hq, Hkv, cap, d = 4, 8, 4, 8192, 128
+    kl, ql = [8192, 100, 0, 5000], [8192, 100, 7, 1000]
+    q, kc, vc = poisoned_inputs(B, Hq, Hkv, cap, cap, d, "bf16", ql, kl, seed=71)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = outputs(q)
+    fa.fwd_kvcache(q.to(DEV), kc.to(DEV), vc.to(DEV), cap, causal=True, scale=scale, out=o, lse=lse,
+                   q_lens=torch.tensor(ql, dtype=torch.int32, device=DEV),
+                   kv_lens=torch.tensor(kl, dtype=torch.int32, device=DEV))
+    torch.cuda.synchronize()
+    assert fa.device_status() == fa.FA_OK
+    o, lse = o.cpu(), lse.cpu()
+    for b in range(B):
+        assert torch.all(o[b, :, ql[b]:] == O_FILL) and torch.all(lse[b, :, ql[b]:] == L_FILL)
+        if kl[b] == 0:
+            assert torch.all(o[b, :, :ql[b]] == 0) and torch.all(torch.isneginf(lse[b, :, :ql[b]]))
+            continue
+        rows = sample_rows(ql[b], 16, seed=b)
+        qb, kb, vb = q[b:b + 1, :, :ql[b]], kc[b:b + 1, :, :kl[b]], vc[b:b + 1, :, :kl[b]]
+        for h in (0, Hq - 1):
+            O, L = attention_rows_f64(qb, kb, vb, True, scale, 0, h, rows)
+            assert_close(o[b, h, rows], lse[b, h, rows], O, L, "bf16", f"ragged gqa b{b} h{h}",
+                         strict=False)
