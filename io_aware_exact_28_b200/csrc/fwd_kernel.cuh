@@ -57,6 +57,13 @@ struct EmptyBase {};
 #ifndef FA_REGSPLIT
 #define FA_REGSPLIT 1
 #endif
+// 64-key tiles: exponential pairs, of the 16 in each 32-score chunk, evaluated on the FMA
+// pipe (exp2_emu) instead of the MUFU unit (0, 1, 2 or 4). A 64-key tile's softmax needs
+// twice the MUFU time of its two products; 128-key tiles (16-bit or E4M3) are faster with
+// every exponential on the MUFU unit.
+#ifndef FA_EXP2_EMU_D64
+#define FA_EXP2_EMU_D64 2
+#endif
 
 // Per head-dimension configuration.
 //  d = 128: 128-key tiles, one CTA per SM, TMEM S 2x128 + O 2x128 = 512 columns.
@@ -81,6 +88,13 @@ struct FwdCfg {
   static constexpr int WARP_PRODUCER = 4 * QT;        // TMA producer warp
   static constexpr int WARP_MMA = 4 * QT + 1;         // TMEM allocator and MMA issuer
   static constexpr bool REGSPLIT = !NARROW && FA_REGSPLIT;
+  // Pairs i (0-15) of a 32-score chunk whose 2^x comes from exp2_emu.
+  static constexpr int EMU_PAIRS = NARROW ? FA_EXP2_EMU_D64 : 0;
+  static_assert(EMU_PAIRS == 0 || EMU_PAIRS == 1 || EMU_PAIRS == 2 || EMU_PAIRS == 4,
+                "exp2 emulation: 0, 1, 2 or 4 pairs of 16");
+  static constexpr uint32_t EMU_MASK = EMU_PAIRS == 1 ? 0x0008u
+                                       : EMU_PAIRS == 2 ? 0x0808u
+                                       : EMU_PAIRS == 4 ? 0x8888u : 0u;
   static constexpr int NCH = ROWB / 128;              // 128-byte swizzle chunks along d
   static constexpr int OCH = D / 64;                  // 64-column chunks of an O row
   static constexpr int Q_CHUNK = kBM * 128;           // 128 rows x 128 bytes
@@ -691,6 +705,14 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         // P of one 32-column chunk v (scores of keys 32 cc ..) against mref, stored as 16
         // packed columns at tS + 16 cc; returns its row sum (unrounded fp32 P). With track,
         // the scores' maximum is gathered in mx8 on the way.
+        // 2^x of pair i of a chunk: MUFU ex2, or exp2_emu for the pairs EMU_MASK names (i is
+        // a compile-time index once the loops are unrolled).
+        auto exp2_pair = [&](uint64_t x2, int i) -> uint64_t {
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          if ((C::EMU_MASK >> i) & 1u) return f2_pack(exp2_emu(x0), exp2_emu(x1));
+          return f2_pack(ex2_approx(x0), ex2_approx(x1));
+        };
         auto chunk_p = [&](const uint32_t* v, int cc, float mref, bool track) -> float {
           const float nm = FP8 ? C::OFF - mref : -mref;
           const uint64_t nm2 = f2_pack(nm, nm);
@@ -705,9 +727,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 mx8[i & 7] = fmax3(mx8[i & 7], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
               const uint64_t x2 =
                   f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2);
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              const uint64_t p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+              const uint64_t p2 = exp2_pair(x2, i);
               if (i & 1) l2b = f2_add(l2b, p2); else l2a = f2_add(l2a, p2);
               float p0, p1;
               f2_unpack(p2, p0, p1);
@@ -730,9 +750,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 mx8[i & 7] = fmax3(mx8[i & 7], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
               const uint64_t x2 =
                   f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), c2, nm2);
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              const uint64_t p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+              const uint64_t p2 = exp2_pair(x2, i);
               if (i & 1) l2b = f2_add(l2b, p2); else l2a = f2_add(l2a, p2);
               float p0, p1;
               f2_unpack(p2, p0, p1);

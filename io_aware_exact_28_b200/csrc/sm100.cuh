@@ -97,6 +97,33 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
   return r;
 }
 
+// 2^x on the FMA and integer pipes instead of the MUFU unit (Cody-Waite style range
+// reduction plus a polynomial), for kernels whose softmax has more exponentials than the
+// MUFU unit keeps up with. x is clamped to >= -127 and split as x = j + f with
+// j = round-to-nearest(x) through the 1.5 * 2^23 shifter (exact for |x| < 2^22);
+// p(f) = 1 + f (c1 + f (c2 + f (c3 + f c4))) ~ 2^f on |f| <= 1/2, and j is added to p's
+// exponent field. Coefficients: minimax relative-error fit by fit_exp2_poly.py (fp32 Horner
+// error 2.9e-6). p(0) = 1 exactly, so x <= -127 (a masked key's -inf included) gives +0;
+// x in (-127, -126.5) gives a positive denormal. x must stay below 128 (callers keep
+// x <= 12). The constants are instruction operands, so the function holds no registers
+// beyond its temporaries.
+constexpr float kExp2C1 = 0x1.62e12cp-1f;   // 0.693124175
+constexpr float kExp2C2 = 0x1.ec0378p-3f;   // 0.240240991
+constexpr float kExp2C3 = 0x1.c9fc46p-5f;   // 0.0559064262
+constexpr float kExp2C4 = 0x1.3a02ccp-7f;   // 0.00958285294
+
+__device__ __forceinline__ float exp2_emu(float x) {
+  const float xc = fmaxf(x, -127.f);
+  const float t = __fadd_rn(xc, 12582912.f);                   // bits: bits(shifter) + j
+  const float f = __fsub_rn(xc, __fsub_rn(t, 12582912.f));     // x - j, exact
+  float p = __fmaf_rn(kExp2C4, f, kExp2C3);
+  p = __fmaf_rn(p, f, kExp2C2);
+  p = __fmaf_rn(p, f, kExp2C1);
+  p = __fmaf_rn(p, f, 1.f);
+  // (bits(t) << 23) keeps exactly j << 23 (mod 2^32): bits(shifter) << 23 vanishes.
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
 // Cluster launch control (sm_100): ask the hardware scheduler for the work of a CTA of
 // this grid that has not started yet. The 16-byte response lands in shared memory and
 // completes 16 transaction bytes on the mbarrier; a CTA taken this way never launches.
