@@ -273,6 +273,7 @@ __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtens
     const int lim = CAUSAL ? min(row + p.causal_offset, p.Nk - 1) : p.Nk - 1;
     const int lim_min = CAUSAL ? min(q0 + p.causal_offset, p.Nk - 1) : p.Nk - 1;
     const float c = p.scale_log2;
+    const uint64_t c2 = f2_pack(c, c), nl2 = f2_pack(-lse2, -lse2), dsum2 = f2_pack(dsum, dsum);
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(bar_s, j & 1, wc))) { ok = false; break; }
@@ -287,15 +288,21 @@ __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtens
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float d2[2];
+          // Pair (2i, 2i+1) in packed fp32: P = 2^(s*c - L), dS = P (dP - D).
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])),
+                                     c2, nl2);
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          float pv[2] = {ex2_approx(x0), ex2_approx(x1)};
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int kk = 2 * i + e;
-            float pv = ex2_approx(__uint_as_float(s[kk]) * c - lse2);
-            if (masked && key0 + 32 * cc + kk > lim) pv = 0.f;
-            d2[e] = pv * (__uint_as_float(dp[kk]) - dsum);
-          }
-          pk[i] = pack_half2(d2[0], d2[1], BF16);
+          for (int e = 0; e < 2; ++e)
+            if (masked && key0 + 32 * cc + 2 * i + e > lim) pv[e] = 0.f;
+          const uint64_t d2 = f2_mul(f2_pack(pv[0], pv[1]),
+                                     f2_sub(f2_pack(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])),
+                                            dsum2));
+          float d0, d1;
+          f2_unpack(d2, d0, d1);
+          pk[i] = pack_half2(d0, d1, BF16);
         }
         tmem_st32x32b_x16(tS + 16 * cc, pk);
       }
@@ -497,6 +504,7 @@ __device__ __forceinline__ void bwd_dkdv_tile(const CUtensorMap& tmQ, const CUte
     const uint32_t tS = tmem + lane_base + g * (TN / G), tP = tS + C::P_COL;
     const uint32_t tV = tmem + lane_base + C::ACC_COL, tK = tV + D;
     const float c = p.scale_log2;
+    const uint64_t c2 = f2_pack(c, c);
     bool ok = true;
     for (int s = 0; s < n_steps; ++s) {
       const int slot = s % NP;
@@ -517,19 +525,38 @@ __device__ __forceinline__ void bwd_dkdv_tile(const CUtensorMap& tmQ, const CUte
         tmem_ld32x32b_x32(tS + 32 * cc, st);
         tmem_ld32x32b_x32(tP + 32 * cc, dpt);
         uint32_t pk[16], dk[16];
+        // This chunk's 32 columns of L and D, read as 16-byte shared-memory loads (the same
+        // address in every lane: one broadcast each), four columns (two pairs) per load.
+        const float4* l4 = reinterpret_cast<const float4*>(lv + g * (TN / G) + 32 * cc);
+        const float4* d4 = reinterpret_cast<const float4*>(dv + g * (TN / G) + 32 * cc);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float pv[2], dsv[2];
+        for (int q = 0; q < 8; ++q) {
+          const float4 lq = l4[q], dq = d4[q];
+          const float lcol[4] = {lq.x, lq.y, lq.z, lq.w};
+          const float dcol[4] = {dq.x, dq.y, dq.z, dq.w};
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = g * (TN / G) + 32 * cc + 2 * i + e;
-            float x = ex2_approx(__uint_as_float(st[2 * i + e]) * c - lv[col]);
-            if (masked && col < first_vis) x = 0.f;
-            pv[e] = x;
-            dsv[e] = x * (__uint_as_float(dpt[2 * i + e]) - dv[col]);
+          for (int h = 0; h < 2; ++h) {
+            const int i = 2 * q + h;
+            // Pair (2i, 2i+1) in packed fp32: x = s*c - L, P = 2^x, dS = P (dP - D).
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(st[2 * i]), __uint_as_float(st[2 * i + 1])),
+                                       c2, f2_pack(-lcol[2 * h], -lcol[2 * h + 1]));
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            float pv[2] = {ex2_approx(x0), ex2_approx(x1)};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int col = g * (TN / G) + 32 * cc + 2 * i + e;
+              if (masked && col < first_vis) pv[e] = 0.f;
+            }
+            const uint64_t p2 = f2_pack(pv[0], pv[1]);
+            const uint64_t ds2 = f2_mul(p2, f2_sub(f2_pack(__uint_as_float(dpt[2 * i]),
+                                                           __uint_as_float(dpt[2 * i + 1])),
+                                                   f2_pack(dcol[2 * h], dcol[2 * h + 1])));
+            float ds0, ds1;
+            f2_unpack(ds2, ds0, ds1);
+            pk[i] = pack_half2(pv[0], pv[1], BF16);
+            dk[i] = pack_half2(ds0, ds1, BF16);
           }
-          pk[i] = pack_half2(pv[0], pv[1], BF16);
-          dk[i] = pack_half2(dsv[0], dsv[1], BF16);
         }
         tmem_st32x32b_x16(tS + 16 * cc, pk);
         tmem_st32x32b_x16(tP + 16 * cc, dk);
