@@ -32,6 +32,13 @@
 namespace fa {
 
 constexpr int kBwdTile = 128;          // query rows and key rows per tile
+
+// Packed fp32 product of two pairs (sm_100 mul.f32x2), beside f2_fma / f2_sub.
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
 // TMEM column of the 16-bit operand that one 16-element K step kk of a P.X product reads.
 // With G elementwise groups, group g owns the streamed columns [g*TN/G, (g+1)*TN/G) of S
 // and dP and packs its share of P (or dS) at the start of that range, so K step kk lies in
