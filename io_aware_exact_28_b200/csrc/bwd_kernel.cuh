@@ -136,13 +136,19 @@ struct BwdCfg {
   static constexpr uint32_t TMEM_COLS = (D == 64) ? 256 : 512;
   static constexpr uint32_t P_COL = TN;              // dP (dQ kernel) / dP^T (dK/dV kernel)
   static constexpr uint32_t ACC_COL = 2 * TN;        // dQ, or dV then dK
+  static constexpr uint32_t DP1_COL = ACC_COL + D;   // dQ kernel: dP of odd key tiles
   static_assert(SMEM_BYTES * CTAS <= 227 * 1024, "shared memory budget");
   static_assert(ACC_COL + 2 * D <= TMEM_COLS, "TMEM budget");
+  static_assert(DP1_COL + TN <= TMEM_COLS, "TMEM budget (second dP buffer)");
 };
 
 // ------------------------------------------------------------------------------------
 // dQ: CTA (query tile qt, head bh), key tiles of TN rows. TMEM: S [0,TN) (dS packed
-// over its first TN/2 columns), dP [TN,2TN), dQ [2TN, 2TN+D).
+// over its first TN/2 columns), dP of even key tiles [TN,2TN), dQ [2TN, 2TN+D), dP of odd
+// key tiles [2TN+D, 3TN+D). With two dP buffers the tensor core computes dP(j+1) while
+// the elementwise warps work on step j; then dQ += dS(j) K_j and S(j+1). The producer
+// loads V_j+1 ahead of K_j+1 (order K_0, V_0, V_1, K_1, V_2, K_2, ...), so that V_j+1's
+// ring slot, freed by dP(j-1), is filled well before it is needed.
 template <int D, bool BF16, bool CAUSAL>
 __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                             const CUtensorMap& tmV, const CUtensorMap& tmDO,
@@ -206,7 +212,8 @@ __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtens
       int it = 0;
       bool ok = true;
       for (int j = 0; j < n_kv && ok; ++j) {
-        for (int kv = 0; kv < 2; ++kv) {                // K_j, then V_j
+        for (int x = 0; x < 2; ++x) {                   // K_0, V_0; then V_j, K_j
+          const int kv = (j == 0) ? x : 1 - x;
           const int slot = it % C::NS, round = it / C::NS;
           if (round > 0 && !mbar_wait(bar_empty(slot), (round - 1) & 1, wc)) { ok = false; break; }
           mbar_arrive_expect_tx(bar_full(slot), C::STILE_BYTES);
@@ -240,26 +247,46 @@ __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtens
       bool issued = false;
       tc_fence_after();
       const uint32_t qa = base + C::A_OFF, doa = base + C::A_OFF + C::TILE_BYTES;
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int kit = 2 * j, kslot = kit % C::NS, vit = kit + 1, vslot = vit % C::NS;
-        if (!mbar_wait(bar_full(kslot), (kit / C::NS) & 1, wc)) { ok = false; break; }
-        if (!mbar_wait(bar_full(vslot), (vit / C::NS) & 1, wc)) { ok = false; break; }
+      // Ring items in load order: K_0 = 0, V_0 = 1, then V_j = 2j, K_j = 2j + 1.
+      auto k_item = [](int j) { return j == 0 ? 0 : 2 * j + 1; };
+      auto v_item = [](int j) { return j == 0 ? 1 : 2 * j; };
+      auto item_addr = [&](int it) { return base + C::RING_OFF + (it % C::NS) * C::STILE_BYTES; };
+      auto wait_item = [&](int it) { return mbar_wait(bar_full(it % C::NS), (it / C::NS) & 1, wc); };
+      auto dp_col = [](int j) { return (j & 1) ? C::DP1_COL : C::P_COL; };
+      // Step 0: S(0) and dP(0).
+      if (ok && wait_item(k_item(0)) && wait_item(v_item(0))) {
         tc_fence_after();
-        const uint32_t ka = base + C::RING_OFF + kslot * C::STILE_BYTES;
-        const uint32_t va = base + C::RING_OFF + vslot * C::STILE_BYTES;
-        issue_abt(0, qa, ka);                          // S = Q K_j^T
-        issue_abt(C::P_COL, doa, va);                  // dP = dO V_j^T
+        issue_abt(0, qa, item_addr(k_item(0)));                 // S = Q K_0^T
+        issue_abt(dp_col(0), doa, item_addr(v_item(0)));        // dP = dO V_0^T
         issued = true;
         mma_commit(bar_s);
-        mma_commit(bar_empty(vslot));                  // V_j no longer needed
+        mma_commit(bar_empty(v_item(0) % C::NS));               // V_0 no longer needed
+      } else {
+        ok = false;
+      }
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const bool next = j + 1 < n_kv;
+        if (next) {                                             // dP(j+1), beside step j
+          if (!wait_item(v_item(j + 1))) { ok = false; break; }
+          tc_fence_after();
+          issue_abt(dp_col(j + 1), doa, item_addr(v_item(j + 1)));
+          mma_commit(bar_empty(v_item(j + 1) % C::NS));
+        }
         if (!mbar_wait(bar_ds, j & 1, wc)) { ok = false; break; }
         tc_fence_after();
         // dQ += dS K_j: A = dS (packed 16-bit in TMEM, per elementwise group), B = K_j MN-major.
+        const uint32_t ka = item_addr(k_item(j));
 #pragma unroll
         for (int kk = 0; kk < TN / 16; ++kk)
           mma_f16_ts(tmem + C::ACC_COL, tmem + packed_col<TN, C::G>(kk),
                      sdesc_mn_sw128(ka + kk * 2048, C::SCHUNK), IDESC_Q, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar_empty(kslot));
+        mma_commit(bar_empty(k_item(j) % C::NS));
+        if (next) {                                             // S(j+1) over dS(j), after dQ
+          if (!wait_item(k_item(j + 1))) { ok = false; break; }
+          tc_fence_after();
+          issue_abt(0, qa, item_addr(k_item(j + 1)));
+          mma_commit(bar_s);                                    // step j+1: S and dP ready
+        }
       }
       if (issued) mma_commit(ok ? bar_done : bar_drain);
       if (issued && !ok) mbar_wait_drain(bar_drain, 0, kDrainNs);
@@ -273,7 +300,7 @@ __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtens
     const int r = (warp & 3) * 32 + lane;                   // query row of the tile
     const int row = q0 + r;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + g * (TN / G), tP = tS + C::P_COL;
+    const uint32_t tS = tmem + lane_base + g * (TN / G);
     const uint32_t tQ = tmem + lane_base + C::ACC_COL + g * (D / G);
     const float lse2 = p.lse2[static_cast<size_t>(bh) * p.Nq_pad + row];
     const float dsum = p.dsum[static_cast<size_t>(bh) * p.Nq_pad + row];
@@ -287,6 +314,7 @@ __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtens
       tc_fence_after();
       const int key0 = j * TN + g * (TN / G);                // first key of this group's columns
       const bool masked = key0 + TN / G - 1 > lim_min;       // warp-uniform per CTA
+      const uint32_t tP = tS + ((j & 1) ? C::DP1_COL : C::P_COL);   // this step's dP buffer
 #pragma unroll
       for (int cc = 0; cc < TN / (32 * G); ++cc) {
         uint32_t s[32], dp[32];
