@@ -143,12 +143,14 @@ struct BwdCfg {
 };
 
 // ------------------------------------------------------------------------------------
-// dQ: CTA (query tile qt, head bh), key tiles of TN rows. TMEM: S [0,TN) (dS packed
-// over its first TN/2 columns), dP of even key tiles [TN,2TN), dQ [2TN, 2TN+D), dP of odd
-// key tiles [2TN+D, 3TN+D). With two dP buffers the tensor core computes dP(j+1) while
-// the elementwise warps work on step j; then dQ += dS(j) K_j and S(j+1). The producer
-// loads V_j+1 ahead of K_j+1 (order K_0, V_0, V_1, K_1, V_2, K_2, ...), so that V_j+1's
-// ring slot, freed by dP(j-1), is filled well before it is needed.
+// dQ: CTA (query tile qt, head bh), key tiles of TN rows. TMEM: S [0,TN), dP of even key
+// tiles [TN,2TN), dQ [2TN, 2TN+D), dP of odd key tiles [2TN+D, 3TN+D); dS(j) is packed
+// over the first TN/2 columns of its step's dP buffer. Once step j's elementwise work is
+// done the tensor core computes S(j+1), which is all step j+1 waits for (its dP was
+// computed earlier), then dQ += dS(j) K_j and dP(j+2) into the buffer dS(j) leaves, both
+// beside step j+1's elementwise work. The producer loads V ahead of K (order K_0, V_0,
+// V_1, K_1, V_2, K_2, ...), so that each V tile's ring slot, freed by the dP two steps
+// back, is filled before it is needed.
 template <int D, bool BF16, bool CAUSAL>
 __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                             const CUtensorMap& tmV, const CUtensorMap& tmDO,
@@ -253,7 +255,7 @@ __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtens
       auto item_addr = [&](int it) { return base + C::RING_OFF + (it % C::NS) * C::STILE_BYTES; };
       auto wait_item = [&](int it) { return mbar_wait(bar_full(it % C::NS), (it / C::NS) & 1, wc); };
       auto dp_col = [](int j) { return (j & 1) ? C::DP1_COL : C::P_COL; };
-      // Step 0: S(0) and dP(0).
+      // Steps 0 and 1: S(0), dP(0), then dP(1) into the other buffer.
       if (ok && wait_item(k_item(0)) && wait_item(v_item(0))) {
         tc_fence_after();
         issue_abt(0, qa, item_addr(k_item(0)));                 // S = Q K_0^T
@@ -261,31 +263,40 @@ __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtens
         issued = true;
         mma_commit(bar_s);
         mma_commit(bar_empty(v_item(0) % C::NS));               // V_0 no longer needed
+        if (n_kv > 1) {
+          if (wait_item(v_item(1))) {
+            tc_fence_after();
+            issue_abt(dp_col(1), doa, item_addr(v_item(1)));
+            mma_commit(bar_empty(v_item(1) % C::NS));
+          } else {
+            ok = false;
+          }
+        }
       } else {
         ok = false;
       }
       for (int j = 0; j < n_kv && ok; ++j) {
-        const bool next = j + 1 < n_kv;
-        if (next) {                                             // dP(j+1), beside step j
-          if (!wait_item(v_item(j + 1))) { ok = false; break; }
-          tc_fence_after();
-          issue_abt(dp_col(j + 1), doa, item_addr(v_item(j + 1)));
-          mma_commit(bar_empty(v_item(j + 1) % C::NS));
-        }
+        // Step j's elementwise work done: S is free, dS(j) is packed over dP buffer j & 1.
         if (!mbar_wait(bar_ds, j & 1, wc)) { ok = false; break; }
         tc_fence_after();
+        if (j + 1 < n_kv) {                                     // S(j+1): step j+1 ready
+          if (!wait_item(k_item(j + 1))) { ok = false; break; }
+          tc_fence_after();
+          issue_abt(0, qa, item_addr(k_item(j + 1)));
+          mma_commit(bar_s);
+        }
         // dQ += dS K_j: A = dS (packed 16-bit in TMEM, per elementwise group), B = K_j MN-major.
         const uint32_t ka = item_addr(k_item(j));
 #pragma unroll
         for (int kk = 0; kk < TN / 16; ++kk)
-          mma_f16_ts(tmem + C::ACC_COL, tmem + packed_col<TN, C::G>(kk),
+          mma_f16_ts(tmem + C::ACC_COL, tmem + dp_col(j) + packed_col<TN, C::G>(kk),
                      sdesc_mn_sw128(ka + kk * 2048, C::SCHUNK), IDESC_Q, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar_empty(k_item(j) % C::NS));
-        if (next) {                                             // S(j+1) over dS(j), after dQ
-          if (!wait_item(k_item(j + 1))) { ok = false; break; }
+        if (j + 2 < n_kv) {                                     // dP(j+2), after dQ(j) read dS(j)
+          if (!wait_item(v_item(j + 2))) { ok = false; break; }
           tc_fence_after();
-          issue_abt(0, qa, item_addr(k_item(j + 1)));
-          mma_commit(bar_s);                                    // step j+1: S and dP ready
+          issue_abt(dp_col(j + 2), doa, item_addr(v_item(j + 2)));
+          mma_commit(bar_empty(v_item(j + 2) % C::NS));
         }
       }
       if (issued) mma_commit(ok ? bar_done : bar_drain);
@@ -339,7 +350,7 @@ __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtens
           f2_unpack(d2, d0, d1);
           pk[i] = pack_half2(d0, d1, BF16);
         }
-        tmem_st32x32b_x16(tS + 16 * cc, pk);
+        tmem_st32x32b_x16(tP + 16 * cc, pk);
       }
       tmem_st_wait();
       tc_fence_before();
