@@ -130,7 +130,7 @@ struct BwdCfg {
   static constexpr int RING_OFF = 2 * TILE_BYTES;
   static constexpr int VEC_OFF = RING_OFF + NS * STILE_BYTES;  // dK/dV: L and D per ring pair
   static constexpr int BAR_OFF = VEC_OFF + (NS / 2) * 2 * TN * 4;
-  static constexpr int NBARS = 1 + 2 * NS + 4;
+  static constexpr int NBARS = 1 + 2 * NS + 6;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = (D == 64) ? 256 : 512;
@@ -432,10 +432,12 @@ __device__ __forceinline__ void bwd_dkdv_tile(const CUtensorMap& tmQ, const CUte
   const uint32_t bar_a = bar0;                                       // K and V landed
   auto bar_full = [&](int i) { return bar0 + 8u * (1 + i); };        // pair slot i (Q, dO, vecs)
   auto bar_empty = [&](int i) { return bar0 + 8u * (1 + C::NS + i); };
-  const uint32_t bar_s = bar0 + 8u * (1 + 2 * C::NS);                // S^T and dP^T ready
-  const uint32_t bar_ps = bar0 + 8u * (2 + 2 * C::NS);               // P^T, dS^T in TMEM (128 rows)
+  const uint32_t bar_s = bar0 + 8u * (1 + 2 * C::NS);                // S^T ready
+  const uint32_t bar_ps = bar0 + 8u * (2 + 2 * C::NS);               // dS^T in TMEM (128 rows)
   const uint32_t bar_done = bar0 + 8u * (3 + 2 * C::NS);
   const uint32_t bar_drain = bar0 + 8u * (4 + 2 * C::NS);
+  const uint32_t bar_pp = bar0 + 8u * (5 + 2 * C::NS);               // P^T in TMEM (128 rows)
+  const uint32_t bar_dp = bar0 + 8u * (6 + 2 * C::NS);               // dP^T ready
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + C::MISC_OFF + 4);
   constexpr int NP = C::NS / 2;                                      // ring pairs
@@ -448,6 +450,8 @@ __device__ __forceinline__ void bwd_dkdv_tile(const CUtensorMap& tmQ, const CUte
     }
     mbar_init(bar_s, 1);
     mbar_init(bar_ps, C::EW_THREADS);
+    mbar_init(bar_pp, C::EW_THREADS);
+    mbar_init(bar_dp, 1);
     mbar_init(bar_done, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -520,19 +524,39 @@ __device__ __forceinline__ void bwd_dkdv_tile(const CUtensorMap& tmQ, const CUte
       bool issued = false;
       tc_fence_after();
       const uint32_t ka = base + C::A_OFF, va = base + C::A_OFF + C::TILE_BYTES;
-      for (int s = 0; s < n_steps && ok; ++s) {
-        const int slot = s % NP;
-        if (!mbar_wait(bar_full(slot), (s / NP) & 1, wc)) { ok = false; break; }
+      // Order: S^T(0), dP^T(0); then per step s: dV(s) once P^T(s) is written, S^T(s+1)
+      // over it; dK(s) once dS^T(s) is written, dP^T(s+1) over it. The elementwise warps'
+      // P^T pass of step s+1 then runs beside dK(s) and dP^T(s+1).
+      if (ok && mbar_wait(bar_full(0), 0, wc)) {
         tc_fence_after();
-        issue_abt(0, ka, q_tile(slot));                 // S^T = K Q_i^T
-        issue_abt(C::P_COL, va, do_tile(slot));         // dP^T = V dO_i^T
+        issue_abt(0, ka, q_tile(0));                    // S^T = K Q_0^T
         issued = true;
         mma_commit(bar_s);
-        if (!mbar_wait(bar_ps, s & 1, wc)) { ok = false; break; }
+        issue_abt(C::P_COL, va, do_tile(0));            // dP^T = V dO_0^T
+        mma_commit(bar_dp);
+      } else {
+        ok = false;
+      }
+      for (int s = 0; s < n_steps && ok; ++s) {
+        const int slot = s % NP, nslot = (s + 1) % NP;
+        const bool next = s + 1 < n_steps;
+        if (!mbar_wait(bar_pp, s & 1, wc)) { ok = false; break; }
         tc_fence_after();
         issue_tb(C::ACC_COL, 0, do_tile(slot), s > 0);          // dV += P^T dO_i
+        if (next) {
+          if (!mbar_wait(bar_full(nslot), ((s + 1) / NP) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          issue_abt(0, ka, q_tile(nslot));                      // S^T(s+1), after dV(s)
+          mma_commit(bar_s);
+        }
+        if (!mbar_wait(bar_ps, s & 1, wc)) { ok = false; break; }
+        tc_fence_after();
         issue_tb(C::ACC_COL + D, C::P_COL, q_tile(slot), s > 0);  // dK += dS^T Q_i
         mma_commit(bar_empty(slot));
+        if (next) {
+          issue_abt(C::P_COL, va, do_tile(nslot));              // dP^T(s+1), after dK(s)
+          mma_commit(bar_dp);
+        }
       }
       if (issued) mma_commit(ok ? bar_done : bar_drain);
       if (issued && !ok) mbar_wait_drain(bar_drain, 0, kDrainNs);
@@ -565,46 +589,70 @@ __device__ __forceinline__ void bwd_dkdv_tile(const CUtensorMap& tmQ, const CUte
       // Key `key` is visible to query q0 + col iff key <= q0 + col + offset.
       const int first_vis = key - p.causal_offset - q0;     // smallest visible column
       const bool masked = CAUSAL && __any_sync(0xffffffffu, first_vis > 0);
+      // Pass 1: P^T = 2^(S^T c - L) for this group's TN/G columns, kept in fp32 for pass 2
+      // and stored packed over S^T's columns, then released to the dV product.
+      constexpr int NCOL = TN / G;
+      float pf[NCOL];
 #pragma unroll
-      for (int cc = 0; cc < TN / (32 * G); ++cc) {
-        uint32_t st[32], dpt[32];
+      for (int cc = 0; cc < NCOL / 32; ++cc) {
+        uint32_t st[32];
         tmem_ld32x32b_x32(tS + 32 * cc, st);
-        tmem_ld32x32b_x32(tP + 32 * cc, dpt);
-        uint32_t pk[16], dk[16];
-        // This chunk's 32 columns of L and D, read as 16-byte shared-memory loads (the same
-        // address in every lane: one broadcast each), four columns (two pairs) per load.
-        const float4* l4 = reinterpret_cast<const float4*>(lv + g * (TN / G) + 32 * cc);
-        const float4* d4 = reinterpret_cast<const float4*>(dv + g * (TN / G) + 32 * cc);
+        uint32_t pk[16];
+        // This chunk's 32 columns of L, read as 16-byte shared-memory loads (the same address
+        // in every lane: one broadcast each), four columns (two pairs) per load.
+        const float4* l4 = reinterpret_cast<const float4*>(lv + g * NCOL + 32 * cc);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const float4 lq = l4[q], dq = d4[q];
+          const float4 lq = l4[q];
           const float lcol[4] = {lq.x, lq.y, lq.z, lq.w};
-          const float dcol[4] = {dq.x, dq.y, dq.z, dq.w};
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int i = 2 * q + h;
-            // Pair (2i, 2i+1) in packed fp32: x = s*c - L, P = 2^x, dS = P (dP - D).
+          for (int hh = 0; hh < 2; ++hh) {
+            const int i = 2 * q + hh;
+            // Pair (2i, 2i+1) in packed fp32: x = s*c - L, P = 2^x.
             const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(st[2 * i]), __uint_as_float(st[2 * i + 1])),
-                                       c2, f2_pack(-lcol[2 * h], -lcol[2 * h + 1]));
+                                       c2, f2_pack(-lcol[2 * hh], -lcol[2 * hh + 1]));
             float x0, x1;
             f2_unpack(x2, x0, x1);
             float pv[2] = {ex2_approx(x0), ex2_approx(x1)};
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const int col = g * (TN / G) + 32 * cc + 2 * i + e;
+              const int col = g * NCOL + 32 * cc + 2 * i + e;
               if (masked && col < first_vis) pv[e] = 0.f;
+              pf[32 * cc + 2 * i + e] = pv[e];
             }
-            const uint64_t p2 = f2_pack(pv[0], pv[1]);
-            const uint64_t ds2 = f2_mul(p2, f2_sub(f2_pack(__uint_as_float(dpt[2 * i]),
-                                                           __uint_as_float(dpt[2 * i + 1])),
-                                                   f2_pack(dcol[2 * h], dcol[2 * h + 1])));
-            float ds0, ds1;
-            f2_unpack(ds2, ds0, ds1);
             pk[i] = pack_half2(pv[0], pv[1], BF16);
-            dk[i] = pack_half2(ds0, ds1, BF16);
           }
         }
         tmem_st32x32b_x16(tS + 16 * cc, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_pp);
+      // Pass 2: dS^T = P^T (dP^T - D), stored packed over dP^T's columns.
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_dp, s & 1, wc))) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < NCOL / 32; ++cc) {
+        uint32_t dpt[32];
+        tmem_ld32x32b_x32(tP + 32 * cc, dpt);
+        uint32_t dk[16];
+        const float4* d4 = reinterpret_cast<const float4*>(dv + g * NCOL + 32 * cc);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 dq = d4[q];
+          const float dcol[4] = {dq.x, dq.y, dq.z, dq.w};
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int i = 2 * q + hh;
+            const uint64_t ds2 = f2_mul(f2_pack(pf[32 * cc + 2 * i], pf[32 * cc + 2 * i + 1]),
+                                        f2_sub(f2_pack(__uint_as_float(dpt[2 * i]),
+                                                       __uint_as_float(dpt[2 * i + 1])),
+                                               f2_pack(dcol[2 * hh], dcol[2 * hh + 1])));
+            float ds0, ds1;
+            f2_unpack(ds2, ds0, ds1);
+            dk[i] = pack_half2(ds0, ds1, BF16);
+          }
+        }
         tmem_st32x32b_x16(tP + 16 * cc, dk);
       }
       tmem_st_wait();
