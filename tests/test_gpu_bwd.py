@@ -83,6 +83,17 @@ def test_rectangular(Nq, Nk, causal):
     check_bwd(1, 4, 2, Nq, Nk, 64, "fp16", causal, seed=Nq + 3 * Nk)
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,dtype,causal", [
+    (2, 8, 2, 1000, 64, "fp16", True),     # 16 key tiles per dQ tile: the ring wraps
+    (1, 4, 1, 777, 128, "bf16", False),    # odd step counts, 4 query heads per KV head
+])
+def test_longer_ragged_sequences(B, Hq, Hkv, N, d, dtype, causal):
+    """Many steps per CTA with a ragged last tile: the dQ pass alternates its two dP
+    buffers and loads V ahead of K through several turns of the ring; the dK/dV pass runs
+    its two elementwise passes across the query heads of a group."""
+    check_bwd(B, Hq, Hkv, N, N, d, dtype, causal, seed=N + Hq)
+
+
 def full_size_case(name, checks):
     """The workload's full backward pass in one call; `checks` = [(b, kv_head)]: dK and dV
     of each listed KV head (all its query heads) and dQ of those query heads against the
