@@ -13,13 +13,17 @@
 //                             tiles; rows without a visible key and rows past Nq get
 //                             +inf, so their P is exactly 0 in both passes below.
 //   dQ pass (bwd_dq_tile)     one CTA per 128-row query tile: per key tile j,
-//                             S = Q K_j^T and dP = dO V_j^T (tcgen05, TMEM), then the
-//                             elementwise warps form dS and dQ += dS K_j (A = dS in TMEM).
+//                             S = Q K_j^T and dP = dO V_j^T (tcgen05, TMEM; two dP
+//                             buffers), then the elementwise warps form dS and
+//                             dQ += dS K_j (A = dS in TMEM); dP(j+1), and dQ(j) once
+//                             S(j+1) is issued, run beside the elementwise work.
 //   dK/dV pass (bwd_dkdv_tile) one CTA per 128-row key tile of a KV head: per query tile i
 //                             of every query head of its group, S^T = K Q_i^T and
-//                             dP^T = V dO_i^T, then P^T and dS^T, and dV += P^T dO_i,
-//                             dK += dS^T Q_i (A operands in TMEM). The group's query heads
-//                             are summed in TMEM, so no atomics are needed.
+//                             dP^T = V dO_i^T; the elementwise warps form P^T, then dS^T,
+//                             each released on its own barrier to dV += P^T dO_i and
+//                             dK += dS^T Q_i (A operands in TMEM), so that the next step's
+//                             P^T pass runs beside dK and the next dP^T. The group's query
+//                             heads are summed in TMEM, so no atomics are needed.
 // Causal masking is bottom-right aligned as in the forward: key j is visible to query i
 // iff j <= i + (Nk - Nq).
 #pragma once
@@ -103,11 +107,11 @@ fa_bwd_preprocess_kernel(const uint16_t* __restrict__ o, const uint16_t* __restr
 }
 
 // Per head-dimension configuration. Each CTA keeps one 128-row tile resident (Q and dO
-// in the dQ kernel, K and V in the dK/dV kernel) and streams the other side in tiles of
-// TN rows. d = 64 streams 64-row tiles, so that TMEM (S | dP | accumulators) fits in 256
-// columns and shared memory in half an SM: two CTAs per SM then overlap one's elementwise
-// step with the other's products (each CTA on its own is serial: products, elementwise,
-// products). d = 128 streams 128-row tiles, one CTA per SM.
+// in the dQ pass, K and V in the dK/dV pass) and streams the other side in tiles of TN
+// rows. d = 64 streams 64-row tiles, so that TMEM (S | dP | accumulators | second dP)
+// fits in 256 columns and shared memory in half an SM, two CTAs per SM; d = 128 streams
+// 128-row tiles, one CTA per SM. Within a CTA the products of one step overlap the
+// elementwise work of another (see the two passes below).
 template <int D>
 struct BwdCfg {
   static constexpr int TN = (D == 64) ? 64 : 128;    // rows of a streamed tile
@@ -399,7 +403,9 @@ __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtens
 // Q_i and dO_i of one TN-row query tile of one query head of the group (a 2-item ring
 // pair) plus that tile's L * log2(e) and D vectors. TMEM: S^T [0,TN) (P^T packed over its
 // first TN/2 columns), dP^T [TN,2TN) (dS^T packed over its first TN/2), dV [2TN, 2TN+D),
-// dK [2TN+D, 2TN+2D).
+// dK [2TN+D, 2TN+2D). Barriers per step: S^T ready, dP^T ready (MMA -> elementwise);
+// P^T written, dS^T written (elementwise -> MMA). Products in the order dV(s), S^T(s+1)
+// over P^T(s), dK(s), dP^T(s+1) over dS^T(s).
 template <int D, bool BF16, bool CAUSAL>
 __device__ __forceinline__ void bwd_dkdv_tile(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                               const CUtensorMap& tmV, const CUtensorMap& tmDO,
