@@ -390,8 +390,7 @@ def run_ours(args):
     calls.append({"name": "decode", "w": wd, "call": dec_call, "kind": "decode",
                   "work": kv_bytes + 2 * (dq.numel() + do.numel()) + 4 * dlse.numel(),
                   "kv_bytes": kv_bytes})
-    dec_kernel = ("fa_decode_tc_kernel" if wd.d == 128 and os.environ.get("FA_DECODE_CUDA_CORES") != "1"
-                  else "fa_decode_split_kernel")
+    dec_kernel = "fa_decode_tc_kernel" if wd.d == 128 else "fa_decode_split_kernel"
 
     def step(ev=None):
         for i, c in enumerate(calls):

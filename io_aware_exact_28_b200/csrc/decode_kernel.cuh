@@ -68,24 +68,11 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
-// A pair of fp32 values: one packed f32x2 register pair (FA_DEC_F32X2 = 1, default) or
-// two scalar floats.
-#ifndef FA_DEC_F32X2
-#define FA_DEC_F32X2 1
-#endif
-#if FA_DEC_F32X2
+// A pair of fp32 values in one packed f32x2 register pair.
 using pair_t = uint64_t;
 __device__ __forceinline__ pair_t pmake(float a, float b) { return f2_pack(a, b); }
 __device__ __forceinline__ void psplit(pair_t v, float& a, float& b) { f2_unpack(v, a, b); }
 __device__ __forceinline__ pair_t pfma(pair_t a, pair_t b, pair_t c) { return f2_fma(a, b, c); }
-#else
-using pair_t = float2;
-__device__ __forceinline__ pair_t pmake(float a, float b) { return make_float2(a, b); }
-__device__ __forceinline__ void psplit(pair_t v, float& a, float& b) { a = v.x; b = v.y; }
-__device__ __forceinline__ pair_t pfma(pair_t a, pair_t b, pair_t c) {
-  return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
-}
-#endif
 
 // Two 16-bit values in one 32-bit word -> a pair (low element first).
 template <bool BF16>

@@ -232,16 +232,16 @@ fa_status dispatch_varlen(bool varlen, int causal, bool paged, int dev, const CU
 // Decode sizing: the split length depends only on (B, Hq, max_kv_len) so that the
 // workspace query and the launch always agree.
 // ---------------------------------------------------------------------------------------
-// FA_DECODE_SPLIT_TOKENS (a power of two in [32, 4096]) overrides the choice; it is read
-// once per process, so the workspace query and the launch still agree.
-int split_tokens_override() {
-  static int v = [] {
-    const char* e = std::getenv("FA_DECODE_SPLIT_TOKENS");
-    const int x = e ? std::atoi(e) : 0;
-    return (x >= 32 && x <= 4096 && (x & (x - 1)) == 0) ? x : 0;
-  }();
-  return v;
-}
+// Build define FA_DECODE_SPLIT_TOKENS (a power of two in [32, 4096]) overrides the choice
+// (0: the sizing below).
+#ifndef FA_DECODE_SPLIT_TOKENS
+#define FA_DECODE_SPLIT_TOKENS 0
+#endif
+static_assert(FA_DECODE_SPLIT_TOKENS == 0 ||
+                  (FA_DECODE_SPLIT_TOKENS >= 32 && FA_DECODE_SPLIT_TOKENS <= 4096 &&
+                   (FA_DECODE_SPLIT_TOKENS & (FA_DECODE_SPLIT_TOKENS - 1)) == 0),
+              "FA_DECODE_SPLIT_TOKENS: a power of two in [32, 4096], or 0");
+constexpr int split_tokens_override() { return FA_DECODE_SPLIT_TOKENS; }
 
 int decode_split_tokens(int B, int Hq, int max_len) {
   if (split_tokens_override()) return split_tokens_override();
@@ -258,15 +258,12 @@ struct DecodeLayout {
   size_t o_bytes, lse_off, ticket_off, total;
 };
 
-// d = 128 decodes on the tensor cores in 128-token tiles (decode_tc_kernel.cuh) unless
-// FA_DECODE_CUDA_CORES=1 selects the CUDA-core kernel (decode_kernel.cuh).
-bool use_tc_decode(int d) {
-  static const bool cuda_cores = [] {
-    const char* e = std::getenv("FA_DECODE_CUDA_CORES");
-    return e && std::atoi(e) == 1;
-  }();
-  return d == fa::kTcD && !cuda_cores;
-}
+// d = 128 decodes on the tensor cores in 128-token tiles (decode_tc_kernel.cuh) unless the
+// build define FA_DECODE_CUDA_CORES=1 selects the CUDA-core kernel (decode_kernel.cuh).
+#ifndef FA_DECODE_CUDA_CORES
+#define FA_DECODE_CUDA_CORES 0
+#endif
+bool use_tc_decode(int d) { return d == fa::kTcD && !FA_DECODE_CUDA_CORES; }
 
 bool decode_layout(int B, int Hq, int max_len, int d, DecodeLayout* L) {
   if (B <= 0 || Hq <= 0 || max_len <= 0 || d <= 0) return false;

@@ -54,9 +54,6 @@ struct EmptyBase {};
 #ifndef FA_D64_BN
 #define FA_D64_BN 64
 #endif
-#ifndef FA_REGSPLIT
-#define FA_REGSPLIT 1
-#endif
 // 64-key tiles: exponential pairs, of the 16 in each 32-score chunk, evaluated on the FMA
 // pipe (exp2_emu) instead of the MUFU unit (0, 1, 2 or 4). A 64-key tile's softmax needs
 // twice the MUFU time of its two products; 128-key tiles (16-bit or E4M3) are faster with
@@ -87,7 +84,7 @@ struct FwdCfg {
   static constexpr int THREADS = NARROW ? 320 : 384;
   static constexpr int WARP_PRODUCER = 4 * QT;        // TMA producer warp
   static constexpr int WARP_MMA = 4 * QT + 1;         // TMEM allocator and MMA issuer
-  static constexpr bool REGSPLIT = !NARROW && FA_REGSPLIT;
+  static constexpr bool REGSPLIT = !NARROW;            // warpgroup register re-split
   // Pairs i (0-15) of a 32-score chunk whose 2^x comes from exp2_emu.
   static constexpr int EMU_PAIRS = NARROW ? FA_EXP2_EMU_D64 : 0;
   static_assert(EMU_PAIRS == 0 || EMU_PAIRS == 1 || EMU_PAIRS == 2 || EMU_PAIRS == 4,
