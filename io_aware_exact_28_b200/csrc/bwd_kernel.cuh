@@ -63,6 +63,7 @@ struct BwdParams {
   int causal_offset;      // Nk - Nq
   float scale, scale_log2;
   uint64_t timeout_ns;
+  int skip_resident_load;   // test hook: the resident tiles are never loaded
 };
 
 // ------------------------------------------------------------------------------------
@@ -211,7 +212,7 @@ __device__ __forceinline__ void bwd_dq_tile(const CUtensorMap& tmQ, const CUtens
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && n_kv > 0) {
       mbar_arrive_expect_tx(bar_a, 2 * C::TILE_BYTES);
-      for (int ch = 0; ch < C::NCH; ++ch) {
+      for (int ch = 0; ch < C::NCH && !p.skip_resident_load; ++ch) {
         tma_load_3d(base + C::A_OFF + ch * C::CHUNK, &tmQ, bar_a, ch * 64, q0, bh);
         tma_load_3d(base + C::A_OFF + C::TILE_BYTES + ch * C::CHUNK, &tmDO, bar_a, ch * 64, q0, bh);
       }
@@ -477,7 +478,7 @@ __device__ __forceinline__ void bwd_dkdv_tile(const CUtensorMap& tmQ, const CUte
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && n_steps > 0) {
       mbar_arrive_expect_tx(bar_a, 2 * C::TILE_BYTES);
-      for (int ch = 0; ch < C::NCH; ++ch) {
+      for (int ch = 0; ch < C::NCH && !p.skip_resident_load; ++ch) {
         tma_load_3d(base + C::A_OFF + ch * C::CHUNK, &tmK, bar_a, ch * 64, k0, bh_kv);
         tma_load_3d(base + C::A_OFF + C::TILE_BYTES + ch * C::CHUNK, &tmV, bar_a, ch * 64, k0, bh_kv);
       }

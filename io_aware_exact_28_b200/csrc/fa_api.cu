@@ -615,6 +615,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   prm.scale = scale;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  prm.skip_resident_load = g_skip_q_load.load(std::memory_order_relaxed);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 64)
     return bf16 ? launch_bwd<64, true>(dev, mp, o, dout, lse, dq, dk, dv, prm, BH, BHkv, n_q, n_k, causal, st)

@@ -94,6 +94,31 @@ def test_longer_ragged_sequences(B, Hq, Hkv, N, d, dtype, causal):
     check_bwd(B, Hq, Hkv, N, N, d, dtype, causal, seed=N + Hq)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_bounded_wait_reports_timeout_and_context_survives(d):
+    """Test hook: neither pass loads its resident tiles, so every wait on them runs out
+    after 20 ms; the kernels record FA_ERR_DEVICE_TIMEOUT, drain and return, and the next
+    call is correct."""
+    dtype = "fp16" if d == 64 else "bf16"
+    q, k, v = make_fwd_inputs(1, 2, 1, 256, 256, d, dtype, seed=31 + d)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(32)).to(q.dtype)
+    qd, kd, vd, dod = q.to(DEV), k.to(DEV), v.to(DEV), dout.to(DEV)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = fa.fwd(qd, kd, vd, causal=True, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.device_status(clear=True) == fa.FA_OK
+    fa.set_wait_timeout_ns(20_000_000)
+    fa.debug_skip_q_load(True)
+    try:
+        fa.bwd(qd, kd, vd, o, lse, dod, causal=True, scale=scale)
+        status = fa.device_status(clear=True)
+    finally:
+        fa.debug_skip_q_load(False)
+        fa.set_wait_timeout_ns(0)
+    assert status == fa.FA_ERR_DEVICE_TIMEOUT
+    check_bwd(1, 2, 1, 256, 256, d, dtype, True, seed=31 + d)
+
+
 def full_size_case(name, checks):
     """The workload's full backward pass in one call; `checks` = [(b, kv_head)]: dK and dV
     of each listed KV head (all its query heads) and dQ of those query heads against the
