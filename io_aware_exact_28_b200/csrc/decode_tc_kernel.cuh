@@ -95,6 +95,7 @@ struct DecodeTcParams {
   int max_len, split_tokens, n_split;
   float scale_log2;
   uint64_t timeout_ns;
+  int skip_q_load;        // test hook: the Q tiles are never loaded
   PagedKV pk;             // PAGED kernels only
 };
 
@@ -314,7 +315,7 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           if (uc >= 2 && !mbar_wait(bar_qempty(qb), ((uc >> 1) - 1) & 1, wc)) { ok = false; break; }
           mbar_arrive_expect_tx(bar_qfull(qb), kTcQBytes);
           const int row0 = w.b * p.Hq + w.kvh * p.G + w.g0;
-          for (int ch = 0; ch < 2; ++ch)
+          for (int ch = 0; ch < 2 && !p.skip_q_load; ++ch)
             tma_load_3d(base + kTcOffQ + qb * kTcQBytes + ch * kTcSmallChunk, &tmQ, bar_qfull(qb),
                         ch * 64, row0, 0);
           ++uc;
@@ -404,7 +405,7 @@ fa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           } else {
             mbar_arrive_expect_tx(bar_qfull(qb), kTcQBytes);
             const int row0 = w.b * p.Hq + w.kvh * p.G + w.g0;
-            for (int ch = 0; ch < 2; ++ch)
+            for (int ch = 0; ch < 2 && !p.skip_q_load; ++ch)
               tma_load_3d(base + kTcOffQ + qb * kTcQBytes + ch * kTcSmallChunk, &tmQ, bar_qfull(qb),
                           ch * 64, row0, 0);
           }

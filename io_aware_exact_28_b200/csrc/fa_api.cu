@@ -410,6 +410,7 @@ fa_status launch_decode_tc_t(int dev, const void* q, const void* kc, const void*
   tp.n_split = L.n_split;
   tp.scale_log2 = scale * 1.4426950408889634f;
   tp.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  tp.skip_q_load = g_skip_q_load.load(std::memory_order_relaxed);
   tp.pk = PAGED ? pg->device(Hkv) : fa::PagedKV{};
   const long long n_units = static_cast<long long>(L.n_split) * B * Hkv * tp.n_gt;
   if (n_units >= (1LL << 31)) return FA_ERR_INVALID_ARG;

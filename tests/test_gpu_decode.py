@@ -136,3 +136,27 @@ def test_many_sequences_every_tail_size():
     clamped = torch.tensor([min(max(n, 0), cache) for n in lens])
     O, L = decode_f64(q, kc, vc, clamped, scale)
     assert_close(o.cpu(), lse.cpu(), O, L, "bf16", "every tail size", strict=False)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """Test hook: the d = 128 decode never loads its query rows, so every wait on them runs
+    out after 20 ms; the split kernel records FA_ERR_DEVICE_TIMEOUT, drains and returns, and
+    the next call (whose counter reset zeroes the ticket counter left behind) is correct."""
+    lens = [700, 1500, 33, 4096]
+    kv_lens, q, kc, vc = make_decode_inputs(4, 8, 2, 4096, 128, "bf16", 1, 4096, 5,
+                                            kv_lens=torch.tensor(lens))
+    qd, kd, vd, ld = q.to(DEV), kc.to(DEV), vc.to(DEV), kv_lens.to(DEV)
+    scale = 1.0 / math.sqrt(128)
+    torch.cuda.synchronize()
+    assert fa.device_status(clear=True) == fa.FA_OK
+    fa.set_wait_timeout_ns(20_000_000)
+    fa.debug_skip_q_load(True)
+    try:
+        fa.decode(qd, kd, vd, ld, scale=scale)
+        torch.cuda.synchronize()
+        status = fa.device_status(clear=True)
+    finally:
+        fa.debug_skip_q_load(False)
+        fa.set_wait_timeout_ns(0)
+    assert status == fa.FA_ERR_DEVICE_TIMEOUT
+    check(4, 8, 2, 4096, 128, "bf16", lens, seed=5)
