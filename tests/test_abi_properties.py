@@ -69,7 +69,7 @@ def invalid_arg_fault(draw, a):
     else:                                   # B * Hq reaches 2^31 query heads
         a["Hkv"] = 1
         a["Hq"] = draw(st.integers(2, 64))
-        a["B"] = min((1 << 31) - 1, (1 << 31) // a["Hq"] + draw(st.integers(0, 64)))
+        a["B"] = -(-(1 << 31) // a["Hq"]) + draw(st.integers(0, 64))   # ceil(2^31 / Hq) + k
         assert a["B"] * a["Hq"] >= (1 << 31)
     return a
 
