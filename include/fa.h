@@ -330,9 +330,10 @@ FA_API void fa_set_wait_timeout_ns(uint64_t ns);
 /*
  * fa_debug_skip_q_load — test hook for the bounded-wait path: when non-zero, fa_fwd
  * kernels launched afterwards never issue the Q-tile load, the d = 128 decode kernels
- * never load their query rows, and fa_bwd kernels never issue the loads of their resident
- * tiles (Q and dO, or K and V), so the barrier that waits for them is never completed and
- * every wait that depends on it runs out. The kernel records
+ * never load their query rows, the other decode kernels never fill their K/V stages, and
+ * fa_bwd kernels never issue the loads of their resident tiles (Q and dO, or K and V), so
+ * the barriers that wait for them are never completed and every wait that depends on them
+ * runs out. The kernel records
  * FA_ERR_DEVICE_TIMEOUT and returns; the outputs are then unspecified. 0 restores normal
  * operation.
  */

@@ -53,6 +53,7 @@ struct DecodeParams {
   int max_len, split_tokens, n_split;
   float scale_log2;
   uint64_t timeout_ns;
+  int skip_kv_load;       // test hook: the ring stages are armed but never filled
   PagedKV pk;             // PAGED kernels only (kc, vc are then the page pools)
 };
 
@@ -169,6 +170,7 @@ fa_decode_split_kernel(const DecodeParams p) {
       const uint32_t b0 = ok0 ? static_cast<uint32_t>(n0) * C::ROW : 0u;
       const uint32_t b1 = ok1 ? static_cast<uint32_t>(n1) * C::ROW : 0u;
       mbar_arrive_expect_tx(bar_full + 8 * slot, 2 * (b0 + b1));
+      if (p.skip_kv_load) return;
       const size_t page_elems = static_cast<size_t>(ps) * D;
       if (ok0) {
         const size_t off = (static_cast<size_t>(e0) * p.Hkv + kvh) * page_elems +
@@ -184,6 +186,7 @@ fa_decode_split_kernel(const DecodeParams p) {
     } else {
       const uint32_t bytes = static_cast<uint32_t>(n) * C::ROW;
       mbar_arrive_expect_tx(bar_full + 8 * slot, 2 * bytes);
+      if (p.skip_kv_load) return;
       bulk_load(sK + slot * C::STAGE_BYTES, kg + static_cast<size_t>(st) * kDecStageTok * D, bytes,
                 bar_full + 8 * slot);
       bulk_load(sV + slot * C::STAGE_BYTES, vg + static_cast<size_t>(st) * kDecStageTok * D, bytes,

@@ -780,6 +780,7 @@ fa_status decode_impl(const void* q, const void* kcache, const void* vcache, con
   dp.n_split = L.n_split;
   dp.scale_log2 = scale * 1.4426950408889634f;
   dp.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  dp.skip_kv_load = g_skip_q_load.load(std::memory_order_relaxed);
   dp.pk = pg ? pg->device(Hkv) : fa::PagedKV{};
 #define FA_DEC_CASE(D_, BF_)                                                         \
   return pg ? launch_decode_g<D_, BF_, true>(dev, dp, cp, B, Hkv, G, st)             \

@@ -160,3 +160,26 @@ def test_bounded_wait_reports_timeout_and_context_survives():
         fa.set_wait_timeout_ns(0)
     assert status == fa.FA_ERR_DEVICE_TIMEOUT
     check(4, 8, 2, 4096, 128, "bf16", lens, seed=5)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives_cuda_cores():
+    """Test hook on the CUDA-core decode (d = 64): the K/V ring stages are armed but never
+    filled, so every wait on them runs out after 20 ms; the kernel records
+    FA_ERR_DEVICE_TIMEOUT, drains and returns, and the next call is correct."""
+    lens = [300, 64, 1000, 5]
+    kv_lens, q, kc, vc = make_decode_inputs(4, 8, 4, 1024, 64, "fp16", 1, 1024, 6,
+                                            kv_lens=torch.tensor(lens))
+    qd, kd, vd, ld = q.to(DEV), kc.to(DEV), vc.to(DEV), kv_lens.to(DEV)
+    torch.cuda.synchronize()
+    assert fa.device_status(clear=True) == fa.FA_OK
+    fa.set_wait_timeout_ns(20_000_000)
+    fa.debug_skip_q_load(True)
+    try:
+        fa.decode(qd, kd, vd, ld, scale=0.125)
+        torch.cuda.synchronize()
+        status = fa.device_status(clear=True)
+    finally:
+        fa.debug_skip_q_load(False)
+        fa.set_wait_timeout_ns(0)
+    assert status == fa.FA_ERR_DEVICE_TIMEOUT
+    check(4, 8, 4, 1024, 64, "fp16", lens, seed=6)
