@@ -1,4 +1,5 @@
-"""Tiled online-softmax attention in plain float64 Python, for tiny inputs.
+"""Tiled online-softmax attention, and its backward pass by tile-wise recomputation, in
+plain float64 Python, for tiny inputs.
 
 TEST INFRASTRUCTURE ONLY (see `oracle/attention.py`). It exists to check the pages'
 exactness claim: processing the keys tile by tile with a running maximum and a running
@@ -28,7 +29,7 @@ import numpy as np
 
 from .attention import _f64, visible_mask
 
-__all__ = ["tiled_attention_f64"]
+__all__ = ["tiled_attention_f64", "tiled_attention_bwd_f64"]
 
 
 def tiled_attention_f64(Q, K, V, causal: bool, scale: float, Br: int, Bc: int):
@@ -63,3 +64,43 @@ def tiled_attention_f64(Q, K, V, causal: bool, scale: float, Br: int, Bc: int):
         O[r0:r1][seen] = Oi[seen] / li[seen, None]
         L[r0:r1][seen] = mi[seen] + np.log(li[seen])
     return O, L
+
+
+def tiled_attention_bwd_f64(Q, K, V, dO, O, L, causal: bool, scale: float, Br: int, Bc: int):
+    """One head's gradients by tile-wise recomputation, float64: (dQ [Nq,d], dK, dV [Nk,d]).
+
+    This restates the backward pass the way the tiled method runs it (page "Flash
+    Attention" (zh), "IO 感知的算法设计": no N x N matrix is kept, so the scores are
+    recomputed tile by tile from Q, K and the saved per-row statistic L). O and L are the
+    forward's outputs. First D_i = sum_c dO_ic O_ic for every row (equal to
+    sum_j P_ij dP_ij because O = P V); then, for every key tile j of Bc keys and every
+    query tile i of Br rows:
+
+        S_ij  = scale * Q_i K_j^T (masked: -inf)     P_ij = exp(S_ij - L_i)
+        dV_j += P_ij^T dO_i                          dP_ij = dO_i V_j^T
+        dS_ij = P_ij * (dP_ij - D_i)
+        dQ_i += scale * dS_ij K_j                    dK_j += scale * dS_ij^T Q_i
+
+    A row with L_i = -inf (no visible key) has P = 0 and contributes nothing."""
+    Q, K, V, dO, O, L = _f64(Q), _f64(K), _f64(V), _f64(dO), _f64(O), _f64(L)
+    Nq, d = Q.shape
+    Nk = K.shape[0]
+    D = (dO * O).sum(axis=1)
+    Lf = np.where(np.isfinite(L), L, np.inf)          # exp(-inf - inf) = 0 for empty rows
+    dQ = np.zeros((Nq, d))
+    dK = np.zeros((Nk, d))
+    dV = np.zeros((Nk, d))
+    for j in range(-(-Nk // Bc)):
+        c0, c1 = j * Bc, min(Nk, (j + 1) * Bc)
+        Kj, Vj = K[c0:c1], V[c0:c1]
+        for i in range(-(-Nq // Br)):
+            r0, r1 = i * Br, min(Nq, (i + 1) * Br)
+            vis = visible_mask(np.arange(r0, r1), Nq, Nk, causal)[:, c0:c1]
+            Sij = np.where(vis, scale * (Q[r0:r1] @ Kj.T), -np.inf)
+            Pij = np.exp(Sij - Lf[r0:r1, None])
+            dV[c0:c1] += Pij.T @ dO[r0:r1]
+            dPij = dO[r0:r1] @ Vj.T
+            dSij = Pij * (dPij - D[r0:r1, None])
+            dQ[r0:r1] += scale * (dSij @ Kj)
+            dK[c0:c1] += scale * (dSij.T @ Q[r0:r1])
+    return dQ, dK, dV

@@ -11,13 +11,15 @@ drawn by hypothesis:
 * constant V rows give dP - D = 0, hence dQ = dK = 0; dV = P^T dO does not depend on V;
 * without the mask, permuting query rows (with their dO rows) permutes dQ and leaves dK,
   dV unchanged; permuting key rows (K and V together) permutes dK, dV and leaves dQ;
-* sequences of a batch are independent.
+* sequences of a batch are independent;
+* the tile-wise recomputation (`tiled_attention_bwd_f64`: P rebuilt from the forward's L,
+  D taken from the forward's O) equals the untiled derivative for any tile sizes.
 """
 import numpy as np
 from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
 
-from oracle import attention_bwd_f64
+from oracle import attention_bwd_f64, attention_f64, tiled_attention_bwd_f64
 
 SETTINGS = settings(derandomize=True, max_examples=40, deadline=None, suppress_health_check=[HealthCheck.too_slow])
 ATOL = 1e-10
@@ -117,3 +119,24 @@ def test_key_rows_are_equivariant_without_mask(s):
     dq1, dk1, dv1 = attention_bwd_f64(q, k, v, do, False, s["scale"])
     dq2, dk2, dv2 = attention_bwd_f64(q, k[:, :, perm], v[:, :, perm], do, False, s["scale"])
     assert allclose([dq2, dk2, dv2], [dq1, dk1[:, :, perm], dv1[:, :, perm]])
+
+
+@SETTINGS
+@given(shapes(), st.booleans(), st.integers(1, 20), st.integers(1, 20))
+def test_tiled_recomputation_matches_for_any_tile_sizes(s, causal, Br, Bc):
+    """The backward pass as the tiled method runs it: for each key tile and query tile, P
+    is recomputed from L and dV, dQ, dK accumulate tile by tile."""
+    q, k, v, do, _ = make(s)
+    O, L = attention_f64(q, k, v, causal, s["scale"])
+    dq, dk, dv = attention_bwd_f64(q, k, v, do, causal, s["scale"])
+    g = s["Hq"] // s["Hkv"]
+    for b in range(s["B"]):
+        dk_t = np.zeros_like(dk[b])
+        dv_t = np.zeros_like(dv[b])
+        for h in range(s["Hq"]):
+            dq_h, dk_h, dv_h = tiled_attention_bwd_f64(q[b, h], k[b, h // g], v[b, h // g], do[b, h],
+                                                       O[b, h], L[b, h], causal, s["scale"], Br, Bc)
+            assert np.allclose(dq_h, dq[b, h], rtol=0, atol=ATOL)
+            dk_t[h // g] += dk_h
+            dv_t[h // g] += dv_h
+        assert allclose([dk_t, dv_t], [dk[b], dv[b]])
