@@ -18,6 +18,16 @@ rows in blocks of Br, keys in blocks of Bc inside each row block, and for every 
 and after the last tile ``O_i / l`` and ``L_i = m + log(l)``. Tr = ceil(Nq/Br),
 Tc = ceil(Nk/Bc); masked scores are -inf.
 
+Two optional arguments restate the kernels' departures from that recurrence, both of which
+cancel in O / l (the properties check that they do, for any tile sizes):
+
+* ``tau`` (log2 units, >= 0): a lazy running maximum. A row's m moves to the tile's
+  maximum only when that maximum exceeds m by more than tau * ln 2; otherwise m, l and O
+  keep their scale and P_ij = exp(S_ij - m) may reach 2^tau. tau = 0 is the recurrence
+  above. The 16-bit kernels use 8, the E4M3 kernel 4.
+* ``offset`` (log2 units): P_ij = exp(S_ij - m + offset * ln 2), and the offset is taken
+  back out of L. The E4M3 kernel uses 4, so that P stays in E4M3's normal range.
+
 Prior art, not followed: the tiling pseudo-code of page "Flash Attention ... IO-aware
 exact" (fr) has the same outer loop over Q_i and returns O and L, but it has no loop over
 j, leaves Tr undefined and applies a separate softmax to each tile before a plain ``+=``,
@@ -32,7 +42,8 @@ from .attention import _f64, visible_mask
 __all__ = ["tiled_attention_f64", "tiled_attention_bwd_f64"]
 
 
-def tiled_attention_f64(Q, K, V, causal: bool, scale: float, Br: int, Bc: int):
+def tiled_attention_f64(Q, K, V, causal: bool, scale: float, Br: int, Bc: int,
+                        tau: float = 0.0, offset: float = 0.0):
     """One head: Q [Nq,d], K and V [Nk,d]. Returns O [Nq,d] and L [Nq] (float64)."""
     Q, K, V = _f64(Q), _f64(K), _f64(V)
     Nq, d = Q.shape
@@ -41,6 +52,7 @@ def tiled_attention_f64(Q, K, V, causal: bool, scale: float, Br: int, Bc: int):
     Tc = -(-Nk // Bc)
     O = np.zeros((Nq, d))
     L = np.full(Nq, -np.inf)
+    tau_ln, off_ln = tau * np.log(2.0), offset * np.log(2.0)
     for i in range(Tr):
         r0, r1 = i * Br, min(Nq, (i + 1) * Br)
         Qi = Q[r0:r1]
@@ -53,16 +65,17 @@ def tiled_attention_f64(Q, K, V, causal: bool, scale: float, Br: int, Bc: int):
             Sij = scale * (Qi @ Kj.T)
             vis = visible_mask(np.arange(r0, r1), Nq, Nk, causal)[:, c0:c1]
             Sij = np.where(vis, Sij, -np.inf)
-            m_new = np.maximum(mi, Sij.max(axis=1))
+            tmax = Sij.max(axis=1)
+            m_new = np.where(tmax > mi + tau_ln, tmax, mi)    # tau = 0: max(m, rowmax)
             ref = np.where(np.isfinite(m_new), m_new, 0.0)   # rows with nothing visible yet
             alpha = np.where(np.isfinite(mi), np.exp(mi - ref), 0.0)
-            Pij = np.exp(Sij - ref[:, None])
+            Pij = np.exp(Sij - ref[:, None] + off_ln)
             li = alpha * li + Pij.sum(axis=1)
             Oi = alpha[:, None] * Oi + Pij @ Vj
             mi = m_new
         seen = li > 0
         O[r0:r1][seen] = Oi[seen] / li[seen, None]
-        L[r0:r1][seen] = mi[seen] + np.log(li[seen])
+        L[r0:r1][seen] = mi[seen] + np.log(li[seen]) - off_ln
     return O, L
 
 

@@ -4,7 +4,9 @@ exactness paragraph), over random shapes drawn by hypothesis. Each property is o
 plausible slip in the oracle would break: a wrong operand order breaks linearity in V or
 row equivariance, a wrong head mapping breaks the grouped-query identity, a misplaced
 scale breaks the scale-folding identity, a mis-aligned causal mask breaks the single-row
-and truncation identities, and mixed-up batch indexing breaks batch independence."""
+and truncation identities, and mixed-up batch indexing breaks batch independence. The
+tiled restatement, with and without the kernels' lazy running maximum and exponent
+offset, must equal the definition for any tile sizes."""
 import numpy as np
 from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
@@ -138,4 +140,20 @@ def test_tiled_restatement_matches_for_any_tile_sizes(s, causal, Br, Bc):
         for h in range(s["Hq"]):
             Ot, Lt = tiled_attention_f64(q[b, h], k[b, h // g], v[b, h // g], causal, s["scale"],
                                          Br, Bc)
+            assert close(Ot, O[b, h]) and close(Lt, L[b, h])
+
+
+@SETTINGS
+@given(shapes(max_n=40), st.booleans(), st.integers(1, 40), st.integers(1, 40),
+       st.floats(0.0, 16.0), st.floats(-4.0, 8.0))
+def test_lazy_rescale_and_exponent_offset_are_exact(s, causal, Br, Bc, tau, offset):
+    """A running maximum that moves only when a tile's maximum passes it by more than
+    2^tau, and an exponent offset taken back out of the LSE, leave O and LSE unchanged."""
+    q, k, v, _ = make(s)
+    O, L = attention_f64(q, k, v, causal, s["scale"])
+    g = s["Hq"] // s["Hkv"]
+    for b in range(s["B"]):
+        for h in range(s["Hq"]):
+            Ot, Lt = tiled_attention_f64(q[b, h], k[b, h // g], v[b, h // g], causal, s["scale"],
+                                         Br, Bc, tau=tau, offset=offset)
             assert close(Ot, O[b, h]) and close(Lt, L[b, h])
