@@ -1,5 +1,5 @@
-"""Tiled online-softmax attention, and its backward pass by tile-wise recomputation, in
-plain float64 Python, for tiny inputs.
+"""Tiled online-softmax attention, its backward pass by tile-wise recomputation, and
+split-KV decode merged by the chunks' LSEs, in plain float64 Python, for tiny inputs.
 
 TEST INFRASTRUCTURE ONLY (see `oracle/attention.py`). It exists to check the pages'
 exactness claim: processing the keys tile by tile with a running maximum and a running
@@ -39,7 +39,7 @@ import numpy as np
 
 from .attention import _f64, visible_mask
 
-__all__ = ["tiled_attention_f64", "tiled_attention_bwd_f64"]
+__all__ = ["tiled_attention_f64", "tiled_attention_bwd_f64", "split_kv_decode_f64"]
 
 
 def tiled_attention_f64(Q, K, V, causal: bool, scale: float, Br: int, Bc: int,
@@ -117,3 +117,39 @@ def tiled_attention_bwd_f64(Q, K, V, dO, O, L, causal: bool, scale: float, Br: i
             dQ[r0:r1] += scale * (dSij @ Kj)
             dK[c0:c1] += scale * (dSij.T @ Q[r0:r1])
     return dQ, dK, dV
+
+
+def split_kv_decode_f64(q, K, V, bounds, scale: float):
+    """One decode head over keys split into chunks, then merged by their LSEs (float64).
+
+    q [d]; K and V [n, d]; bounds: 0 = b_0 <= b_1 <= ... <= b_S = n, chunk s holding keys
+    [b_s, b_{s+1}) (a chunk may be empty). Each chunk is its own attention problem, giving
+    a partial O_s and LSE_s (an empty chunk gives O_s = 0, LSE_s = -inf); the merge is
+
+        LSE = log sum_s exp(LSE_s)        O = sum_s exp(LSE_s - LSE) O_s
+
+    which is exact because the softmax normaliser is a sum over keys, the same
+    associativity the online-softmax update uses (page "Kotaemon FlashAttention",
+    exactness paragraph: the block-wise result is identical to the original). Returns
+    (O [d], LSE); no keys at all gives O = 0, LSE = -inf."""
+    q, K, V = _f64(q), _f64(K), _f64(V)
+    bounds = [int(x) for x in bounds]
+    parts = []
+    for s0, s1 in zip(bounds[:-1], bounds[1:]):
+        if s1 <= s0:
+            parts.append((np.zeros(V.shape[1]), -np.inf))
+            continue
+        sc = scale * (K[s0:s1] @ q)
+        m = sc.max()
+        e = np.exp(sc - m)
+        parts.append(((e @ V[s0:s1]) / e.sum(), m + np.log(e.sum())))
+    lses = np.array([l for _, l in parts])
+    if not np.isfinite(lses).any():
+        return np.zeros(V.shape[1]), -np.inf
+    mx = lses[np.isfinite(lses)].max()
+    lse = mx + np.log(np.sum(np.exp(lses[np.isfinite(lses)] - mx)))
+    O = np.zeros(V.shape[1])
+    for o_s, l_s in parts:
+        if np.isfinite(l_s):
+            O += np.exp(l_s - lse) * o_s
+    return O, lse

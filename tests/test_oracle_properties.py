@@ -11,7 +11,7 @@ import numpy as np
 from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
 
-from oracle import attention_f64, tiled_attention_f64
+from oracle import attention_f64, decode_f64, split_kv_decode_f64, tiled_attention_f64
 
 SETTINGS = settings(derandomize=True, max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
 ATOL = 1e-11
@@ -157,3 +157,19 @@ def test_lazy_rescale_and_exponent_offset_are_exact(s, causal, Br, Bc, tau, offs
             Ot, Lt = tiled_attention_f64(q[b, h], k[b, h // g], v[b, h // g], causal, s["scale"],
                                          Br, Bc, tau=tau, offset=offset)
             assert close(Ot, O[b, h]) and close(Lt, L[b, h])
+
+
+@SETTINGS
+@given(st.integers(0, 40), st.sampled_from([1, 4, 8]), st.integers(0, 2**31 - 1),
+       st.floats(0.05, 2.0), st.lists(st.integers(0, 40), max_size=8))
+def test_split_kv_decode_merge_is_exact(n, d, seed, scale, cuts):
+    """Decode over keys cut into chunks (empty ones included), each chunk's (O, LSE) merged
+    by the LSE weights, equals decode over all keys at once."""
+    r = np.random.default_rng(seed)
+    q = r.standard_normal((1, 1, d))
+    k = r.standard_normal((1, 1, max(n, 1), d))
+    v = r.standard_normal((1, 1, max(n, 1), d))
+    bounds = [0] + sorted(min(c, n) for c in cuts) + [n]
+    O, L = split_kv_decode_f64(q[0, 0], k[0, 0, :n], v[0, 0, :n], bounds, scale)
+    Od, Ld = decode_f64(q, k, v, [n], scale)
+    assert close(O, Od[0, 0]) and close(np.array(L), Ld[0, 0])
