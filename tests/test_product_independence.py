@@ -1,0 +1,102 @@
+"""The product path and the oracle are independent, and the product has no fallback.
+
+* No file of the package (Python binding, CUDA sources, headers) imports, includes or
+  names the oracle, and importing the package loads no oracle module.
+* No oracle file imports the package or its compiled library.
+* The seeded input generators (`workloads/`), the one module both sides use, import
+  neither of them.
+* With its shared library missing, the binding raises `FALibraryError` on first use:
+  there is no CPU path to fall back to.
+CPU only.
+"""
+import ast
+import os
+import re
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+PKG = os.path.join(ROOT, "io_aware_exact_28_b200")
+
+
+def _files(top, exts):
+    for dirpath, _, names in os.walk(top):
+        if "__pycache__" in dirpath:
+            continue
+        for n in names:
+            if n.endswith(exts):
+                yield os.path.join(dirpath, n)
+
+
+def _imported_roots(path):
+    """Top-level module names a Python file imports (absolute imports only)."""
+    with open(path, encoding="utf-8") as f:
+        tree = ast.parse(f.read(), path)
+    roots = set()
+    for node in ast.walk(tree):
+        if isinstance(node, ast.Import):
+            roots.update(a.name.split(".")[0] for a in node.names)
+        elif isinstance(node, ast.ImportFrom) and node.level == 0 and node.module:
+            roots.add(node.module.split(".")[0])
+    return roots
+
+
+def test_package_sources_never_reach_the_oracle():
+    py = list(_files(PKG, (".py",)))
+    assert py
+    for p in py:
+        assert "oracle" not in _imported_roots(p), p
+    native = list(_files(PKG, (".cu", ".cuh", ".h", ".cpp"))) + \
+        list(_files(os.path.join(ROOT, "include"), (".h",)))
+    assert native
+    for p in native:
+        with open(p, encoding="utf-8") as f:
+            src = f.read()
+        assert not re.search(r'#\s*include\s*[<"][^>"]*oracle', src), p
+
+
+def test_oracle_never_imports_the_package():
+    files = list(_files(os.path.join(ROOT, "oracle"), (".py",)))
+    assert files
+    for p in files:
+        roots = _imported_roots(p)
+        assert "io_aware_exact_28_b200" not in roots and "ctypes" not in roots, p
+        with open(p, encoding="utf-8") as f:
+            assert "libfa_b200" not in f.read(), p
+
+
+def test_input_generators_import_neither_side():
+    files = list(_files(os.path.join(ROOT, "workloads"), (".py",)))
+    assert files
+    for p in files:
+        roots = _imported_roots(p)
+        assert not roots & {"oracle", "io_aware_exact_28_b200"}, (p, roots)
+
+
+def _run(code, **env):
+    e = dict(os.environ, **env)
+    e["PYTHONPATH"] = ROOT + os.pathsep + e.get("PYTHONPATH", "")
+    return subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                          cwd=ROOT, env=e, timeout=300)
+
+
+def test_importing_the_package_loads_no_oracle_module():
+    r = _run("import sys, io_aware_exact_28_b200 as fa\n"
+             "fa.lib()\n"
+             "bad = [m for m in sys.modules if m == 'oracle' or m.startswith('oracle.')]\n"
+             "print('LOADED', bad)\n")
+    assert r.returncode == 0, r.stderr
+    assert "LOADED []" in r.stdout, r.stdout
+
+
+def test_missing_library_fails_loudly():
+    missing = os.path.join(ROOT, "io_aware_exact_28_b200", "no_such_dir", "libfa_b200.so")
+    r = _run("import io_aware_exact_28_b200 as fa\n"
+             "try:\n"
+             "    fa.lib()\n"
+             "except fa.FALibraryError as e:\n"
+             "    print('RAISED', type(e).__name__)\n"
+             "else:\n"
+             "    print('LOADED')\n", FA_B200_LIB=missing)
+    assert r.returncode == 0, r.stderr
+    assert "RAISED FALibraryError" in r.stdout, r.stdout
