@@ -7,6 +7,8 @@
   neither of them.
 * With its shared library missing, the binding raises `FALibraryError` on first use:
   there is no CPU path to fall back to.
+* Outside the tests, the oracle is imported only by `smoke()` of the entry module and by
+  the CPU timing functions of `bench.py` (the CPU baseline and the reference arm).
 CPU only.
 """
 import ast
@@ -100,3 +102,31 @@ def test_missing_library_fails_loudly():
              "    print('LOADED')\n", FA_B200_LIB=missing)
     assert r.returncode == 0, r.stderr
     assert "RAISED FALibraryError" in r.stdout, r.stdout
+
+
+def _oracle_imports_by_function(path):
+    """{enclosing top-level function name or '<module>': count} of oracle imports."""
+    with open(path, encoding="utf-8") as f:
+        tree = ast.parse(f.read(), path)
+    found = {}
+
+    def visit(node, owner):
+        for child in ast.iter_child_nodes(node):
+            name = owner
+            if owner == "<module>" and isinstance(child, (ast.FunctionDef, ast.AsyncFunctionDef)):
+                name = child.name
+            if isinstance(child, ast.Import) and any(a.name.split(".")[0] == "oracle" for a in child.names):
+                found[name] = found.get(name, 0) + 1
+            if isinstance(child, ast.ImportFrom) and child.level == 0 and child.module and \
+                    child.module.split(".")[0] == "oracle":
+                found[name] = found.get(name, 0) + 1
+            visit(child, name)
+    visit(tree, "<module>")
+    return found
+
+
+def test_entry_points_reach_the_oracle_only_from_their_checking_legs():
+    entry = _oracle_imports_by_function(os.path.join(ROOT, "__graft_entry__.py"))
+    assert set(entry) == {"smoke"}, entry
+    bench = _oracle_imports_by_function(os.path.join(ROOT, "bench.py"))
+    assert bench and set(bench) <= {"oracle_rows_time", "oracle_baselines"}, bench
