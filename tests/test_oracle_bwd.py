@@ -1,6 +1,6 @@
 """Pins for the float64 backward oracle (oracle/backward.py), independent of its formulas:
-central finite differences of the forward oracle, closed-form invariants, and the
-grouped-query sum. CPU only."""
+central finite differences of the forward oracle, hand-worked gradients with exact
+closed-form values, closed-form invariants, and the grouped-query sum. CPU only."""
 import numpy as np
 import pytest
 
@@ -107,6 +107,64 @@ def test_rows_without_keys_contribute_nothing():
     np.testing.assert_allclose(dv, dv2, rtol=1e-12)
 
 
+LN2, LN3 = np.log(2.0), np.log(3.0)
+
+
+def _hand_worked_cases():
+    """Three tiny problems (d = 1, scale = 1/2) whose gradients were derived on paper from
+    O = softmax(scale * Q K^T) V. The scores are 0, ln 2, 2 ln 2 or 0, ln 3, so every P is
+    rational, and with L = sum(O * dO):
+        dV_j = sum_i P_ij dO_i,   dS_ij = P_ij (dO_i v_j - dO_i O_i),
+        dQ_i = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i.
+
+    A: q = 2 ln 2, k = (0, 1, 2), v = (7, 0, -7), dO = 2. P = (1/7, 2/7, 4/7), O = -3,
+       dS = (20/7, 12/7, -32/7): dQ = -26/7, dK = (20/7, 12/7, -32/7) ln 2,
+       dV = (2/7, 4/7, 8/7).
+    B: causal, two queries and two keys (bottom-right: row 0 sees key 0 only). Row 0:
+       q = 5, dO = 2, P = (1, 0), so dS = 0 and only dV_0 gains 2. Row 1: q = 2 ln 3,
+       k = (0, 1), v = (4, 0), dO = 1, P = (1/4, 3/4), O = 1, dS = (3/4, -3/4):
+       dQ = (0, -3/8), dK = (3/4, -3/4) ln 3, dV = (9/4, 3/4).
+    C: two query heads on one KV head (A's keys and values). Head 0 is A. Head 1: q = 0,
+       dO = 3, P = 1/3 each, O = 0, dS = (7, 0, -7): dQ = -7 and no dK. The KV head
+       sums both: dK = A's, dV = (9/7, 11/7, 15/7)."""
+    col = lambda *x: np.array(x, dtype=np.float64).reshape(-1, 1)
+    A = dict(q=col(2 * LN2)[None, None], k=col(0, 1, 2)[None, None], v=col(7, 0, -7)[None, None],
+             do=col(2)[None, None], causal=False,
+             dq=col(-26 / 7)[None, None], dk=(col(20, 12, -32) / 7 * LN2)[None, None],
+             dv=(col(2, 4, 8) / 7)[None, None])
+    B = dict(q=col(5, 2 * LN3)[None, None], k=col(0, 1)[None, None], v=col(4, 0)[None, None],
+             do=col(2, 1)[None, None], causal=True,
+             dq=col(0, -3 / 8)[None, None], dk=(col(3, -3) / 4 * LN3)[None, None],
+             dv=col(9 / 4, 3 / 4)[None, None])
+    C = dict(q=np.stack([col(2 * LN2), col(0)])[None], k=A["k"], v=A["v"],
+             do=np.stack([col(2), col(3)])[None], causal=False,
+             dq=np.stack([col(-26 / 7), col(-7)])[None], dk=A["dk"],
+             dv=(col(9, 11, 15) / 7)[None, None])
+    return {"A": A, "B": B, "C": C}
+
+
+def _hand_worked_matches(bwd):
+    """True if `bwd` (a replacement for the per-head gradient) reproduces every hand-worked
+    gradient to 1e-12."""
+    import oracle.backward as ob
+    saved = ob._head_bwd
+    ob._head_bwd = bwd
+    try:
+        for c in _hand_worked_cases().values():
+            got = ob.attention_bwd_f64(c["q"], c["k"], c["v"], c["do"], c["causal"], 0.5)
+            for g, want in zip(got, (c["dq"], c["dk"], c["dv"])):
+                if g.shape != want.shape or not np.allclose(g, want, rtol=0, atol=1e-12):
+                    return False
+    finally:
+        ob._head_bwd = saved
+    return True
+
+
+def test_hand_worked_gradients():
+    import oracle.backward as ob
+    assert _hand_worked_matches(ob._head_bwd)
+
+
 def _fd_matches(bwd, causal):
     """True if `bwd` (a replacement for the per-head gradient) agrees with finite
     differences of the forward oracle on a small problem."""
@@ -136,7 +194,8 @@ def _fd_matches(bwd, causal):
 
 
 def test_mutants_fail_the_finite_difference_pin():
-    """Plausible mistakes in the gradient formulas are caught by the pin above."""
+    """Plausible mistakes in the gradient formulas are caught by the finite-difference pin
+    and by the hand-worked one."""
     import oracle.backward as ob
     right = ob._head_bwd
 
@@ -155,6 +214,7 @@ def test_mutants_fail_the_finite_difference_pin():
         dQ, dK, dV = right(Q, K, V, dO, vis, scale)
         return dQ, np.flipud(dK), dV
 
-    assert _fd_matches(right, True)
+    assert _fd_matches(right, True) and _hand_worked_matches(right)
     for bad in (drop_d, no_scale_dq, misindexed_dk):
         assert not _fd_matches(bad, True), bad.__name__
+        assert not _hand_worked_matches(bad), bad.__name__
