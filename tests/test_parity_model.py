@@ -24,7 +24,11 @@ The rounding points emulated:
   dS = P * (dP - D) rounded to 16 bits as the operand of dQ and dK; each gradient rounded
   to 16 bits at the end (a KV head's dK, dV summed over its query heads first);
 * E4M3: P = 2^(log2(e) * (s - m) + 4) (the kernel's offset keeps P normal), rounded to
-  E4M3 as the operand of P.V; the row sum from P before rounding; O rounded to bf16.
+  E4M3 as the operand of P.V; the row sum from P before rounding; O rounded to bf16;
+* 16-bit forward: P rounded to 16 bits as the operand of P.V, the row sum from P before
+  rounding, O rounded to 16 bits. Its tolerances are fixed numbers, not a model; the
+  emulated errors must stay inside them with room to spare (max-abs at most 3/4 of the
+  bound), so that a kernel with these roundings passes for a reason, not by luck.
 """
 import math
 
@@ -32,8 +36,9 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import attention_bwd_f64, attention_fp8_f64, e4m3_to_f64, visible_mask
-from tests.parity import assert_close_bwd, assert_close_fp8, bwd_head_terms, fp8_sigma, to_f64
+from oracle import attention_bwd_f64, attention_f64, attention_fp8_f64, e4m3_to_f64, visible_mask
+from tests.parity import (LSE_REL, MAX_ABS, RMS_TOL, assert_close_bwd, assert_close_fp8,
+                          bwd_head_terms, fp8_sigma, metrics, to_f64)
 from workloads import make_fp8_inputs, make_fwd_inputs
 
 TIGHT = (0.5, 0.9)
@@ -141,3 +146,27 @@ def test_fp8_model_accepts_and_is_tight(causal):
                              f"fp8 h{h}")
         ratio = s["rms"] / s["rms_sigma"]
         assert TIGHT_FP8[0] <= ratio <= TIGHT_FP8[1], s
+
+
+def emulate_fwd_head(Q, K, V, vis, scale, dtype):
+    """O (16-bit-rounded) and LSE of one head with the 16-bit kernel's roundings."""
+    S = np.where(vis, scale * (Q @ K.T), -np.inf)
+    m = S.max(axis=1)
+    E = np.exp(S - m[:, None])
+    l = E.sum(axis=1)
+    return r16((r16(E, dtype) @ V) / l[:, None], dtype), m + np.log(l)
+
+
+@pytest.mark.parametrize("d,dtype", [(64, "fp16"), (128, "bf16")])
+@pytest.mark.parametrize("causal", [False, True])
+def test_forward_roundings_fit_the_fixed_tolerances(d, dtype, causal):
+    N = 2048
+    q, k, v = make_fwd_inputs(1, 1, 1, N, N, d, dtype, seed=d + 2 * causal)
+    q, k, v = to_f64(q), to_f64(k), to_f64(v)
+    scale = 1.0 / math.sqrt(d)
+    O, L = attention_f64(q, k, v, causal, scale)
+    got, lse = emulate_fwd_head(q[0, 0], k[0, 0], v[0, 0], visible_mask(np.arange(N), N, N, causal),
+                                scale, dtype)
+    m = metrics(got, lse, O[0, 0], L[0, 0])
+    assert m["max_abs"] <= 0.75 * MAX_ABS[dtype], m
+    assert m["rms"] <= 0.5 * RMS_TOL and m["lse_rel"] <= 0.01 * LSE_REL, m
