@@ -28,7 +28,11 @@ The rounding points emulated:
 * 16-bit forward: P rounded to 16 bits as the operand of P.V, the row sum from P before
   rounding, O rounded to 16 bits. Its tolerances are fixed numbers, not a model; the
   emulated errors must stay inside them with room to spare (max-abs at most 3/4 of the
-  bound), so that a kernel with these roundings passes for a reason, not by luck.
+  bound), so that a kernel with these roundings passes for a reason, not by luck;
+* decode: per split of 1024 keys (d = 128, tensor cores) P rounded to 16 bits as the P.V
+  operand and the split's row sum from P before rounding; the fp32 partials merged by
+  their LSEs; O rounded to 16 bits. At d = 64 (CUDA cores) P stays fp32 and only O is
+  rounded. Same fixed tolerances, same room.
 """
 import math
 
@@ -36,10 +40,11 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import attention_bwd_f64, attention_f64, attention_fp8_f64, e4m3_to_f64, visible_mask
+from oracle import (attention_bwd_f64, attention_f64, attention_fp8_f64, decode_f64, e4m3_to_f64,
+                    visible_mask)
 from tests.parity import (LSE_REL, MAX_ABS, RMS_TOL, assert_close_bwd, assert_close_fp8,
                           bwd_head_terms, fp8_sigma, metrics, to_f64)
-from workloads import make_fp8_inputs, make_fwd_inputs
+from workloads import make_decode_inputs, make_fp8_inputs, make_fwd_inputs
 
 TIGHT = (0.5, 0.9)
 TIGHT_FP8 = (0.4, 0.9)
@@ -168,5 +173,37 @@ def test_forward_roundings_fit_the_fixed_tolerances(d, dtype, causal):
     got, lse = emulate_fwd_head(q[0, 0], k[0, 0], v[0, 0], visible_mask(np.arange(N), N, N, causal),
                                 scale, dtype)
     m = metrics(got, lse, O[0, 0], L[0, 0])
+    assert m["max_abs"] <= 0.75 * MAX_ABS[dtype], m
+    assert m["rms"] <= 0.5 * RMS_TOL and m["lse_rel"] <= 0.01 * LSE_REL, m
+
+
+def emulate_decode_head(q, K, V, split, round_p, dtype):
+    """O (16-bit-rounded) and LSE of one decode row: splits of `split` keys, each with its
+    own maximum (P rounded to 16 bits when round_p), merged by the splits' LSEs."""
+    parts = []
+    for s0 in range(0, K.shape[0], split):
+        sc = (K[s0:s0 + split] @ q)
+        m = sc.max()
+        e = np.exp(sc - m)
+        pv = (r16(e, dtype) if round_p else e) @ V[s0:s0 + split]
+        parts.append((pv / e.sum(), m + np.log(e.sum())))
+    lse = np.logaddexp.reduce([l for _, l in parts])
+    return r16(sum(np.exp(l - lse) * o for o, l in parts), dtype), lse
+
+
+@pytest.mark.parametrize("d,dtype,round_p", [(128, "bf16", True), (64, "fp16", False)])
+def test_decode_roundings_fit_the_fixed_tolerances(d, dtype, round_p):
+    lens, q, kc, vc = make_decode_inputs(4, 32, 8, 4096, d, dtype, 512, 4096, seed=d)
+    q, kc, vc = to_f64(q), to_f64(kc), to_f64(vc)
+    scale = 1.0 / math.sqrt(d)
+    O, L = decode_f64(q, kc, vc, lens, scale)
+    got = np.zeros_like(O)
+    lse = np.zeros_like(L)
+    for b in range(4):
+        n = int(lens[b])
+        for h in range(32):
+            got[b, h], lse[b, h] = emulate_decode_head(scale * q[b, h], kc[b, h // 4, :n],
+                                                       vc[b, h // 4, :n], 1024, round_p, dtype)
+    m = metrics(got, lse, O, L)
     assert m["max_abs"] <= 0.75 * MAX_ABS[dtype], m
     assert m["rms"] <= 0.5 * RMS_TOL and m["lse_rel"] <= 0.01 * LSE_REL, m
