@@ -736,20 +736,25 @@ def main():
                                        "fwd_fp8", "fwd_varlen"],
                     default=None,
                     help="launch one entry point alone (profiling helper; prints its own line)")
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mha2k", choices=[k for k, v in WORKLOADS.items() if v.kind == "fwd"])
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="ranks of the job (one per GPU, launched by torchrun when > 1)")
+    ap.add_argument("--steps", type=int, default=50, help="timed steps")
+    ap.add_argument("--warmup", type=int, default=10, help="untimed warm-up steps (at least 3)")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours",
+                    help="reference: time the float64 CPU oracle on the headline workload")
+    ap.add_argument("--workload", default="mha2k", choices=[k for k, v in WORKLOADS.items() if v.kind == "fwd"],
+                    help="--only: the prefill workload")
     ap.add_argument("--chunk", type=int, default=1024, help="--only chunked: tokens per chunk")
     ap.add_argument("--page-size", type=int, default=64, help="--only *_paged: tokens per page")
     ap.add_argument("--varlen-lens", default="8192,6144,3072,1024",
                     help="--only fwd_varlen: comma-separated sequence lengths of the batch")
-    ap.add_argument("--decode-workload", default="decode")
-    ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--decode-workload", default="decode", help="--only decode*: the decode workload")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end run from pinned host buffers")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle timing")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0,
+                    help="host seconds the CPU oracle timing may take in all")
+    ap.add_argument("--e2e-steps", type=int, default=20, help="steps of the end-to-end run")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
     if args.impl == "reference":
