@@ -11,7 +11,8 @@ import numpy as np
 from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
 
-from oracle import attention_f64, decode_f64, split_kv_decode_f64, tiled_attention_f64
+from oracle import (attention_f64, attention_rows_f64, decode_f64, split_kv_decode_f64,
+                    tiled_attention_f64)
 
 SETTINGS = settings(derandomize=True, max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
 ATOL = 1e-11
@@ -173,3 +174,17 @@ def test_split_kv_decode_merge_is_exact(n, d, seed, scale, cuts):
     O, L = split_kv_decode_f64(q[0, 0], k[0, 0, :n], v[0, 0, :n], bounds, scale)
     Od, Ld = decode_f64(q, k, v, [n], scale)
     assert close(O, Od[0, 0]) and close(np.array(L), Ld[0, 0])
+
+
+@SETTINGS
+@given(shapes(), st.booleans(), st.data())
+def test_sampled_rows_equal_the_full_result(s, causal, data):
+    """The sampled-rows form (used on the largest workloads) gives exactly the full
+    result's rows, for any subset in any order, repeats included, under either mask."""
+    q, k, v, _ = make(s)
+    O, L = attention_f64(q, k, v, causal, s["scale"])
+    rows = np.array(data.draw(st.lists(st.integers(0, s["Nq"] - 1), min_size=1, max_size=12)))
+    b = data.draw(st.integers(0, s["B"] - 1))
+    h = data.draw(st.integers(0, s["Hq"] - 1))
+    Or, Lr = attention_rows_f64(q, k, v, causal, s["scale"], b, h, rows)
+    assert close(Or, O[b, h, rows]) and close(Lr, L[b, h, rows])
