@@ -7,7 +7,9 @@ counting by brute force:
 * the K and V bytes a decode step must read;
 * the per-launch timing spread (linear-interpolated percentiles);
 * the DRAM traffic taken from the committed ncu captures, which counts only while the
-  hash of the kernel sources it was taken on still matches.
+  hash of the kernel sources it was taken on still matches;
+* the clock record (median SM clock, named throttle reasons) read from NVML, here a
+  read-only stand-in.
 """
 import hashlib
 import json
@@ -103,3 +105,60 @@ def test_measured_traffic_follows_the_source_hash():
 def test_job_rate_is_whole_job_work_over_the_slowest_rank():
     assert bench.job_rate(4, 20, 1.5, 10.0) == pytest.approx(4 * 20 * 1.5 / 0.010)
     assert math.isclose(bench.job_rate(1, 1, 1.0, 1000.0), 1.0)
+
+
+class _FakeNvml:
+    """Read-only NVML stand-in: a fixed clock sequence and throttle-reason bitmask."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self, clocks, reasons):
+        self.clocks, self.reasons, self.i = list(clocks), reasons, 0
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetHandleByUUID(self, u):
+        raise RuntimeError("no uuid")
+
+    def nvmlDeviceGetHandleByIndex(self, idx):
+        return ("handle", idx)
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        c = self.clocks[min(self.i, len(self.clocks) - 1)]
+        self.i += 1
+        return c
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.reasons
+
+
+def test_clock_sampler_reports_median_and_named_reasons(monkeypatch):
+    fake = _FakeNvml([1700, 1755, 1740, 1965, 1725], 0x1 | 0x4 | 0x8)
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    cs = bench.ClockSampler(0, period_s=0.001)
+    assert cs.nvml is fake and cs.max_mhz == 1965
+    cs.start()
+    import time
+    t0 = time.monotonic()
+    while len(cs.samples) < 5 and time.monotonic() - t0 < 2.0:
+        time.sleep(0.005)
+    cs.stop()
+    s = cs.summary()
+    assert s["samples"] >= 5 and s["sm_max_mhz"] == 1965
+    assert s["sm_mhz"] == float(np.median([fake.clocks[min(i, 4)] for i in range(s["samples"])]))
+    assert s["reasons"] == ["sw_power_cap", "hw_slowdown"]      # gpu_idle is not reported
+
+
+def test_clock_sampler_without_nvml_reports_no_samples(monkeypatch):
+    class Broken:
+        def nvmlInit(self):
+            raise RuntimeError("NVML not found")
+    monkeypatch.setitem(sys.modules, "pynvml", Broken())
+    cs = bench.ClockSampler(0)
+    cs.start()
+    cs.stop()
+    s = cs.summary()
+    assert s["samples"] == 0 and s["sm_mhz"] is None and "NVML not found" in s["note"]
