@@ -92,3 +92,41 @@ def test_mutant_is_caught(name):
         except Exception as e:
             failed.append((pin.__name__, type(e).__name__))
     assert failed, f"mutant {name!r} passed every pin"
+
+
+# ---- descale identities (hypothesis) -------------------------------------------------
+from hypothesis import HealthCheck, given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+SETTINGS = settings(derandomize=True, max_examples=40, deadline=None,
+                    suppress_health_check=[HealthCheck.too_slow])
+
+
+def _codes(rng, shape):
+    """Random finite E4M3 codes (the two NaN codes excluded)."""
+    c = rng.integers(0, 256, size=shape, dtype=np.uint8)
+    return np.where((c & 0x7F) == 0x7F, c & 0xF0, c).astype(np.uint8)
+
+
+@SETTINGS
+@given(st.integers(0, 2**31 - 1), st.booleans(), st.floats(2.0 ** -8, 2.0 ** -2),
+       st.floats(2.0 ** -8, 2.0 ** -2), st.floats(1e-3, 10.0), st.floats(0.25, 4.0))
+def test_descales_fold_as_the_definition_says(seed, causal, dq, dk, dv, alpha):
+    """Q and K descales multiply the scores (so they fold into the scale), V's descale
+    multiplies O and leaves the LSE alone."""
+    rng = np.random.default_rng(seed)
+    Hkv = int(rng.integers(1, 3))
+    Hq = Hkv * int(rng.integers(1, 3))
+    Nq, Nk = int(rng.integers(1, 12)), int(rng.integers(1, 12))
+    q8, k8, v8 = _codes(rng, (1, Hq, Nq, 8)), _codes(rng, (1, Hkv, Nk, 8)), _codes(rng, (1, Hkv, Nk, 8))
+    s = 0.3
+    O, L = attention_fp8_f64(q8, k8, v8, dq, dk, dv, causal, s)
+    O2, L2 = attention_fp8_f64(q8, k8, v8, dq * alpha, dk, dv, causal, s / alpha)
+    O3, L3 = attention_fp8_f64(q8, k8, v8, dq, dk * alpha, dv, causal, s / alpha)
+    O4, L4 = attention_fp8_f64(q8, k8, v8, dq, dk, dv * alpha, causal, s)
+    fin = np.isfinite(L)
+    for Ox, Lx in ((O2, L2), (O3, L3)):
+        assert np.allclose(Ox, O, rtol=1e-9, atol=1e-9 * max(1.0, float(np.abs(O).max())))
+        assert np.array_equal(np.isfinite(Lx), fin) and np.allclose(Lx[fin], L[fin], rtol=1e-9, atol=1e-9)
+    assert np.allclose(O4, alpha * O, rtol=1e-12, atol=0)
+    assert np.array_equal(np.isfinite(L4), fin) and np.allclose(L4[fin], L[fin], rtol=0, atol=0)
