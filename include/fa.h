@@ -141,6 +141,10 @@ FA_API fa_status fa_fwd_kvcache(const void* q, const void* kcache, const void* v
  * fa_fwd_paged — fa_fwd_kvcache with the keys and values in a paged pool: each of the B
  * sequences attends to its first nk_b tokens, found through its block-table row.
  *
+ * Defined by: the per-session cache of page "Flash Attention ... IO-aware exact" (fr),
+ * "Optimisation avancée : KV Cache et persistent attention", laid out as the paged pool
+ * above; the attention itself is fa_fwd_kvcache's.
+ *
  *   q, o, lse         as fa_fwd, [B, Hq, Nq, d] / [B, Hq, Nq]: Nq is the row capacity
  *   q_lens, kv_lens   as fa_fwd_kvcache (NULL: Nq rows and Nk keys for every sequence;
  *                     otherwise per-sequence values clamped to [0, Nq] and [0, Nk])
@@ -183,6 +187,10 @@ FA_API fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o
 
 /*
  * fa_bwd_workspace_bytes — bytes of scratch that fa_bwd needs for these sizes.
+ *
+ * Not an operation of the pages: a size query for fa_bwd's per-row scratch (the LSE in
+ * log2 units and D_i = sum_d dO_id O_id, one fp32 each per padded query row). Pure host
+ * arithmetic; returns 0 for invalid sizes.
  */
 FA_API size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq);
 
@@ -215,6 +223,9 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
 
 /*
  * fa_decode_workspace_bytes — bytes of scratch that fa_decode needs for these sizes.
+ *
+ * Not an operation of the pages: a size query (pure host arithmetic) for fa_decode's
+ * split-KV scratch.
  *
  * The split-KV decode writes, per (sequence, query head, KV split), a partial output
  * row (d fp32) and its logsumexp (fp32), then merges them. max_kv_len is the cache
@@ -259,6 +270,10 @@ FA_API fa_status fa_decode(const void* q, const void* kcache, const void* vcache
 /*
  * fa_decode_paged — fa_decode over a paged pool (see "Paged KV cache" above): sequence b
  * attends to its first kv_lens[b] tokens, found through its block-table row.
+ *
+ * Defined by: the per-session cache of page "Flash Attention ... IO-aware exact" (fr),
+ * "Optimisation avancée : KV Cache et persistent attention", laid out as the paged pool
+ * above; the decode itself is fa_decode's.
  *
  *   q, o, lse, kv_lens   as fa_decode; kv_lens are clamped to
  *                        [0, max_pages_per_seq * page_size]
@@ -308,10 +323,13 @@ FA_API fa_status fa_decode_noalloc(const void* q, const void* kcache, const void
                                    int B, int Hq, int Hkv, int max_kv_len, int d,
                                    float scale, fa_dtype dtype, void* stream);
 
-/* fa_status_string — static, human-readable name of a status code (never NULL). */
+/* fa_status_string — static, human-readable name of a status code (never NULL). Not an
+ * operation of the pages: error reporting. */
 FA_API const char* fa_status_string(fa_status s);
 
 /*
+ * Not operations of the pages: error reporting and the test hooks of the bounded waits.
+ *
  * fa_device_status — synchronises the current device, then returns FA_OK or the first
  * error a kernel of this library recorded on it (FA_ERR_DEVICE_TIMEOUT, or
  * FA_ERR_INVALID_ARG for a paged-cache table entry outside the pool). If `clear` is
@@ -321,6 +339,8 @@ FA_API const char* fa_status_string(fa_status s);
 FA_API fa_status fa_device_status(int clear);
 
 /*
+ * Not an operation of the pages.
+ *
  * fa_set_wait_timeout_ns — upper bound, in nanoseconds, on every device-side barrier wait
  * of kernels launched afterwards from this process (default 2e9, i.e. 2 s). 0 restores
  * the default. Test hook for the timeout path; normal callers never need it.
@@ -328,6 +348,8 @@ FA_API fa_status fa_device_status(int clear);
 FA_API void fa_set_wait_timeout_ns(uint64_t ns);
 
 /*
+ * Not an operation of the pages.
+ *
  * fa_debug_skip_q_load — test hook for the bounded-wait path: when non-zero, fa_fwd
  * kernels launched afterwards never issue the Q-tile load, the d = 128 decode kernels
  * never load their query rows, the other decode kernels never fill their K/V stages, and
@@ -339,7 +361,8 @@ FA_API void fa_set_wait_timeout_ns(uint64_t ns);
  */
 FA_API void fa_debug_skip_q_load(int enable);
 
-/* fa_build_info — static string: library version and the GPU architecture it targets. */
+/* fa_build_info — static string: library version and the GPU architecture it targets.
+ * Not an operation of the pages. */
 FA_API const char* fa_build_info(void);
 
 #ifdef __cplusplus

@@ -171,3 +171,23 @@ def test_fwd_fp8_rejects_bad_arguments_without_cuda():
     assert call(dk=-1.0) == fa.FA_ERR_INVALID_ARG
     assert call(d=64) == fa.FA_ERR_UNSUPPORTED        # d = 128 only
     assert call(v=40) == fa.FA_ERR_ALIGNMENT
+
+
+def test_every_declaration_states_its_source():
+    """Each FA_API declaration sits under a comment block that cites the page passage
+    defining the operation, or says it is not an operation of the pages."""
+    import re
+    with open(os.path.join(ROOT, "include", "fa.h"), encoding="utf-8") as f:
+        src = f.read()
+    names = []
+    for m in re.finditer(r"FA_API\s+[^;]*?\b(fa_\w+)\s*\(", src):
+        before = src[:m.start()]
+        block = before[before.rfind("/*"):]
+        assert "*/" in block, m.group(1)
+        block = re.sub(r"\s*\n\s*\*(?!/)\s*", " ", block)     # one line, no leading stars
+        low = block.lower()
+        assert 'page "' in block or "not an operation of the pages" in low or \
+            "not operations of the pages" in low or "not from the pages" in low or \
+            "not on the pages" in low, m.group(1)
+        names.append(m.group(1))
+    assert len(names) >= 15
