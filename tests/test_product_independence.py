@@ -130,3 +130,23 @@ def test_entry_points_reach_the_oracle_only_from_their_checking_legs():
     assert set(entry) == {"smoke"}, entry
     bench = _oracle_imports_by_function(os.path.join(ROOT, "bench.py"))
     assert bench and set(bench) <= {"oracle_rows_time", "oracle_baselines"}, bench
+
+
+def test_bench_without_a_gpu_fails_instead_of_reporting():
+    """On a machine without a GPU the benchmark's own arm exits non-zero and prints no
+    result line: there is no CPU path that could stand in for the kernels."""
+    import json
+    import pytest
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; this checks the GPU-less case")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "1",
+                        "--warmup", "3", "--no-cpu-baseline", "--no-e2e"],
+                       capture_output=True, text=True, cwd=ROOT, timeout=300)
+    assert r.returncode != 0
+    for line in r.stdout.splitlines():
+        try:
+            obj = json.loads(line)
+        except ValueError:
+            continue
+        assert "value" not in obj, line
