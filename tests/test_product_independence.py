@@ -150,3 +150,12 @@ def test_bench_without_a_gpu_fails_instead_of_reporting():
         except ValueError:
             continue
         assert "value" not in obj, line
+
+
+def test_every_oracle_module_says_it_is_test_infrastructure():
+    files = list(_files(os.path.join(ROOT, "oracle"), (".py",)))
+    assert files
+    for p in files:
+        with open(p, encoding="utf-8") as f:
+            doc = ast.get_docstring(ast.parse(f.read())) or ""
+        assert "TEST INFRASTRUCTURE ONLY" in doc, p
